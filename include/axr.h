@@ -1,0 +1,129 @@
+/*
+ * axr.h -- C ABI of libaxr: AXELRAM-style quantize-on-write and LUT score-on-read
+ * for the key cache of attention, on NVIDIA B200 (sm_100a).
+ *
+ * Method: "AXELRAM: Quantize Once, Never Dequantize" (arXiv 2604.02638), abstract.
+ * Keys are rotated by a sign-flipped orthonormal Walsh-Hadamard transform, which
+ * makes every coordinate of a unit key close to N(0, 1/d); each coordinate is then
+ * scalar-quantized to a codebook fixed at design time by d and b alone.  Scores
+ * are read straight from the stored indices through lookup tables built from the
+ * once-rotated query; the keys are never dequantized or rotated back.
+ *
+ * Conventions shared by every entry point
+ *   - All buffers are owned by the caller.  The library never allocates device
+ *     memory; it keeps only a host-side, thread-safe cache of codebooks.
+ *   - Device-pointer arguments must be device (or managed) memory of the current
+ *     device.  Calls enqueue work on `stream` and return without synchronising;
+ *     results are valid once the stream has reached that point.
+ *   - Argument errors are detected on the host before any launch and return
+ *     AXR_EINVAL / AXR_EUNSUPPORTED with nothing enqueued.  A failed launch
+ *     returns AXR_ECUDA.  axr_last_error() gives a message for the calling thread.
+ *   - n == 0 is a no-op that returns AXR_OK.
+ *   - Inputs must be finite, with squared key norms inside the fp32 range.
+ *   - The sign pattern `signs` is an int8 device vector of length d with entries
+ *     +1 or -1 (any negative entry counts as -1, anything else as +1).  One
+ *     pattern serves a whole layer: keys and queries of that layer must use the
+ *     same one (AXELRAM abstract: the transform's sign pattern, chosen once).
+ *   - Supported shapes: d a power of two in [8, 512]; b in {1, 2, 3, 4};
+ *     group in [1, 8].
+ *
+ * Packed index layout (one row per key, P = d*b/8 bytes, rows back to back):
+ *   bit i of idx_j is bit (j*b + i) of the row's bit stream, and byte k of the
+ *   row holds stream bits 8k .. 8k+7, least significant first.  idx 0 is the most
+ *   negative centroid.  (The pages only say the indices are stored; this dense
+ *   little-endian layout is this library's choice.)
+ */
+#ifndef AXR_H
+#define AXR_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum axr_status {
+    AXR_OK = 0,
+    AXR_EINVAL = -1,        /* null/misaligned pointer, negative size, bad dtype   */
+    AXR_EUNSUPPORTED = -2,  /* d, b or group outside the supported set            */
+    AXR_ECUDA = -3          /* a CUDA call failed; see axr_last_error()           */
+} axr_status;
+
+typedef enum axr_dtype {
+    AXR_F32 = 0,
+    AXR_F16 = 1,
+    AXR_BF16 = 2
+} axr_dtype;
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *axr_stream;
+
+/*
+ * Design-time codebook (AXELRAM abstract: the optimal scalar quantizer of a
+ * rotated coordinate depends on d and b only, never on the data; the paper's
+ * repository lists a Lloyd-Max solver for it).
+ *
+ * Host only.  Fills caller-owned HOST arrays:
+ *   centroids[2^b]   Lloyd-Max centroids of N(0, 1/d), ascending, fp32,
+ *                    exactly symmetric (c[L-1-i] == -c[i]);
+ *   boundaries[2^b-1] fp32 of the midpoint of neighbouring centroids
+ *                    (may be NULL if not wanted).
+ * Returns AXR_OK, AXR_EINVAL (centroids NULL) or AXR_EUNSUPPORTED (d, b).
+ */
+int axr_make_codebook(int d, int b, float *centroids, float *boundaries);
+
+/*
+ * Quantize-on-write (AXELRAM abstract: keys are transformed once, on write).
+ * For every key row k (length d):
+ *   norm = ||k||_2 (fp32 accumulation), stored;
+ *   y = H * diag(signs) * k, H the Sylvester-ordered Walsh-Hadamard matrix;
+ *   u = y / (sqrt(d) * norm)          (the unit key in the rotated basis);
+ *   idx_j = number of codebook boundaries t_i with u_j > t_i
+ *           (= nearest centroid, ties to the lower index);
+ *   the d indices are bit-packed into P = d*b/8 bytes (layout above).
+ * A key of norm 0 stores norm 0 and idx_j = 2^(b-1) - 1 for every j.
+ *
+ * K      device, n x d row-major, element type kdtype; 16-byte aligned.
+ * signs  device int8[d].
+ * idx    device uint8[n * P] output; 16-byte aligned.
+ * norms  device float[n] output; 4-byte aligned.
+ */
+int axr_quantize_keys(const void *K, int kdtype, int64_t n, int d, int b,
+                      const int8_t *signs, uint8_t *idx, float *norms,
+                      axr_stream stream);
+
+/*
+ * Score-on-read (AXELRAM abstract: table lookup on read, no inverse transform).
+ * Each query is rotated once, q' = H * diag(signs) * q / sqrt(d); then for every
+ * stored key t of its KV head
+ *   scores[t] = norms[t] * sum_j q'_j * c[idx_t[j]] / sqrt(d)
+ * where the last 1/sqrt(d) is the attention temperature.  The keys are never
+ * dequantized.  Grouped-query attention: query head h*group + g reads KV head h,
+ * so one index stream serves all `group` queries of a KV head.  A batch is
+ * folded into `heads` (heads = batch * KV heads).
+ *
+ * q       device, (heads*group) x d row-major, element type qdtype; 16-byte aligned.
+ * idx     device, heads x n x P bytes (as written by axr_quantize_keys); 16-byte aligned.
+ * norms   device float[heads * n].
+ * signs   device int8[d], the pattern the keys were written with.
+ * scores  device float[(heads*group) * n] output, row h*group+g holds the n
+ *         scores of that query head.
+ */
+int axr_scores(const void *q, int qdtype, const uint8_t *idx, const float *norms,
+               int64_t n, int heads, int group, int d, int b, const int8_t *signs,
+               float *scores, axr_stream stream);
+
+/* Static string naming a status code. */
+const char *axr_status_string(int status);
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char *axr_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int axr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AXR_H */

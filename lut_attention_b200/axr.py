@@ -1,0 +1,154 @@
+"""Python binding of libaxr (the C ABI in include/axr.h): argument marshalling only.
+
+Every computation runs in libaxr's CUDA kernels.  This module checks tensor
+shapes, allocates outputs when the caller gives none, passes raw device
+pointers and the current CUDA stream, and turns status codes into exceptions.
+There is no CPU path: without the built library or a CUDA device the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libaxr.so")
+
+AXR_OK, AXR_EINVAL, AXR_EUNSUPPORTED, AXR_ECUDA = 0, -1, -2, -3
+AXR_F32, AXR_F16, AXR_BF16 = 0, 1, 2
+_DTYPE_CODE = {torch.float32: AXR_F32, torch.float16: AXR_F16, torch.bfloat16: AXR_BF16}
+
+# every symbol include/axr.h declares, with its ctypes signature
+_P, _I32, _I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+SIGNATURES = {
+    "axr_make_codebook": (_I32, [_I32, _I32, _P, _P]),
+    "axr_quantize_keys": (_I32, [_P, _I32, _I64, _I32, _I32, _P, _P, _P, _P]),
+    "axr_scores": (_I32, [_P, _I32, _P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
+    "axr_status_string": (ctypes.c_char_p, [_I32]),
+    "axr_last_error": (ctypes.c_char_p, []),
+    "axr_version": (_I32, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AxrError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: status {status} ({detail})")
+        self.status = status
+
+
+def library() -> ctypes.CDLL:
+    """Load libaxr.so (built in-tree by ``python -m lut_attention_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"libaxr.so is missing at {LIB_PATH}: build it with "
+                    "`python -m lut_attention_b200.build` (needs nvcc)")
+            lib = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+        return _lib
+
+
+def _raise(rc: int, where: str) -> None:
+    if rc != AXR_OK:
+        lib = library()
+        detail = lib.axr_last_error().decode() or lib.axr_status_string(rc).decode()
+        raise AxrError(rc, where, detail)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _require_cuda(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libaxr has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def axr_make_codebook(d: int, b: int) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 centroids (2^b, ascending) and boundaries (2^b - 1) for (d, b)."""
+    L = 1 << b if 0 < b < 31 else 1
+    cent = np.zeros(max(L, 1), dtype=np.float32)
+    bnd = np.zeros(max(L - 1, 1), dtype=np.float32)
+    rc = library().axr_make_codebook(d, b, cent.ctypes.data_as(_P), bnd.ctypes.data_as(_P))
+    _raise(rc, "axr_make_codebook")
+    return cent[:L], bnd[:L - 1]
+
+
+def packed_row_bytes(d: int, b: int) -> int:
+    return d * b // 8
+
+
+def axr_quantize_keys(K: torch.Tensor, b: int, signs: torch.Tensor,
+                      idx: torch.Tensor | None = None, norms: torch.Tensor | None = None,
+                      stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Quantize-on-write of keys K (..., d) -> (idx (..., d*b/8) uint8, norms (...) fp32)."""
+    _require_cuda(K, "K")
+    _require_cuda(signs, "signs")
+    if K.dtype not in _DTYPE_CODE:
+        raise ValueError(f"K dtype {K.dtype} not supported")
+    if signs.dtype != torch.int8:
+        raise ValueError("signs must be int8")
+    d = K.shape[-1]
+    lead = K.shape[:-1]
+    n = K.numel() // d if d else 0
+    P = packed_row_bytes(d, b)
+    if idx is None:
+        idx = torch.empty(lead + (P,), dtype=torch.uint8, device=K.device)
+    if norms is None:
+        norms = torch.empty(lead, dtype=torch.float32, device=K.device)
+    _require_cuda(idx, "idx")
+    _require_cuda(norms, "norms")
+    if idx.numel() < n * P or norms.numel() < n:
+        raise ValueError("idx/norms too small")
+    rc = library().axr_quantize_keys(K.data_ptr(), _DTYPE_CODE[K.dtype], n, d, b, signs.data_ptr(),
+                                     idx.data_ptr(), norms.data_ptr(), _stream_handle(stream))
+    _raise(rc, "axr_quantize_keys")
+    return idx, norms
+
+
+def axr_scores(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, group: int, b: int,
+               signs: torch.Tensor, scores: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """LUT scores (heads*group, n) fp32 of queries q (heads*group, d) against packed
+    keys idx (heads, n, d*b/8) with norms (heads, n)."""
+    for t, name in ((q, "q"), (idx, "idx"), (norms, "norms"), (signs, "signs")):
+        _require_cuda(t, name)
+    if q.dtype not in _DTYPE_CODE:
+        raise ValueError(f"q dtype {q.dtype} not supported")
+    if idx.dtype != torch.uint8 or norms.dtype != torch.float32 or signs.dtype != torch.int8:
+        raise ValueError("idx must be uint8, norms float32, signs int8")
+    hg, d = q.shape
+    if group < 1 or hg % group:
+        raise ValueError("q must have heads*group rows")
+    heads = hg // group
+    if idx.dim() != 3 or idx.shape[0] != heads or idx.shape[2] != packed_row_bytes(d, b):
+        raise ValueError(f"idx must be (heads={heads}, n, {packed_row_bytes(d, b)})")
+    n = idx.shape[1]
+    if tuple(norms.shape) != (heads, n):
+        raise ValueError(f"norms must be ({heads}, {n})")
+    if scores is None:
+        scores = torch.empty((hg, n), dtype=torch.float32, device=q.device)
+    _require_cuda(scores, "scores")
+    if scores.numel() < hg * n or scores.dtype != torch.float32:
+        raise ValueError("scores must be float32 with (heads*group)*n elements")
+    rc = library().axr_scores(q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), n,
+                              heads, group, d, b, signs.data_ptr(), scores.data_ptr(),
+                              _stream_handle(stream))
+    _raise(rc, "axr_scores")
+    return scores

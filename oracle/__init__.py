@@ -1,0 +1,195 @@
+"""CPU oracle for the AXELRAM write and read path: test infrastructure.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never uses it, and it
+imports nothing from the library.  The arithmetic lives in ``oracle.c`` (plain
+C, fp64); this module compiles it with gcc and marshals numpy arrays into it.
+
+Every function takes and returns numpy arrays on the host.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, -O2, no fast-math)."""
+    up_to_date = (
+        os.path.exists(_LIB_PATH)
+        and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)
+    )
+    if force or not up_to_date:
+        tmp = f"{_LIB_PATH}.{os.getpid()}.tmp"
+        subprocess.check_call(
+            ["gcc", "-std=c11", "-O2", "-Wall", "-Wextra", "-shared", "-fPIC",
+             "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64 = ctypes.c_int, ctypes.c_int64
+        sig = {
+            "oracle_hadamard": [i32, P],
+            "oracle_rotation": [i32, P, P],
+            "oracle_lloyd_max_std": [i32, P, P],
+            "oracle_codebook": [i32, i32, P, P],
+            "oracle_pack": [P, i64, i32, i32, P],
+            "oracle_unpack": [P, i64, i32, i32, P],
+            "oracle_rotate_unit": [P, i64, i32, P, P, P],
+            "oracle_quantize": [P, i64, i32, i32, P, P, P, P],
+            "oracle_scores": [P, P, P, i64, i32, i32, i32, i32, P, P],
+            "oracle_dequant_scores": [P, P, P, i64, i32, i32, i32, i32, P, P],
+        }
+        for name, args in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise ValueError(f"oracle: {what} rejected its arguments (rc={rc})")
+
+
+def _signs(signs, d: int) -> np.ndarray:
+    s = np.ascontiguousarray(np.asarray(signs), dtype=np.int8).reshape(-1)
+    if s.shape[0] != d:
+        raise ValueError(f"signs must have {d} entries, got {s.shape[0]}")
+    return s
+
+
+def hadamard(d: int) -> np.ndarray:
+    """Sylvester-ordered Walsh-Hadamard matrix, entries +-1, shape (d, d)."""
+    H = np.empty((d, d), dtype=np.float64)
+    _check(_load().oracle_hadamard(d, _ptr(H)), "hadamard")
+    return H
+
+
+def rotation(d: int, signs) -> np.ndarray:
+    """R = H diag(signs) / sqrt(d), shape (d, d)."""
+    R = np.empty((d, d), dtype=np.float64)
+    _check(_load().oracle_rotation(d, _ptr(_signs(signs, d)), _ptr(R)), "rotation")
+    return R
+
+
+def lloyd_max_std(b: int) -> tuple[np.ndarray, int]:
+    """Lloyd-Max centroids of N(0,1), 2^b levels ascending (fp64), and iteration count."""
+    c = np.empty(1 << b, dtype=np.float64)
+    it = ctypes.c_int(0)
+    _check(_load().oracle_lloyd_max_std(b, _ptr(c), ctypes.byref(it)), "lloyd_max_std")
+    return c, it.value
+
+
+def codebook(d: int, b: int) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 centroids (2^b, ascending) and fp32 decision boundaries (2^b - 1)."""
+    L = 1 << b
+    cent = np.empty(L, dtype=np.float32)
+    bnd = np.empty(L - 1, dtype=np.float32)
+    _check(_load().oracle_codebook(d, b, _ptr(cent), _ptr(bnd)), "codebook")
+    return cent, bnd
+
+
+def pack(codes: np.ndarray, b: int) -> np.ndarray:
+    """(n, d) codes in [0, 2^b) -> (n, d*b/8) bytes, dense LSB-first bit stream."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    n, d = codes.shape
+    out = np.empty((n, d * b // 8), dtype=np.uint8)
+    _check(_load().oracle_pack(_ptr(codes), n, d, b, _ptr(out)), "pack")
+    return out
+
+
+def unpack(packed: np.ndarray, d: int, b: int) -> np.ndarray:
+    """Inverse of :func:`pack`: (..., d*b/8) bytes -> (..., d) codes."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    lead = packed.shape[:-1]
+    n = int(np.prod(lead)) if lead else 1
+    out = np.empty(lead + (d,), dtype=np.uint8)
+    _check(_load().oracle_unpack(_ptr(packed), n, d, b, _ptr(out)), "unpack")
+    return out
+
+
+def rotate_unit(K: np.ndarray, signs) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 norms (n,) and rotated unit keys U = R K / norm (n, d, fp64)."""
+    K = np.ascontiguousarray(K, dtype=np.float64)
+    n, d = K.shape
+    norms = np.empty(n, dtype=np.float32)
+    U = np.empty((n, d), dtype=np.float64)
+    _check(_load().oracle_rotate_unit(_ptr(K), n, d, _ptr(_signs(signs, d)), _ptr(norms), _ptr(U)),
+           "rotate_unit")
+    return norms, U
+
+
+def quantize(K: np.ndarray, b: int, signs, margins: bool = False):
+    """Quantize-on-write of K (n, d).
+
+    Returns ``(packed (n, d*b/8) uint8, norms (n,) fp32, margins)`` where
+    ``margins`` is None unless requested, else (n, d) fp64 distances of every
+    rotated unit coordinate to its nearest decision point.
+    """
+    K = np.ascontiguousarray(K, dtype=np.float64)
+    n, d = K.shape
+    packed = np.empty((n, d * b // 8), dtype=np.uint8)
+    norms = np.empty(n, dtype=np.float32)
+    marg = np.empty((n, d), dtype=np.float64) if margins else None
+    _check(_load().oracle_quantize(_ptr(K), n, d, b, _ptr(_signs(signs, d)), _ptr(packed),
+                                   _ptr(norms), _ptr(marg)), "quantize")
+    return packed, norms, marg
+
+
+def _read_args(q, packed, norms, group, b):
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    hg, d = q.shape
+    if hg % group:
+        raise ValueError("q rows must be heads*group")
+    heads = hg // group
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    norms = np.ascontiguousarray(norms, dtype=np.float32)
+    if packed.ndim != 3 or packed.shape[0] != heads or packed.shape[2] != d * b // 8:
+        raise ValueError(f"packed must be (heads, n, {d * b // 8})")
+    n = packed.shape[1]
+    if norms.shape != (heads, n):
+        raise ValueError("norms must be (heads, n)")
+    return q, packed, norms, heads, n, d
+
+
+def scores(q, packed, norms, group: int, b: int, signs) -> np.ndarray:
+    """LUT scores (heads*group, n), fp64: norm * sum_j (R q)_j c[idx_j] / sqrt(d)."""
+    q, packed, norms, heads, n, d = _read_args(q, packed, norms, group, b)
+    out = np.empty((heads * group, n), dtype=np.float64)
+    _check(_load().oracle_scores(_ptr(q), _ptr(packed), _ptr(norms), n, heads, group, d, b,
+                                 _ptr(_signs(signs, d)), _ptr(out)), "scores")
+    return out
+
+
+def dequant_scores(q, packed, norms, group: int, b: int, signs) -> np.ndarray:
+    """Scores on dequantized, inverse-rotated keys: q . (norm R^T c[idx]) / sqrt(d)."""
+    q, packed, norms, heads, n, d = _read_args(q, packed, norms, group, b)
+    out = np.empty((heads * group, n), dtype=np.float64)
+    _check(_load().oracle_dequant_scores(_ptr(q), _ptr(packed), _ptr(norms), n, heads, group, d,
+                                         b, _ptr(_signs(signs, d)), _ptr(out)), "dequant_scores")
+    return out

@@ -1,0 +1,472 @@
+"""Benchmark of the AXELRAM hot path on B200: quantize-on-write + LUT score-on-read.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl axr|reference]
+                    [--workload gqa_decode_128k] [--b 4]
+
+One step is one pass of the whole path over one batch of the workload: every key
+of the batch is quantized (sign flip, Walsh-Hadamard, norm, Lloyd-Max indices,
+packing) and every query head is scored against every key of its KV head by
+table lookup on the packed indices.  The read kernel scores the cache written one
+step earlier (two cache buffers, same keys), so neither kernel finds the other's
+output in L2; every input is larger than the 126 MB L2.
+
+Multi-GPU: one process per GPU (torchrun).  The batch is sharded: every rank runs
+its own batch of the workload (weak scaling), with no collective on the data
+path; the only collectives are the barrier and the max-over-ranks of the time.
+
+Prints ONE JSON line on rank 0.  ``value`` is LUT attention scores per second for
+the whole job; keys quantized per second and each kernel's HBM throughput are
+reported beside it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from lut_attention_b200 import axr, workloads  # noqa: E402
+
+NOMINAL_HBM_GBS = 8000.0          # B200 HBM3e nominal figure the targets are quoted against
+FALLBACK_HBM_GBS = 6650.0         # earlier measurement on this machine, used only without a measured file
+L2_BYTES = 126 * 2 ** 20
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ------------------------------------------------------------------ helpers --
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def shard_workload(wl: workloads.Workload, rank: int, world: int) -> workloads.Workload:
+    """Weak scaling: rank r runs batch elements [r*B, (r+1)*B) of a global batch
+    of world*B, i.e. the workload with its own seed.  Rank 0 keeps the base seed."""
+    return wl.with_(seed=wl.seed + 7919 * rank)
+
+
+def algorithmic_bytes(wl: workloads.Workload, elem_bytes: int) -> dict:
+    """Bytes each kernel must move per launch (one step of the workload).
+
+    write: key row in (d * elem) + packed row out (d*b/8) + norm out (4) per key;
+    read:  packed row (d*b/8) + norm (4) in + G scores out (4G) per key row,
+           plus the queries (B*H*G*d*elem) and the sign vector (d) once per call.
+    """
+    P = wl.d * wl.b // 8
+    rows = wl.rows
+    write = rows * (wl.d * elem_bytes + P + 4)
+    read = rows * (P + 4 + 4 * wl.group) + wl.heads * wl.group * wl.d * elem_bytes + wl.d
+    return {"write": write, "read": read, "write_per_key": wl.d * elem_bytes + P + 4,
+            "read_per_row": P + 4 + 4 * wl.group}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "lut_attention_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel_file: str, workload: str, b: int):
+    """DRAM bytes per launch from the committed ncu summary, when that summary was
+    taken on the current kernel source (its hash line matches); else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash(kernel_file)
+    with open(path) as f:
+        for line in f:
+            parts = line.split("#")[0].split()
+            if len(parts) == 5 and parts[0] == kernel_file and parts[1] == workload \
+                    and parts[2] == f"b={b}" and parts[3] == want:
+                return int(float(parts[4]))
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._busy = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = None
+            try:
+                uuid = torch.cuda.get_device_properties(device_index).uuid
+            except Exception:
+                pass
+            handle = None
+            if uuid is not None:
+                s = str(uuid)
+                s = s if s.startswith("GPU-") else "GPU-" + s
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByUUID(s.encode())
+                except Exception:
+                    handle = None
+            if handle is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = int(vis.split(",")[device_index]) if vis and vis.split(",")[0].isdigit() else device_index
+                handle = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nvml, self._h = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report no clocks rather than guess
+            log(f"clock sampling unavailable: {e}")
+            self._nvml = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            if self._busy.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                    get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                        nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                    reasons = get(self._h)
+                    self.samples.append((mhz, reasons))
+                except Exception:
+                    pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def busy(self, on: bool):
+        (self._busy.set if on else self._busy.clear)()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = statistics.median(s[0] for s in self.samples)
+        active = set()
+        for _, r in self.samples:
+            for name, bit in self.REASONS.items():
+                if r & bit:
+                    active.add(name)
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": sorted(active),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- the step --
+
+class Path:
+    """Device buffers and the two kernels of one step."""
+
+    def __init__(self, wl: workloads.Workload, device):
+        self.wl = wl
+        self.K = workloads.make_keys(wl, device)                 # (heads, T, d)
+        self.q = workloads.make_queries(wl, device)
+        self.signs = workloads.make_signs(wl).to(device)
+        P = wl.d * wl.b // 8
+        self.idx = [torch.empty((wl.heads, wl.T, P), dtype=torch.uint8, device=device) for _ in range(2)]
+        self.norms = [torch.empty((wl.heads, wl.T), dtype=torch.float32, device=device) for _ in range(2)]
+        self.scores = torch.empty((wl.heads * wl.group, wl.T), dtype=torch.float32, device=device)
+        for i in range(2):
+            self.quantize(i)
+
+    def quantize(self, i):
+        axr.axr_quantize_keys(self.K, self.wl.b, self.signs, idx=self.idx[i], norms=self.norms[i])
+
+    def score(self, i):
+        axr.axr_scores(self.q, self.idx[i], self.norms[i], self.wl.group, self.wl.b, self.signs,
+                       scores=self.scores)
+
+
+def run_cpu_baseline(wl: workloads.Workload, target_s: float):
+    """The oracle, as it stands (single thread), on a bounded sample of the
+    workload: the first S keys of KV head 0 quantized and scored against that
+    head's G query heads.  Returns scores/s and a description."""
+    import oracle
+
+    oracle.build()
+    K = workloads.make_keys(wl.with_(batch=1, kv_heads=1, T=min(wl.T, 1 << 16)), "cpu")[0]
+    q = workloads.make_queries(wl.with_(batch=1, kv_heads=1), "cpu").double().numpy()
+    s = workloads.make_signs(wl).numpy()
+    Kd = K.double().numpy()
+
+    def once(S):
+        t0 = time.perf_counter()
+        packed, norms, _ = oracle.quantize(Kd[:S], wl.b, s)
+        oracle.scores(q, packed[None], norms[None], wl.group, wl.b, s)
+        return time.perf_counter() - t0
+
+    S = 256
+    dt = once(S)
+    S = int(min(Kd.shape[0], max(256, S * target_s / max(dt, 1e-6))))
+    dt = once(S)
+    rate = wl.group * S / dt
+    return rate, {
+        "value": rate, "unit": "scores/s", "cores": 1, "kind": "oracle",
+        "sample": (f"first {S} keys of KV head 0 of {wl.name} (b={wl.b}): quantize + score against "
+                   f"its {wl.group} query heads; {dt:.1f} s on one host thread"),
+    }
+
+
+def reference_arm(args, wl, world, rank):
+    """--impl reference: the CPU oracle on this machine's host cores, same metric."""
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    per_step_s = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
+    K = workloads.make_keys(wl.with_(batch=1, kv_heads=1, T=min(wl.T, 1 << 16)), "cpu")[0].double().numpy()
+    q = workloads.make_queries(wl.with_(batch=1, kv_heads=1), "cpu").double().numpy()
+    s = workloads.make_signs(wl).numpy()
+
+    def step(S):
+        packed, norms, _ = oracle.quantize(K[:S], wl.b, s)
+        oracle.scores(q, packed[None], norms[None], wl.group, wl.b, s)
+
+    t0 = time.perf_counter()
+    step(128)
+    dt = time.perf_counter() - t0
+    S = int(min(K.shape[0], max(64, 128 * per_step_s / max(dt, 1e-6))))
+    for _ in range(args.warmup):
+        step(S)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step(S)
+    el = time.perf_counter() - t0
+    rate = wl.group * S * args.steps / el
+    sample = (f"each step: first {S} keys of KV head 0 of {wl.name} (b={wl.b}) quantized and scored "
+              f"against its {wl.group} query heads by the fp64 oracle, one host thread")
+    line = {
+        "impl": "reference", "metric": "lut_attention_scores_per_s", "value": rate, "unit": "scores/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl, world),
+        "cpu_baseline": {"value": rate, "unit": "scores/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": rate, "unit": "scores/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(wl, world):
+    return {
+        "workload": wl.name, "batch": wl.batch, "kv_heads": wl.kv_heads, "group": wl.group,
+        "d": wl.d, "b": wl.b, "context": wl.T, "key_dtype": wl.dtype,
+        "global_batch": wl.batch * world, "parallelism": f"shard{world}" if world > 1 else "single",
+        "l2": "inputs larger than L2 (126 MB); read kernel scores the cache written one step earlier",
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["axr", "reference"], default="axr")
+    ap.add_argument("--workload", default="gqa_decode_128k", choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--b", type=int, default=None, help="bits per coordinate (default: the workload's)")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_env()
+    base = workloads.BY_NAME[args.workload]
+    if args.b is not None:
+        base = base.with_(b=args.b)
+
+    if args.impl == "reference":
+        reference_arm(args, base, world, rank)
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    wl = shard_workload(base, rank, world)
+    elem = torch.tensor([], dtype=wl.torch_dtype).element_size()
+    algo = algorithmic_bytes(wl, elem)
+
+    # cpu baseline first (rank 0, N=1): the host is idle while the GPU runs later
+    cpu_baseline = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        _, cpu_baseline = run_cpu_baseline(wl, args.cpu_baseline_seconds)
+
+    path = Path(wl, device)
+    stream = torch.cuda.current_stream(device)
+    clocks = ClockSampler(local)
+    clocks.start()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    clocks.busy(True)
+    for i in range(args.warmup):
+        path.quantize(i % 2)
+        path.score((i + 1) % 2)
+    barrier()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        path.quantize(i % 2)
+        ev[i][1].record(stream)
+        path.score((i + 1) % 2)
+        ev[i][2].record(stream)
+    end.record(stream)
+    barrier()
+    clocks.busy(False)
+    elapsed_ms = start.elapsed_time(end)
+    t_write = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    t_read = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+
+    # max over ranks
+    t = torch.tensor([elapsed_ms, t_write, t_read], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, t_write, t_read = t.tolist()
+    ms_per_step = elapsed_ms / args.steps
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(wl, path, device, args.e2e_steps, world)
+    clocks.stop()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    scores_per_step = wl.heads * wl.group * wl.T * world
+    keys_per_step = wl.rows * world
+    peak, peak_kind = measured_peak()
+    write_gbs = algo["write"] / (t_write * 1e-3) / 1e9
+    read_gbs = algo["read"] / (t_read * 1e-3) / 1e9
+    kernels = {
+        "quantize_keys": {"ms": t_write, "algo_bytes": algo["write"], "gbs": write_gbs,
+                          "frac_of_measured": write_gbs / peak, "frac_of_8tbs": write_gbs / NOMINAL_HBM_GBS,
+                          "keys_per_s": wl.rows / (t_write * 1e-3),
+                          "bytes_per_key": algo["write_per_key"]},
+        "scores": {"ms": t_read, "algo_bytes": algo["read"], "gbs": read_gbs,
+                   "frac_of_measured": read_gbs / peak, "frac_of_8tbs": read_gbs / NOMINAL_HBM_GBS,
+                   "scores_per_s": wl.heads * wl.group * wl.T / (t_read * 1e-3),
+                   "bytes_per_row": algo["read_per_row"]},
+    }
+    dominant = "quantize_keys" if t_write >= t_read else "scores"
+    dk = kernels[dominant]
+    src = "quantize_keys.cu" if dominant == "quantize_keys" else "scores.cu"
+    line = {
+        "metric": "lut_attention_scores_per_s",
+        "value": scores_per_step / (ms_per_step * 1e-3),
+        "unit": "scores/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": config_dict(wl, world),
+        "keys_per_s": keys_per_step / (ms_per_step * 1e-3),
+        "kernels": kernels,
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dk["gbs"], "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": dk["gbs"] / peak,
+                     "frac_of_8tbs": dk["gbs"] / NOMINAL_HBM_GBS,
+                     "traffic": profiled_traffic(src, wl.name, wl.b)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "cpu_baseline": cpu_baseline,
+    }
+    print(json.dumps(line), flush=True)
+    del path
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(wl, path, device, steps, world):
+    """Same metric through the public API, inputs starting in pinned host memory:
+    per step H2D of the keys and queries, both kernels, D2H of the scores."""
+    K_host = path.K.cpu().pin_memory()
+    q_host = path.q.cpu().pin_memory()
+    out_host = torch.empty(path.scores.shape, dtype=torch.float32).pin_memory()
+    K_dev = torch.empty_like(path.K)
+    q_dev = torch.empty_like(path.q)
+    stream = torch.cuda.current_stream(device)
+    h2d = K_host.numel() * K_host.element_size() + q_host.numel() * q_host.element_size()
+    d2h = out_host.numel() * 4
+
+    def step():
+        K_dev.copy_(K_host, non_blocking=True)
+        q_dev.copy_(q_host, non_blocking=True)
+        idx, norms = axr.axr_quantize_keys(K_dev, wl.b, path.signs, idx=path.idx[0], norms=path.norms[0])
+        axr.axr_scores(q_dev, idx, norms, wl.group, wl.b, path.signs, scores=path.scores)
+        out_host.copy_(path.scores, non_blocking=True)
+
+    step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = torch.tensor([a.elapsed_time(b) / steps], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    ms = ms.item()
+    return {"value": wl.heads * wl.group * wl.T * world / (ms * 1e-3), "unit": "scores/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+// extern "C" entry points of libaxr: argument validation, codebook lookup and
+// kernel launch.  Every check runs on the host before anything is enqueued.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "axr_internal.cuh"
+
+namespace axr {
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int status, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int ok()
+{
+    g_last_error[0] = '\0';
+    return AXR_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool pow2_in_range(int d) { return d >= 8 && d <= 512 && (d & (d - 1)) == 0; }
+
+int elem_size(int dtype)
+{
+    switch (dtype) {
+    case AXR_F32: return 4;
+    case AXR_F16: return 2;
+    case AXR_BF16: return 2;
+    default: return 0;
+    }
+}
+
+// A device pointer the current device's kernels can dereference: device memory,
+// managed memory, or host memory mapped into the device address space.
+bool device_accessible(const void *p)
+{
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    switch (attr.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged: return true;
+    case cudaMemoryTypeHost: return attr.devicePointer != nullptr;
+    default: return false;
+    }
+}
+
+int check_device_ptr(const void *p, uintptr_t align, const char *name)
+{
+    if (!p) return fail(AXR_EINVAL, "%s is NULL", name);
+    if (!aligned(p, align)) return fail(AXR_EINVAL, "%s is not %u-byte aligned", name, (unsigned)align);
+    if (!device_accessible(p)) return fail(AXR_EINVAL, "%s is not device-accessible memory", name);
+    return AXR_OK;
+}
+
+int check_shape(int d, int b)
+{
+    if (!pow2_in_range(d)) return fail(AXR_EUNSUPPORTED, "d=%d: must be a power of two in [8, 512]", d);
+    if (b < 1 || b > kMaxBits) return fail(AXR_EUNSUPPORTED, "b=%d: must be in [1, %d]", b, kMaxBits);
+    return AXR_OK;
+}
+
+}  // namespace
+
+int device_sm_count()
+{
+    static std::mutex mu;
+    static std::vector<int> counts;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)counts.size() <= dev) counts.resize(dev + 1, 0);
+    if (counts[dev] == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+        counts[dev] = sms;
+    }
+    return counts[dev];
+}
+
+}  // namespace axr
+
+using namespace axr;
+
+extern "C" int axr_make_codebook(int d, int b, float *centroids, float *boundaries)
+{
+    int rc = check_shape(d, b);
+    if (rc != AXR_OK) return rc;
+    if (!centroids) return fail(AXR_EINVAL, "centroids is NULL");
+    Codebook cb;
+    if (!get_codebook(d, b, &cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
+    const int L = 1 << b;
+    std::memcpy(centroids, cb.centroids, sizeof(float) * L);
+    if (boundaries) std::memcpy(boundaries, cb.boundaries, sizeof(float) * (L - 1));
+    return ok();
+}
+
+extern "C" int axr_quantize_keys(const void *K, int kdtype, int64_t n, int d, int b,
+                                 const int8_t *signs, uint8_t *idx, float *norms,
+                                 axr_stream stream)
+{
+    int rc = check_shape(d, b);
+    if (rc != AXR_OK) return rc;
+    if (elem_size(kdtype) == 0) return fail(AXR_EINVAL, "kdtype=%d is not an axr_dtype", kdtype);
+    if (n < 0) return fail(AXR_EINVAL, "n=%lld is negative", (long long)n);
+    if (n == 0) return ok();
+    if ((rc = check_device_ptr(K, 16, "K")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(signs, 1, "signs")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(idx, 16, "idx")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(norms, 4, "norms")) != AXR_OK) return rc;
+
+    QuantizeArgs a{K, kdtype, n, d, b, signs, idx, norms, Codebook{}};
+    if (!get_codebook(d, b, &a.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
+    cudaError_t e = launch_quantize_keys(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "quantize_keys launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+extern "C" int axr_scores(const void *q, int qdtype, const uint8_t *idx, const float *norms,
+                          int64_t n, int heads, int group, int d, int b, const int8_t *signs,
+                          float *scores, axr_stream stream)
+{
+    int rc = check_shape(d, b);
+    if (rc != AXR_OK) return rc;
+    if (elem_size(qdtype) == 0) return fail(AXR_EINVAL, "qdtype=%d is not an axr_dtype", qdtype);
+    if (n < 0) return fail(AXR_EINVAL, "n=%lld is negative", (long long)n);
+    if (heads < 1) return fail(AXR_EINVAL, "heads=%d must be >= 1", heads);
+    if (group < 1) return fail(AXR_EINVAL, "group=%d must be >= 1", group);
+    if (group > kMaxGroup) return fail(AXR_EUNSUPPORTED, "group=%d: at most %d", group, kMaxGroup);
+    if (n == 0) return ok();
+    if (n > (int64_t)INT32_MAX) return fail(AXR_EUNSUPPORTED, "n=%lld: at most 2^31-1 keys per head", (long long)n);
+    if ((rc = check_device_ptr(q, 16, "q")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(idx, 16, "idx")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(norms, 4, "norms")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(signs, 1, "signs")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(scores, 4, "scores")) != AXR_OK) return rc;
+
+    ScoresArgs a{q, qdtype, idx, norms, n, heads, group, d, b, signs, scores, Codebook{}};
+    if (!get_codebook(d, b, &a.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
+    cudaError_t e = launch_scores(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "scores launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+extern "C" const char *axr_status_string(int status)
+{
+    switch (status) {
+    case AXR_OK: return "AXR_OK";
+    case AXR_EINVAL: return "AXR_EINVAL: invalid argument";
+    case AXR_EUNSUPPORTED: return "AXR_EUNSUPPORTED: unsupported d, b or group";
+    case AXR_ECUDA: return "AXR_ECUDA: CUDA error";
+    default: return "unknown axr status";
+    }
+}
+
+extern "C" const char *axr_last_error(void) { return g_last_error; }
+
+extern "C" int axr_version(void) { return 100; }

@@ -1,0 +1,225 @@
+"""Parity of the CUDA path (called through the C ABI) with the CPU oracle.
+
+Small cases are compared element by element; they span several CTAs and end in
+a ragged tail.  The decode workloads run at full size and are compared on
+sampled keys (first, last and seeded random keys of every head), which the
+oracle computes one by one.  Tolerances are in tests/parity.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lut_attention_b200 import axr, workloads
+from parity import check_quantize, check_scores, gpu_quantize, gpu_scores
+
+pytestmark = pytest.mark.gpu
+
+DIMS = (8, 16, 32, 64, 128, 256, 512)
+DTYPES = ("f32", "f16", "bf16")
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _libs(axr_lib, oracle_lib):
+    return axr_lib
+
+
+def _rows_for(d):
+    # several CTAs of warp steps plus a ragged tail, oracle time ~ n * d^2
+    return {8: 5001, 16: 5001, 32: 4001, 64: 3001, 128: 3001, 256: 1201, 512: 601}[d]
+
+
+def _keys(d, dtype, n, seed):
+    wl = workloads.MHA_DECODE_32K.with_(d=d, dtype=dtype, T=n, batch=1, kv_heads=1, seed=seed)
+    return workloads.make_keys(wl, DEV).reshape(n, d), workloads.make_signs(wl).to(DEV)
+
+
+def _assert_quantize(rep, what):
+    assert rep.ok(), f"{what}: {rep}"
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+@pytest.mark.parametrize("d", DIMS)
+def test_quantize_parity_grid(d, b, dtype):
+    n = _rows_for(d)
+    K, s = _keys(d, dtype, n, seed=1000 + d + b)
+    idx, norms = gpu_quantize(K, b, s)
+    assert idx.shape == (n, d * b // 8) and norms.shape == (n,)
+    _assert_quantize(check_quantize(K, idx, norms, b, s), f"d={d} b={b} {dtype}")
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+@pytest.mark.parametrize("d", DIMS)
+@pytest.mark.parametrize("group", [1, 4])
+def test_scores_parity_random_packed(d, b, group):
+    """The read kernel alone, on seeded random packed rows (every bit pattern is
+    a valid index), so it is tested independently of the write kernel."""
+    heads, n = 3, 2500
+    packed, norms = workloads.make_random_packed(heads, n, d, b, seed=d * 10 + b, device=DEV)
+    wl = workloads.GQA_DECODE_128K.with_(d=d, batch=1, kv_heads=heads, group=group, T=n)
+    q = workloads.make_queries(wl, DEV)
+    s = workloads.make_signs(wl).to(DEV)
+    out = gpu_scores(q, packed, norms, group, b, s)
+    assert out.shape == (heads * group, n)
+    assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
+
+
+@pytest.mark.parametrize("group", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("qdtype", DTYPES)
+def test_scores_parity_groups_and_query_dtypes(group, qdtype):
+    d, b, heads, n = 128, 3, 2, 1500
+    packed, norms = workloads.make_random_packed(heads, n, d, b, seed=77 + group, device=DEV)
+    wl = workloads.GQA_DECODE_128K.with_(batch=1, kv_heads=heads, group=group, T=n, dtype=qdtype)
+    q = workloads.make_queries(wl, DEV)
+    s = workloads.make_signs(wl).to(DEV)
+    out = gpu_scores(q, packed, norms, group, b, s)
+    assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
+
+
+def test_scores_group8_wide_head():
+    d, b, heads, n, group = 512, 2, 1, 700, 8
+    packed, norms = workloads.make_random_packed(heads, n, d, b, seed=5, device=DEV)
+    wl = workloads.WIDE_D512.with_(batch=1, kv_heads=heads, group=group, T=n)
+    q = workloads.make_queries(wl, DEV)
+    s = workloads.make_signs(wl).to(DEV)
+    out = gpu_scores(q, packed, norms, group, b, s)
+    assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
+
+
+# ----------------------------------------------------------- whole pipeline --
+
+def _sample_tokens(T, count, seed):
+    rng = np.random.default_rng(seed)
+    pick = {0, 1, T - 2, T - 1} | set(rng.integers(0, T, count).tolist())
+    return torch.tensor(sorted(t for t in pick if 0 <= t < T), dtype=torch.long)
+
+
+def _pipeline(wl, sample_per_head=None):
+    K = workloads.make_keys(wl, DEV)                       # (heads, T, d)
+    q = workloads.make_queries(wl, DEV)
+    s = workloads.make_signs(wl).to(DEV)
+    idx, norms = axr.axr_quantize_keys(K, wl.b, s)
+    scores = axr.axr_scores(q, idx, norms, wl.group, wl.b, s)
+    torch.cuda.synchronize()
+    if sample_per_head is None:
+        tok = torch.arange(wl.T)
+    else:
+        tok = _sample_tokens(wl.T, sample_per_head, wl.seed)
+    tok_d = tok.to(DEV)
+    Ks, idxs, norms_s = K[:, tok_d], idx[:, tok_d], norms[:, tok_d]
+    rep = check_quantize(Ks, idxs, norms_s, wl.b, s)
+    _assert_quantize(rep, wl.describe())
+    # read kernel on the library's own indices (keys it wrote), sampled tokens
+    err = check_scores(q, idxs, norms_s, scores[:, tok_d], wl.group, wl.b, s)
+    assert err <= 1e-4, f"{wl.describe()}: score error {err}"
+    return rep, err
+
+
+@pytest.mark.parametrize("name", [w.name for w in workloads.ALL])
+def test_pipeline_small_all_recipes(name):
+    wl = workloads.BY_NAME[name]
+    small = wl.with_(batch=1, kv_heads=min(wl.kv_heads, 2), T=1537)
+    _pipeline(small)
+
+
+FULL = [(w.name, w.b) for w in workloads.ALL if w.name != "gqa_decode_128k"] + \
+       [("gqa_decode_128k", b) for b in (2, 3, 4)]
+
+
+@pytest.mark.parametrize("name,b", FULL)
+def test_pipeline_full_size_sampled(name, b):
+    wl = workloads.BY_NAME[name].with_(b=b)
+    per_head = max(16, 4096 // wl.heads)
+    rep, err = _pipeline(wl, sample_per_head=per_head)
+    print(f"{wl.describe()}: flips={rep.flips}/{rep.coords} in-window={rep.in_window} "
+          f"norm_rel={rep.max_norm_rel:.2e} score_err={err:.2e}")
+
+
+# --------------------------------------------------------------- edge cases --
+
+def test_zero_rows_is_a_noop():
+    K = torch.zeros((0, 128), dtype=torch.bfloat16, device=DEV)
+    s = torch.ones(128, dtype=torch.int8, device=DEV)
+    idx = torch.full((4, 64), 0xAB, dtype=torch.uint8, device=DEV)
+    norms = torch.full((4,), 7.0, device=DEV)
+    axr.axr_quantize_keys(K, 4, s, idx=idx, norms=norms)
+    torch.cuda.synchronize()
+    assert torch.all(idx == 0xAB) and torch.all(norms == 7.0)
+    out = torch.full((2, 0), 1.0, device=DEV)
+    axr.axr_scores(torch.zeros((2, 128), device=DEV), torch.zeros((2, 0, 64), dtype=torch.uint8, device=DEV),
+                   torch.zeros((2, 0), device=DEV), 1, 4, s, scores=out)
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_zero_and_constant_keys(b):
+    """Zero keys store norm 0 and index 2^(b-1)-1; a constant key with all-plus
+    signs rotates onto one axis, so most coordinates are exactly 0 and sit on the
+    central boundary (ties go to the lower index on both sides)."""
+    d = 128
+    K = torch.zeros((67, d), dtype=torch.float32, device=DEV)
+    K[1::2] = 3.0
+    s = torch.ones(d, dtype=torch.int8, device=DEV)
+    idx, norms = gpu_quantize(K, b, s)
+    o_idx, o_norms, _ = oracle.quantize(K.double().cpu().numpy(), b, s.cpu().numpy())
+    assert np.array_equal(idx.cpu().numpy(), o_idx)
+    assert np.array_equal(norms.cpu().numpy(), o_norms)
+    q = torch.randn((2, d), device=DEV)
+    out = gpu_scores(q, idx[None], norms[None], 2, b, s)
+    assert torch.all(out[:, 0::2] == 0)
+
+
+def test_single_key_single_head():
+    d, b = 64, 3
+    K, s = _keys(d, "bf16", 1, seed=9)
+    idx, norms = gpu_quantize(K, b, s)
+    _assert_quantize(check_quantize(K, idx, norms, b, s), "n=1")
+    q = torch.randn((1, d), device=DEV)
+    out = gpu_scores(q, idx[None], norms[None], 1, b, s)
+    assert check_scores(q, idx[None], norms[None], out, 1, b, s) <= 1e-4
+
+
+def test_outputs_stay_inside_their_buffers():
+    """Canary bytes around every output survive both kernels."""
+    d, b, n, group = 128, 3, 1000, 4
+    K, s = _keys(d, "bf16", n, seed=3)
+    P = d * b // 8
+    guard = 4096
+    idx_buf = torch.full((guard + n * P + guard,), 0x5A, dtype=torch.uint8, device=DEV)
+    norm_buf = torch.full((guard + n + guard,), -123.0, device=DEV)
+    idx = idx_buf[guard:guard + n * P].view(n, P)
+    norms = norm_buf[guard:guard + n]
+    axr.axr_quantize_keys(K, b, s, idx=idx, norms=norms)
+    q = torch.randn((group, d), device=DEV)
+    sc_buf = torch.full((guard + group * n + guard,), -321.0, device=DEV)
+    sc = sc_buf[guard:guard + group * n].view(group, n)
+    axr.axr_scores(q, idx[None], norms[None], group, b, s, scores=sc)
+    torch.cuda.synchronize()
+    for buf, val in ((idx_buf, 0x5A), (norm_buf, -123.0), (sc_buf, -321.0)):
+        assert torch.all(buf[:guard] == val) and torch.all(buf[-guard:] == val)
+
+
+def test_device_argument_errors_do_not_launch():
+    lib = axr.library()
+    x = torch.zeros(1024, dtype=torch.uint8, device=DEV)
+    p = x.data_ptr()
+    assert lib.axr_quantize_keys(p + 4, 2, 8, 128, 4, p, p, p, None) == axr.AXR_EINVAL
+    assert lib.axr_quantize_keys(p, 2, 8, 128, 4, p, p + 4, p, None) == axr.AXR_EINVAL
+    assert lib.axr_scores(p, 2, p + 8, p, 8, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL
+    torch.cuda.synchronize()
+
+
+def test_streams_are_respected():
+    d, b, n = 128, 4, 20000
+    K, s = _keys(d, "bf16", n, seed=4)
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        idx, norms = axr.axr_quantize_keys(K, b, s)
+        out = axr.axr_scores(torch.randn((1, d), device=DEV), idx[None], norms[None], 1, b, s)
+    st.synchronize()
+    ref_idx, ref_norms = gpu_quantize(K, b, s)
+    assert torch.equal(idx, ref_idx) and torch.equal(norms, ref_norms)
+    assert torch.isfinite(out).all()

@@ -34,9 +34,11 @@ class QuantizeReport:
     max_norm_rel: float
     bytes_mismatch_rows_without_flip: int
 
-    def ok(self) -> bool:
+    def ok(self, flip_fraction: float | None = FLIP_FRACTION) -> bool:
+        """flip_fraction=None drops the cap on in-window flips (for degenerate
+        inputs built to sit exactly on a boundary)."""
         return (self.flips_outside_window == 0
-                and self.flips <= FLIP_FRACTION * self.coords
+                and (flip_fraction is None or self.flips <= flip_fraction * self.coords)
                 and self.max_norm_rel <= NORM_RTOL
                 and self.bytes_mismatch_rows_without_flip == 0)
 

@@ -156,17 +156,25 @@ def test_zero_rows_is_a_noop():
 
 @pytest.mark.parametrize("b", [1, 2, 3, 4])
 def test_zero_and_constant_keys(b):
-    """Zero keys store norm 0 and index 2^(b-1)-1; a constant key with all-plus
-    signs rotates onto one axis, so most coordinates are exactly 0 and sit on the
-    central boundary (ties go to the lower index on both sides)."""
+    """Zero keys store norm 0 and index 2^(b-1)-1.  A constant key with all-plus
+    signs rotates onto the first axis: every other rotated coordinate is exactly
+    0, on the central boundary, and the kernel's exact Hadamard sum sends it to
+    the lower index.  (The oracle's dense fp64 product leaves ~1e-17 residues
+    there, inside the 1e-6 window, so those coordinates are compared through the
+    window rule.)"""
     d = 128
+    L = 1 << b
     K = torch.zeros((67, d), dtype=torch.float32, device=DEV)
     K[1::2] = 3.0
     s = torch.ones(d, dtype=torch.int8, device=DEV)
     idx, norms = gpu_quantize(K, b, s)
-    o_idx, o_norms, _ = oracle.quantize(K.double().cpu().numpy(), b, s.cpu().numpy())
-    assert np.array_equal(idx.cpu().numpy(), o_idx)
-    assert np.array_equal(norms.cpu().numpy(), o_norms)
+    rep = check_quantize(K, idx, norms, b, s)
+    assert rep.ok(flip_fraction=None), f"constant keys b={b}: {rep}"
+    codes = oracle.unpack(idx.cpu().numpy(), d, b)
+    assert np.all(codes[0::2] == L // 2 - 1)
+    assert np.all(norms[0::2].cpu().numpy() == 0)
+    assert np.all(codes[1::2, 0] == L - 1) and np.all(codes[1::2, 1:] == L // 2 - 1)
+    assert np.all(norms[1::2].cpu().numpy() == np.float32(np.sqrt(9.0 * d)))
     q = torch.randn((2, d), device=DEV)
     out = gpu_scores(q, idx[None], norms[None], 2, b, s)
     assert torch.all(out[:, 0::2] == 0)
@@ -216,6 +224,7 @@ def test_streams_are_respected():
     d, b, n = 128, 4, 20000
     K, s = _keys(d, "bf16", n, seed=4)
     st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(st):
         idx, norms = axr.axr_quantize_keys(K, b, s)
         out = axr.axr_scores(torch.randn((1, d), device=DEV), idx[None], norms[None], 1, b, s)

@@ -113,6 +113,16 @@ int axr_scores(const void *q, int qdtype, const uint8_t *idx, const float *norms
                int64_t n, int heads, int group, int d, int b, const int8_t *signs,
                float *scores, axr_stream stream);
 
+/*
+ * Device-side status of the tensor-core kernels (no counterpart in the method;
+ * a diagnostic).  Every wait inside those kernels is bounded; a wait that runs
+ * out records a bit here instead of hanging: 1 = a tile load never arrived,
+ * 2 = a matrix product never completed, 4 = an accumulator was never released.
+ * Synchronizes the current device, writes the OR of the recorded bits to
+ * *status (0 = none) and clears them if `clear` is non-zero.
+ */
+int axr_device_status(int clear, unsigned int *status);
+
 /* Static string naming a status code. */
 const char *axr_status_string(int status);
 

@@ -30,6 +30,7 @@ SIGNATURES = {
     "axr_status_string": (ctypes.c_char_p, [_I32]),
     "axr_last_error": (ctypes.c_char_p, []),
     "axr_version": (_I32, []),
+    "axr_device_status": (_I32, [_I32, _P]),
 }
 
 _lock = threading.Lock()
@@ -152,3 +153,10 @@ def axr_scores(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, group: i
                               _stream_handle(stream))
     _raise(rc, "axr_scores")
     return scores
+
+
+def axr_device_status(clear: bool = True) -> int:
+    """Bits recorded by a bounded wait that ran out in a tensor-core kernel (0 = none)."""
+    out = ctypes.c_uint(0)
+    _raise(library().axr_device_status(1 if clear else 0, ctypes.byref(out)), "axr_device_status")
+    return out.value

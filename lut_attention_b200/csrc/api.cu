@@ -126,7 +126,8 @@ extern "C" int axr_quantize_keys(const void *K, int kdtype, int64_t n, int d, in
 
     QuantizeArgs a{K, kdtype, n, d, b, signs, idx, norms, Codebook{}};
     if (!get_codebook(d, b, &a.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
-    cudaError_t e = launch_quantize_keys(a, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = quantize_tc_supported(a) ? launch_quantize_keys_tc(a, reinterpret_cast<cudaStream_t>(stream))
+                                             : launch_quantize_keys(a, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(AXR_ECUDA, "quantize_keys launch: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -152,7 +153,8 @@ extern "C" int axr_scores(const void *q, int qdtype, const uint8_t *idx, const f
 
     ScoresArgs a{q, qdtype, idx, norms, n, heads, group, d, b, signs, scores, Codebook{}};
     if (!get_codebook(d, b, &a.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
-    cudaError_t e = launch_scores(a, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = scores_tc_supported(a) ? launch_scores_tc(a, reinterpret_cast<cudaStream_t>(stream))
+                                           : launch_scores(a, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(AXR_ECUDA, "scores launch: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -166,6 +168,18 @@ extern "C" const char *axr_status_string(int status)
     case AXR_ECUDA: return "AXR_ECUDA: CUDA error";
     default: return "unknown axr status";
     }
+}
+
+extern "C" int axr_device_status(int clear, unsigned int *status)
+{
+    if (!status) return fail(AXR_EINVAL, "status is NULL");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "device synchronize: %s", cudaGetErrorString(e));
+    const unsigned int q = quantize_tc_status(clear != 0);
+    const unsigned int r = scores_tc_status(clear != 0);
+    if (q == ~0u || r == ~0u) return fail(AXR_ECUDA, "reading the device status words failed");
+    *status = q | r;
+    return ok();
 }
 
 extern "C" const char *axr_last_error(void) { return g_last_error; }

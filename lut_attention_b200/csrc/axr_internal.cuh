@@ -23,6 +23,21 @@ struct Codebook {
 // Host solver and cache (codebook.cpp).  Returns false for unsupported (d, b).
 bool get_codebook(int d, int b, Codebook *out);
 
+// Bucket table for quantizing without a search (codebook.cpp).  A rotated unit
+// coordinate u maps to g = u * g_scale + g_off; bucket j covers g in
+// [j - 0.5, j + 0.5) and holds at most one decision boundary, tau[j] (in g
+// units, +inf if none); base[j] is the number of boundaries below the bucket.
+// Then idx(u) = base[round(g)] + (g > tau[round(g)]).  g_off is an integer and
+// no boundary lies within `margin` (in g units) of a bucket edge.
+constexpr int kMaxBuckets = 256;
+struct BucketTable {
+    int d = 0, b = 0, nt = 0;
+    float g_scale = 0.0f, g_off = 0.0f, margin = 0.0f;
+    float tau[kMaxBuckets] = {};
+    int base[kMaxBuckets] = {};
+};
+bool get_bucket_table(int d, int b, BucketTable *out);
+
 struct QuantizeArgs {
     const void *K;
     int kdtype;
@@ -53,7 +68,17 @@ struct ScoresArgs {
 // Kernel launchers (quantize_keys.cu, scores.cu).  They return cudaSuccess or
 // the launch error; arguments are already validated.
 cudaError_t launch_quantize_keys(const QuantizeArgs &a, cudaStream_t stream);
+
+// Tensor-core write path (quantize_keys_tc.cu): d = 128, bf16/fp16 keys.
+bool quantize_tc_supported(const QuantizeArgs &a);
+cudaError_t launch_quantize_keys_tc(const QuantizeArgs &a, cudaStream_t stream);
+unsigned int quantize_tc_status(bool clear);
 cudaError_t launch_scores(const ScoresArgs &a, cudaStream_t stream);
+
+// Tensor-core read path (scores_tc.cu): d = 128.
+bool scores_tc_supported(const ScoresArgs &a);
+cudaError_t launch_scores_tc(const ScoresArgs &a, cudaStream_t stream);
+unsigned int scores_tc_status(bool clear);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

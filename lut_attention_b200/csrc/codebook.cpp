@@ -87,7 +87,76 @@ Codebook build(int d, int b)
     return cb;
 }
 
+// Bucket width in sigma units: below the smallest gap between neighbouring
+// boundaries (0.258 sigma at b = 4), so no bucket holds two of them; the first
+// width whose boundaries all keep `kMinMargin` from the bucket edges is used.
+constexpr float kWidths[] = {0.25f, 0.24f, 0.23f, 0.22f, 0.21f, 0.2f, 0.19f, 0.18f};
+constexpr float kMinMargin = 0.05f;
+
+bool build_table(const Codebook &cb, BucketTable *t)
+{
+    const int L = 1 << cb.b;
+    const float sqrt_d = std::sqrt(static_cast<float>(cb.d));
+    for (float h : kWidths) {
+        BucketTable tab;
+        tab.d = cb.d;
+        tab.b = cb.b;
+        tab.g_scale = sqrt_d / h;
+        // |u| <= 1, so g stays within g_off +- g_scale (+ rounding)
+        int nt = 1;
+        while (nt < 2 * static_cast<int>(std::ceil(tab.g_scale)) + 8) nt *= 2;
+        if (nt > kMaxBuckets) continue;
+        tab.nt = nt;
+        tab.g_off = static_cast<float>(nt / 2);
+        float tg[kMaxLevels];
+        float margin = 1.0f;
+        bool ok = true;
+        for (int i = 0; i + 1 < L; ++i) {
+            tg[i] = std::fma(cb.boundaries[i], tab.g_scale, tab.g_off);
+            const float frac = tg[i] - std::floor(tg[i]);
+            margin = std::fmin(margin, std::fabs(frac - 0.5f));
+            if (i > 0 && std::floor(tg[i] + 0.5f) == std::floor(tg[i - 1] + 0.5f)) ok = false;
+        }
+        if (!ok || margin < kMinMargin) continue;
+        tab.margin = margin;
+        for (int j = 0; j < nt; ++j) {
+            tab.tau[j] = INFINITY;
+            int below = 0;
+            for (int i = 0; i + 1 < L; ++i) {
+                if (tg[i] < j - 0.5f) ++below;
+                else if (tg[i] < j + 0.5f) tab.tau[j] = tg[i];
+            }
+            tab.base[j] = below;
+        }
+        for (int j = nt; j < kMaxBuckets; ++j) {
+            tab.tau[j] = INFINITY;
+            tab.base[j] = L - 1;
+        }
+        *t = tab;
+        return true;
+    }
+    return false;
+}
+
 }  // namespace
+
+bool get_bucket_table(int d, int b, BucketTable *out)
+{
+    Codebook cb;
+    if (!out || !get_codebook(d, b, &cb)) return false;
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, BucketTable> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(d, b);
+    auto it = cache.find(key);
+    if (it == cache.end()) {
+        BucketTable t;
+        if (!build_table(cb, &t)) return false;
+        it = cache.emplace(key, t).first;
+    }
+    *out = it->second;
+    return true;
+}
 
 bool get_codebook(int d, int b, Codebook *out)
 {

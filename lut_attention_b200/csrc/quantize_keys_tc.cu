@@ -1,0 +1,440 @@
+// Quantize-on-write on the 5th-generation tensor cores, head dimension 128,
+// bf16 or fp16 keys (AXELRAM, arXiv 2604.02638, abstract: keys are transformed
+// once on write and stored as indices into a design-time codebook).
+//
+// The sign-flipped Walsh-Hadamard transform is a matrix product:
+//     y = H diag(s) k   for every key   <=>   Y = K (H diag(s))^T
+// H diag(s) has entries +-1, exact in bf16/fp16, and the keys are bf16/fp16, so
+// every product is exact and tcgen05 accumulates in fp32: the same arithmetic as
+// a butterfly transform, without spending CUDA-core instructions on it.
+//
+// One CTA per SM, persistent over 128-key tiles:
+//   warp 8 (TMA)  : streams key tiles HBM -> shared memory (4-stage ring,
+//                   128-byte swizzle, one 32 KB tile per stage);
+//   warp 9 (MMA)  : 8 tcgen05.mma (M=128, N=128, K=16) per tile into one of two
+//                   128-column fp32 accumulators in tensor memory;
+//   warps 0-7     : two warps per 32 keys (a tensor-memory lane quadrant), one
+//                   per half of the 128 columns: read y, exchange the partial
+//                   sums of y^2 (= d ||k||^2 in total), quantize, pack, store.
+// Quantization: u = y / sqrt(sum y^2); with g = u * G_SCALE + G_OFF every
+// bucket [j - 0.5, j + 0.5) of g holds at most one decision boundary, so
+//     idx = base[j] + (g > tau[j]),   j = round(g)
+// is the count of boundaries below u (one table lookup and one compare instead
+// of a b-level binary search).  tau[j] is the boundary inside bucket j (+inf if
+// none); no boundary lies near a bucket edge, so the rounding of j never
+// changes the result.  Zero keys and exact zeros land on tau = G_OFF, the
+// central boundary, and take the lower index, as ties do.  A key with a
+// non-finite entry (outside the contract) stores its non-finite norm and the
+// central index instead of reading the table out of range.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "axr_internal.cuh"
+#include "sm100.cuh"
+
+namespace axr {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kTileRows = 128;
+constexpr int kStages = 4;
+constexpr int kABytes = kTileRows * kD * 2;     // one tile of keys, 32 KB
+constexpr int kBBytes = kD * kD * 2;            // H diag(s), 32 KB
+constexpr int kHalfBytes = kTileRows * 128;     // one 64-element K block of a tile
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (kEpiWarps + 2) * 32;
+constexpr int kTmemCols = 256;                  // two 128-column accumulators
+constexpr int kWarpTma = kEpiWarps, kWarpMma = kEpiWarps + 1;
+constexpr uint32_t kMagicBits = 0x4B400000u;    // bits of 1.5 * 2^23
+constexpr float kMagic = 12582912.0f;
+
+__device__ unsigned int g_status;
+
+struct TcParams {
+    CUtensorMap tmap;              // keys as a [n, 128] tensor, box 64 x 128, 128-byte swizzle
+    uint8_t *idx;
+    float *norms;
+    const int8_t *signs;
+    int64_t n;
+    int ntiles;
+    float g_scale;
+    float g_off;
+    float inv_sqrt_d;
+    int nt;
+    float tau[kMaxBuckets];
+    int base[kMaxBuckets];
+};
+
+struct Smem {
+    uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain;
+    uint64_t pair[2][4];           // [accumulator][lane quadrant]: both halves posted their sums
+    uint32_t tmem_base;
+    float ss[2][2][kTileRows];     // [accumulator][column half][key]: partial sums of y^2
+};
+
+// Quantize one rotated coordinate y (bucket table at shared address tab, bias
+// folded so that the entry address is bits(f) * 8 + bias) and add its code into
+// the packed words at bit offset O.  Codes occupy disjoint bit fields, so adding
+// the bucket's base and then the compare bit is the same as or-ing the code.
+template <int B, int O, bool kClamp>
+__device__ __forceinline__ void quantize_one(float y, float a, float g_off, float off_magic, uint32_t tab,
+                                             uint32_t bias, uint32_t *w)
+{
+    const float g = fmaf(y, a, g_off);
+    const float f = fmaf(y, a, off_magic);          // round(g) sits in the low bits of f
+    uint32_t addr;
+    if constexpr (kClamp) {
+        const uint32_t bucket = min(__float_as_uint(f) - kMagicBits, static_cast<uint32_t>(kMaxBuckets - 1));
+        addr = tab + bucket * 8u;
+    } else {
+        addr = __float_as_uint(f) * 8u + bias;
+    }
+    float tau;
+    uint32_t base;
+    asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(tau), "=r"(base) : "r"(addr));
+    constexpr int k = O >> 5, sh = O & 31;
+    if constexpr (sh + B <= 32) {
+        w[k] += base << sh;
+        if (g > tau) w[k] += 1u << sh;
+    } else {
+        const uint32_t code = base + (g > tau ? 1u : 0u);
+        w[k] += code << sh;
+        w[k + 1] += code >> (32 - sh);
+    }
+}
+
+template <int B, int C0, int E, bool kClamp>
+__device__ __forceinline__ void quantize_chunk(const uint32_t (&v)[32], float a, float g_off, float off_magic,
+                                               uint32_t tab, uint32_t bias, uint32_t *w)
+{
+    if constexpr (E < 32) {
+        quantize_one<B, (C0 + E) * B, kClamp>(__uint_as_float(v[E]), a, g_off, off_magic, tab, bias, w);
+        quantize_chunk<B, C0, E + 1, kClamp>(v, a, g_off, off_magic, tab, bias, w);
+    }
+}
+
+template <int B, bool kBF16>
+__global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __grid_constant__ TcParams p)
+{
+    constexpr int P = kD * B / 8;            // packed bytes per key
+    constexpr int NW = P / 4;                // packed 32-bit words per key
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    uint8_t *sA = base;                                      // kStages x 32 KB
+    uint8_t *sB = sA + kStages * kABytes;                    // 32 KB
+    float2 *sTab = reinterpret_cast<float2 *>(sB + kBBytes); // kMaxBuckets entries
+    Smem &S = *reinterpret_cast<Smem *>(sTab + kMaxBuckets);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&S.full[s]), 1);
+            mbar_init(smem_u32(&S.empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&S.acc_full[a]), 1);
+            mbar_init(smem_u32(&S.acc_empty[a]), kEpiWarps * 32);   // every epilogue thread
+        }
+        mbar_init(smem_u32(&S.drain), 1);
+        for (int a = 0; a < 2; ++a)
+            for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&S.pair[a][q]), 64);   // two warps
+        fence_mbar_init();
+    }
+    if (warp == kWarpTma && lane == 0) prefetch_tensormap(&p.tmap);
+
+    // B = H diag(s) as [n = output coordinate][k = input coordinate], K-major,
+    // two 64-column blocks of 128-byte swizzled rows (the layout TMA gives A).
+    for (int chunk = threadIdx.x; chunk < kD * (kD / 8); chunk += kThreads) {
+        const int n = chunk / (kD / 8);
+        const int c = chunk % (kD / 8);          // 8-element chunk along k
+        uint32_t w[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+            uint32_t pair = 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int k = 8 * c + 2 * e2 + h;
+                const bool neg = ((__popc(n & k) & 1) != 0) != (p.signs[k] < 0);
+                const uint16_t one = kBF16 ? (neg ? 0xBF80 : 0x3F80) : (neg ? 0xBC00 : 0x3C00);
+                pair |= static_cast<uint32_t>(one) << (16 * h);
+            }
+            w[e2] = pair;
+        }
+        const int kb = c / 8, cc = c % 8;
+        uint4 *dst = reinterpret_cast<uint4 *>(sB + kb * kHalfBytes + n * 128 + ((cc ^ (n & 7)) * 16));
+        *dst = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    for (int j = threadIdx.x; j < kMaxBuckets; j += kThreads)
+        sTab[j] = make_float2(j < p.nt ? p.tau[j] : __int_as_float(0x7f800000),
+                              __int_as_float(j < p.nt ? p.base[j] : 0));
+    fence_proxy_async_smem();
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&S.tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == kWarpTma) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            int it = 0;
+            for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                if (!mbar_wait(smem_u32(&S.empty[s]), ph ^ 1)) {
+                    atomicOr(&g_status, kErrTimeoutMma);
+                    break;
+                }
+                const uint32_t full = smem_u32(&S.full[s]);
+                mbar_arrive_expect_tx(full, kABytes);
+                tma_load_2d(smem_u32(sA + s * kABytes), &p.tmap, 0, t * kTileRows, full);
+                tma_load_2d(smem_u32(sA + s * kABytes + kHalfBytes), &p.tmap, 64, t * kTileRows, full);
+            }
+            // let every load this thread issued land before the CTA exits
+            for (int k = 0; k < kStages && k < it; ++k) {
+                const int j = it - 1 - k;
+                mbar_wait(smem_u32(&S.full[j % kStages]), (j / kStages) & 1);
+            }
+        }
+    } else if (warp == kWarpMma) {
+        // --------------------------------------------------------------- MMA
+        if (lane == 0) {
+            const uint32_t id = idesc(kAccF32, kBF16 ? kFmtBF16 : kFmtF16, kBF16 ? kFmtBF16 : kFmtF16, 128, kD);
+            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+            int it = 0;
+            for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                const int acc = it & 1;
+                const uint32_t aph = (it >> 1) & 1;
+                if (!mbar_wait(smem_u32(&S.full[s]), ph)) {
+                    atomicOr(&g_status, kErrTimeoutLoad);
+                    break;
+                }
+                if (!mbar_wait(smem_u32(&S.acc_empty[acc]), aph ^ 1)) {
+                    atomicOr(&g_status, kErrTimeoutDrain);
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d = tmem + acc * kD;
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
+                    mma_f16_ss(d, desc_k_sw128(a0 + s * kABytes + off), desc_k_sw128(b0 + off), id, k > 0);
+                }
+                mma_commit(smem_u32(&S.empty[s]));
+                mma_commit(smem_u32(&S.acc_full[acc]));
+            }
+            // all MMAs of this thread complete before the tensor memory is freed
+            mma_commit(smem_u32(&S.drain));
+            mbar_wait(smem_u32(&S.drain), 0);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        constexpr int kHalfCols = kD / 2;
+        constexpr int NWH = NW / 2;                  // packed words per half row
+        const int quad = warp & 3, half = warp >> 2;
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        const int key = quad * 32 + lane;            // key within the tile
+        constexpr uint32_t kCentral = (1u << (B - 1)) - 1u;
+        const uint32_t tab_u32 = smem_u32(sTab);
+        const uint32_t tab_bias = tab_u32 - kMagicBits * 8u;     // wraps mod 2^32 by design
+        int it = 0;
+        for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t aph = (it >> 1) & 1;
+            if (!mbar_wait_warp(smem_u32(&S.acc_full[acc]), aph)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t col_addr = tmem + lane_base + acc * kD + half * kHalfCols;
+            // pass 1: this half's sum of y^2 (four interleaved partial sums); the
+            // pair adds both halves in a fixed order
+            float part4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int c = 0; c < kHalfCols / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(col_addr + 32 * c, v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    part4[e & 3] = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), part4[e & 3]);
+            }
+            S.ss[acc][half][key] = (part4[0] + part4[1]) + (part4[2] + part4[3]);
+            mbar_arrive(smem_u32(&S.pair[acc][quad]));
+            if (!mbar_wait_warp(smem_u32(&S.pair[acc][quad]), aph)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                break;
+            }
+            const float ss = S.ss[acc][0][key] + S.ss[acc][1][key];
+            const float norm = sqrtf(ss) * p.inv_sqrt_d;
+
+            uint32_t w[NWH + 1];
+#pragma unroll
+            for (int i = 0; i <= NWH; ++i) w[i] = 0;
+            // pass 2: quantize and pack this half, 32 coordinates at a time.  The
+            // tensor-memory loads stay outside the per-key branches (warp-collective).
+            // |y| <= sqrt(ss) keeps round(g) inside the table; a zero or denormal
+            // sum, where that bound can fail, takes the clamped copy of the body; a
+            // non-finite key stores the central index.
+            const bool finite = ss <= 3.402823466e38f;
+            const bool clamp = !(ss >= 1e-36f);
+            const float a = (finite && ss > 0.0f) ? p.g_scale / sqrtf(ss) : 0.0f;
+            const float g_off = p.g_off;
+            const float off_magic = g_off + kMagic;
+            {
+                uint32_t v[32];
+                tmem_ld32(col_addr, v);
+                if (finite && !clamp) quantize_chunk<B, 0, 0, false>(v, a, g_off, off_magic, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 0, 0, true>(v, a, g_off, off_magic, tab_u32, tab_bias, w);
+                tmem_ld32(col_addr + 32, v);
+                if (finite && !clamp) quantize_chunk<B, 32, 0, false>(v, a, g_off, off_magic, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 32, 0, true>(v, a, g_off, off_magic, tab_u32, tab_bias, w);
+            }
+            if (!finite) {
+#pragma unroll
+                for (int j = 0; j < kHalfCols; ++j) {
+                    const int o = j * B;
+                    w[o >> 5] |= kCentral << (o & 31);
+                    if ((o & 31) + B > 32) w[(o >> 5) + 1] |= kCentral >> (32 - (o & 31));
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&S.acc_empty[acc]));
+
+            const int64_t row = static_cast<int64_t>(t) * kTileRows + key;
+            if (row < p.n) {
+                uint8_t *dst = p.idx + row * P + half * (P / 2);
+                if constexpr (NWH % 4 == 0) {
+#pragma unroll
+                    for (int i = 0; i < NWH / 4; ++i)
+                        __stcs(reinterpret_cast<uint4 *>(dst) + i,
+                               make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < NWH / 2; ++i)
+                        __stcs(reinterpret_cast<uint2 *>(dst) + i, make_uint2(w[2 * i], w[2 * i + 1]));
+                }
+                if (half == 0) __stcs(p.norms + row, norm);
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int B, bool kBF16>
+cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_t stream)
+{
+    auto kernel = quantize_keys_tc_kernel<B, kBF16>;
+    const size_t smem = 1024 + kStages * kABytes + kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem);
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    TcParams p{};
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(a.n)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+    const cuuint32_t box[2] = {64, kTileRows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&p.tmap, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                     const_cast<void *>(a.K), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    p.idx = a.idx;
+    p.norms = a.norms;
+    p.signs = a.signs;
+    p.n = a.n;
+    p.ntiles = static_cast<int>((a.n + kTileRows - 1) / kTileRows);
+    p.g_scale = tab.g_scale;
+    p.g_off = tab.g_off;
+    p.inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(kD));
+    p.nt = tab.nt;
+    for (int j = 0; j < kMaxBuckets; ++j) {
+        p.tau[j] = tab.tau[j];
+        p.base[j] = tab.base[j];
+    }
+    const int grid = p.ntiles < device_sm_count() ? p.ntiles : device_sm_count();
+    kernel<<<grid, kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <bool kBF16>
+cudaError_t launch_typed(const QuantizeArgs &a, const BucketTable &tab, cudaStream_t stream)
+{
+    switch (a.b) {
+    case 1: return launch_tc<1, kBF16>(a, tab, stream);
+    case 2: return launch_tc<2, kBF16>(a, tab, stream);
+    case 3: return launch_tc<3, kBF16>(a, tab, stream);
+    default: return launch_tc<4, kBF16>(a, tab, stream);
+    }
+}
+
+}  // namespace
+
+bool quantize_tc_supported(const QuantizeArgs &a)
+{
+    return a.d == kD && (a.kdtype == AXR_BF16 || a.kdtype == AXR_F16) && a.n > 0 &&
+           a.n <= static_cast<int64_t>(0x7fffffff) - kTileRows && encode_tiled() != nullptr;
+}
+
+cudaError_t launch_quantize_keys_tc(const QuantizeArgs &a, cudaStream_t stream)
+{
+    BucketTable tab;
+    if (!get_bucket_table(a.d, a.b, &tab)) return cudaErrorInvalidValue;
+    return a.kdtype == AXR_BF16 ? launch_typed<true>(a, tab, stream) : launch_typed<false>(a, tab, stream);
+}
+
+unsigned int quantize_tc_status(bool clear)
+{
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return ~0u;
+    if (clear) {
+        const unsigned int z = 0;
+        cudaMemcpyToSymbol(g_status, &z, sizeof(z));
+    }
+    return v;
+}
+
+}  // namespace axr

@@ -80,6 +80,21 @@ def test_scores_parity_groups_and_query_dtypes(group, qdtype):
     assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
 
 
+@pytest.mark.parametrize("b", [2, 3, 4])
+@pytest.mark.parametrize("heads,n,group", [(64, 3001, 4), (50, 100, 2), (3, 131, 8), (200, 77, 1)])
+def test_scores_tile_ranges_cross_heads(heads, n, group, b):
+    """d = 128 reads run on the tensor-core kernel, whose CTAs walk contiguous
+    ranges of 128-key tiles: ranges cross KV heads (the query digits are rebuilt
+    mid-range) and, for n < 128, one tile spans several heads."""
+    d = 128
+    packed, norms = workloads.make_random_packed(heads, n, d, b, seed=heads + n + b, device=DEV)
+    wl = workloads.GQA_DECODE_128K.with_(batch=1, kv_heads=heads, group=group, T=n)
+    q = workloads.make_queries(wl, DEV)
+    s = workloads.make_signs(wl).to(DEV)
+    out = gpu_scores(q, packed, norms, group, b, s)
+    assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
+
+
 def test_scores_group8_wide_head():
     d, b, heads, n, group = 512, 2, 1, 700, 8
     packed, norms = workloads.make_random_packed(heads, n, d, b, seed=5, device=DEV)
@@ -88,6 +103,26 @@ def test_scores_group8_wide_head():
     s = workloads.make_signs(wl).to(DEV)
     out = gpu_scores(q, packed, norms, group, b, s)
     assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("n", [1, 5, 127, 128, 129, 255])
+def test_quantize_tensor_core_partial_tiles(n, dtype):
+    """d = 128 runs on the tensor-core kernel: tiles of 128 keys, the last one
+    partly outside the tensor (loaded as zeros, never stored)."""
+    K, s = _keys(128, dtype, n, seed=50 + n)
+    idx, norms = gpu_quantize(K, 4, s)
+    _assert_quantize(check_quantize(K, idx, norms, 4, s), f"n={n} {dtype}")
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_quantize_tensor_core_many_tiles_per_cta(b):
+    """Enough tiles that every CTA of the persistent grid runs several of them,
+    wrapping the 4-stage load ring and both accumulators; every key checked."""
+    n = 148 * 128 * 6 + 77
+    K, s = _keys(128, "bf16", n, seed=60 + b)
+    idx, norms = gpu_quantize(K, b, s)
+    _assert_quantize(check_quantize(K, idx, norms, b, s), f"n={n} b={b}")
 
 
 # ----------------------------------------------------------- whole pipeline --
@@ -104,7 +139,7 @@ def _pipeline(wl, sample_per_head=None):
     s = workloads.make_signs(wl).to(DEV)
     idx, norms = axr.axr_quantize_keys(K, wl.b, s)
     scores = axr.axr_scores(q, idx, norms, wl.group, wl.b, s)
-    torch.cuda.synchronize()
+    assert axr.axr_device_status() == 0
     if sample_per_head is None:
         tok = torch.arange(wl.T)
     else:

@@ -49,20 +49,24 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTileRows = 128;
-constexpr int kStages = 6;
-constexpr int kWorkWarps = 4;
-constexpr int kWorkers = kWorkWarps * 32;
+constexpr int kStages = 6;            // even: each stream owns every other stage
+constexpr int kStreams = 2;           // tile streams: even and odd tiles of a CTA's range
+constexpr int kGroupThreads = 128;    // decoder threads of one stream (one per key of a tile)
+constexpr int kDecodeWarps = kStreams * kGroupThreads / 32;
+constexpr int kOutWarps = 4;          // one per tensor-memory lane quadrant
+constexpr int kWorkWarps = kDecodeWarps + kOutWarps;
 constexpr int kThreads = (kWorkWarps + 2) * 32;
-constexpr int kWarpTma = kWorkWarps, kWarpMma = kWorkWarps + 1;
+constexpr int kWarpOut0 = kDecodeWarps, kWarpTma = kWorkWarps, kWarpMma = kWorkWarps + 1;
 constexpr int kK = 2 * kD;            // two digits per coordinate
 constexpr int kACols = kK / 4;        // tensor-memory columns of one A buffer
-constexpr int kTmemCols = 256;
-constexpr int kAOff = 0;              // A buffers: columns [0, 128)
-constexpr int kDOff = 128;            // D buffers: columns [128, 128 + 2*N)
+constexpr int kTmemCols = 512;
 constexpr int kNMax = 32;             // at most 8 queries x 4 digit columns
+constexpr int kDOff = kStreams * 2 * kACols;   // A buffers first, then D buffers
 constexpr int kBBytesMax = kNMax * kK; // one B buffer: N rows x K bytes
 constexpr int kStageBytes = kTileRows * 64;   // packed rows of one tile (P <= 64)
 constexpr int kLutBytes = 256 * 256;          // up to 256 fields x 256 bytes
+static_assert(kStages % kStreams == 0, "streams must own whole stages");
+static_assert(kDOff + kStreams * 2 * kNMax <= kTmemCols, "tensor memory budget");
 
 __device__ unsigned int g_status;
 
@@ -94,13 +98,17 @@ struct TcParams {
 };
 
 struct Smem {
-    uint64_t full[kStages], empty[kStages], a_full[2], a_empty[2], d_full[2], d_empty[2], drain;
-    uint64_t wsync;            // all worker threads (query rotation steps)
+    uint64_t full[kStages], empty[kStages];
+    uint64_t a_full[kStreams][2], a_empty[kStreams][2], d_full[kStreams][2], d_empty[kStreams][2];
+    uint64_t drain;
+    uint64_t wsync[kStreams];          // the threads of one stream (query rotation steps)
     uint32_t tmem_base;
-    float inv[2][8];           // per B buffer and query: 1 / (128 * S_q * S_c)
-    float q[8][kD];            // rotation scratch
-    float qmax[kWorkWarps][8];
+    float inv[kStreams][2][8];         // per stream, B buffer and query: 1 / (128 * S_q * S_c)
+    float q[kStreams][8][kD];          // rotation scratch
+    float qmax[kStreams][4][8];        // per stream warp and query: max |q''|
 };
+constexpr int kSmemBook = 12288;
+static_assert(sizeof(Smem) <= kSmemBook, "bookkeeping area too small");
 
 __device__ __forceinline__ float load_q(const void *q, int dtype, int64_t i)
 {
@@ -111,11 +119,11 @@ __device__ __forceinline__ float load_q(const void *q, int dtype, int64_t i)
     }
 }
 
-// bounded barrier of the worker threads; `phase` counts the syncs so far
-__device__ __forceinline__ bool workers_sync(Smem &S, int &phase)
+// bounded barrier of the threads of stream g; `phase` counts the syncs so far
+__device__ __forceinline__ bool stream_sync(Smem &S, int g, int &phase)
 {
-    mbar_arrive(smem_u32(&S.wsync));
-    const bool ok = mbar_wait_warp(smem_u32(&S.wsync), phase & 1);
+    mbar_arrive(smem_u32(&S.wsync[g]));
+    const bool ok = mbar_wait_warp(smem_u32(&S.wsync[g]), phase & 1);
     ++phase;
     return ok;
 }
@@ -127,52 +135,53 @@ __device__ __forceinline__ int b_offset(int n, int k)
     return ((n >> 3) * (kK / 16) + (k >> 4)) * 128 + (n & 7) * 16 + (k & 15);
 }
 
-// Rotate the G queries of KV head h and write their digits into B buffer `bbuf`
-// (all worker threads; thread j owns coordinate j).
+// Rotate the G queries of KV head h and write their digits into B buffer `b`
+// of stream g (the stream's 128 threads; thread j owns coordinate j).
 template <int B, int NQ>
-__device__ bool build_b(const TcParams &p, Smem &S, uint8_t *sB, int bbuf, int h, int &phase)
+__device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *inv, int h, int &phase)
 {
     using LK = Lookup<B>;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x & (kGroupThreads - 1);
+    float(*q)[kD] = S.q[g];
     const float sg = p.signs[tid] < 0 ? -1.0f : 1.0f;
 #pragma unroll
-    for (int g = 0; g < NQ; ++g)
-        S.q[g][tid] = (g < p.group) ? sg * load_q(p.q, p.qdtype, (static_cast<int64_t>(h) * p.group + g) * kD + tid)
-                                    : 0.0f;
-    if (!workers_sync(S, phase)) return false;
+    for (int qi = 0; qi < NQ; ++qi)
+        q[qi][tid] = (qi < p.group)
+                         ? sg * load_q(p.q, p.qdtype, (static_cast<int64_t>(h) * p.group + qi) * kD + tid)
+                         : 0.0f;
+    if (!stream_sync(S, g, phase)) return false;
     for (int hh = 1; hh < kD; hh <<= 1) {
-        for (int t = tid; t < NQ * (kD / 2); t += kWorkers) {
-            const int g = t / (kD / 2), pi = t % (kD / 2);
+        for (int t = tid; t < NQ * (kD / 2); t += kGroupThreads) {
+            const int qi = t / (kD / 2), pi = t % (kD / 2);
             const int i = (pi / hh) * 2 * hh + (pi % hh);
-            const float a = S.q[g][i], b = S.q[g][i + hh];
-            S.q[g][i] = a + b;
-            S.q[g][i + hh] = a - b;
+            const float x = q[qi][i], y = q[qi][i + hh];
+            q[qi][i] = x + y;
+            q[qi][i + hh] = x - y;
         }
-        if (!workers_sync(S, phase)) return false;
+        if (!stream_sync(S, g, phase)) return false;
     }
     // q'' = H diag(s) q / d  (rotation 1/sqrt(d) times temperature 1/sqrt(d))
     float qq[NQ];
 #pragma unroll
-    for (int g = 0; g < NQ; ++g) {
-        qq[g] = S.q[g][tid] * (1.0f / kD);
-        float m = fabsf(qq[g]);
+    for (int qi = 0; qi < NQ; ++qi) {
+        qq[qi] = q[qi][tid] * (1.0f / kD);
+        float m = fabsf(qq[qi]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if ((tid & 31) == 0) S.qmax[tid >> 5][g] = m;
+        if ((tid & 31) == 0) S.qmax[g][tid >> 5][qi] = m;
     }
-    if (!workers_sync(S, phase)) return false;
+    if (!stream_sync(S, g, phase)) return false;
     // this coordinate's hi and lo K rows: lookup l = j / C covers K indices EB*l ..
     const int l = tid / LK::C, t = tid % LK::C;
     const int k_hi = LK::EB * l + t, k_lo = LK::EB * l + LK::C + t;
-    uint8_t *b = sB + bbuf * kBBytesMax;
 #pragma unroll
-    for (int g = 0; g < NQ; ++g) {
+    for (int qi = 0; qi < NQ; ++qi) {
         float m = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kWorkWarps; ++w) m = fmaxf(m, S.qmax[w][g]);
+        for (int w = 0; w < 4; ++w) m = fmaxf(m, S.qmax[g][w][qi]);
         const float sq = (m > 0.0f) ? 64.0f / m : 1.0f;
-        if (tid == 0) S.inv[bbuf][g] = p.inv_sc / sq;
-        const float Q = qq[g] * sq;                       // |Q| <= 64
+        if (tid == 0) inv[qi] = p.inv_sc / sq;
+        const float Q = qq[qi] * sq;                      // |Q| <= 64
         const float d0 = rintf(Q);
         const float r1 = (Q - d0) * 128.0f;
         const float d1 = rintf(r1);
@@ -181,25 +190,27 @@ __device__ bool build_b(const TcParams &p, Smem &S, uint8_t *sB, int bbuf, int h
         const uint8_t D1 = static_cast<uint8_t>(static_cast<int8_t>(d1));
         const uint8_t D2 = static_cast<uint8_t>(static_cast<int8_t>(d2));
         // column weights (128, 1, 1/128, 1/128^2): hi rows (D0, D1, D2, 0), lo rows (0, D0, D1, D2)
-        b[b_offset(4 * g + 0, k_hi)] = D0;
-        b[b_offset(4 * g + 1, k_hi)] = D1;
-        b[b_offset(4 * g + 2, k_hi)] = D2;
-        b[b_offset(4 * g + 3, k_hi)] = 0;
-        b[b_offset(4 * g + 0, k_lo)] = 0;
-        b[b_offset(4 * g + 1, k_lo)] = D0;
-        b[b_offset(4 * g + 2, k_lo)] = D1;
-        b[b_offset(4 * g + 3, k_lo)] = D2;
+        b[b_offset(4 * qi + 0, k_hi)] = D0;
+        b[b_offset(4 * qi + 1, k_hi)] = D1;
+        b[b_offset(4 * qi + 2, k_hi)] = D2;
+        b[b_offset(4 * qi + 3, k_hi)] = 0;
+        b[b_offset(4 * qi + 0, k_lo)] = 0;
+        b[b_offset(4 * qi + 1, k_lo)] = D0;
+        b[b_offset(4 * qi + 2, k_lo)] = D1;
+        b[b_offset(4 * qi + 3, k_lo)] = D2;
     }
     fence_proxy_async_smem();
-    return workers_sync(S, phase);
+    return stream_sync(S, g, phase);
 }
 
-// table entry of one field value: C hi digits then C lo digits
+// table entry of one field value: C hi digits then C lo digits, replicated for
+// the 32 lanes (entry (field, lane) at field * 256 + lane * EB)
 template <int B>
 __device__ void build_lut(const TcParams &p, uint8_t *lut)
 {
     using LK = Lookup<B>;
     constexpr uint32_t mask = (1u << B) - 1u;
+    constexpr int kWorkers = kWorkWarps * 32;    // every worker thread helps
     for (int e = threadIdx.x; e < LK::NF * 32; e += kWorkers) {
         const int field = e / 32, ln = e % 32;
         uint8_t bytes[LK::EB];
@@ -225,31 +236,199 @@ __device__ __forceinline__ int chunk_offset(int r, int c)
     else return r * P + (c << 4);
 }
 
-// shared-memory address of the table entry for lookup l of a row held in w[]
+// shared-memory address of the table entry for lookup l of a row held in w[].
+// base_lane = table base (64 KB aligned) | lane * entry size, so the field
+// only has to be placed in bits 8.. of it: one PRMT for byte fields, a shift
+// and one LOP3 otherwise.
 template <int B>
-__device__ __forceinline__ uint32_t lut_addr(const uint32_t *w, int l, uint32_t lane_off)
+__device__ __forceinline__ uint32_t lut_addr(const uint32_t *w, int l, uint32_t base_lane)
 {
     using LK = Lookup<B>;
-    constexpr int o = LK::FB * 0;   // (placeholder to keep the form uniform)
-    (void)o;
     const int bit = l * LK::FB;
     const int wi = bit >> 5, sh = bit & 31;
     if constexpr (LK::FB == 8) {
-        // one PRMT: byte (sh/8) of w[wi] into bits 8..15, lane offset into bits 0..7
-        const uint32_t sel = 0x5504u | (static_cast<uint32_t>(sh >> 3) << 4);
-        return __byte_perm(w[wi], lane_off, sel);
+        // bytes: [lane offset, field, table base bits 16..23, 24..31]
+        const uint32_t sel = 0x7604u | (static_cast<uint32_t>(sh >> 3) << 4);
+        return __byte_perm(w[wi], base_lane, sel);
     } else {
         constexpr uint32_t fmask = ((1u << LK::FB) - 1u) << 8;
         uint32_t x;
         if (sh >= 8) {
-            x = (sh + LK::FB <= 32) ? (w[wi] >> (sh - 8))
-                                    : __funnelshift_r(w[wi], w[wi + 1], sh - 8);
+            x = (sh + LK::FB <= 32) ? (w[wi] >> (sh - 8)) : __funnelshift_r(w[wi], w[wi + 1], sh - 8);
         } else {
             x = w[wi] << (8 - sh);
         }
-        return (x & fmask) | lane_off;
+        return (x & fmask) | base_lane;
     }
 }
+
+// Dynamic shared memory: the table on a 64 KB boundary of the shared window
+// (so one PRMT forms a full address), the rest below it when the gap is large
+// enough, else after it.
+constexpr int kRestBytes = kStages * kStageBytes + kStreams * 2 * kBBytesMax + kSmemBook;
+constexpr size_t kSmemRequest = 1024 + 65536 + kLutBytes + kRestBytes;
+static_assert(kSmemRequest <= 232448, "shared memory per block");
+
+// Decoder threads of tile stream g (local tiles g, g+2, ...): one thread per
+// key, packed row -> table lookups -> A in tensor memory.  They also rotate the
+// queries of every new KV head into the stream's B buffers.
+template <int B, int NQ>
+struct Decoder {
+    using LK = Lookup<B>;
+    static constexpr int P = kD * B / 8;
+    static constexpr int NW = P / 4;
+
+    static __device__ void run(const TcParams &p, Smem &S, int g, uint8_t *sStage, uint8_t *sB, uint32_t lut_base,
+                               uint32_t tmem, int t0, int t1)
+    {
+        const int lane = threadIdx.x & 31;
+        const int r = threadIdx.x & (kGroupThreads - 1);   // key within the tile = tensor-memory lane
+        const uint32_t lane_base = static_cast<uint32_t>(r & ~31) << 16;
+        const uint32_t base_lane = lut_base | static_cast<uint32_t>(lane * LK::EB);
+        int bsel = -1, prev_h = -1, sync_phase = 0;
+        int h = (t0 + g) / p.tiles_per_head, ti = (t0 + g) - h * p.tiles_per_head;
+        int s = g, k = 0;
+        uint32_t sph = 0;
+
+        for (int tile = t0 + g; tile < t1; tile += kStreams, ++k) {
+            if (!mbar_wait_warp(smem_u32(&S.full[s]), sph)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutLoad);
+                return;
+            }
+            uint32_t w[NW + 1];
+            {
+                const uint8_t *st = sStage + s * kStageBytes;
+#pragma unroll
+                for (int c = 0; c < P / 16; ++c) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(st + chunk_offset<P>(r, c));
+                    w[4 * c] = x.x; w[4 * c + 1] = x.y; w[4 * c + 2] = x.z; w[4 * c + 3] = x.w;
+                }
+                w[NW] = 0;
+            }
+            mbar_arrive(smem_u32(&S.empty[s]));
+
+            if (h != prev_h) {
+                bsel = (bsel < 0) ? 0 : (bsel ^ 1);
+                prev_h = h;
+                if (!build_b<B, NQ>(p, S, g, sB + (2 * g + bsel) * kBBytesMax, S.inv[g][bsel], h, sync_phase)) {
+                    if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                    return;
+                }
+            }
+
+            const int ab = k & 1;
+            if (!mbar_wait_warp(smem_u32(&S.a_empty[g][ab]), ((k >> 1) & 1) ^ 1)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                return;
+            }
+            tc_fence_after_sync();
+            const uint32_t a_addr = tmem + lane_base + (2 * g + ab) * kACols;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t a[32];
+                if constexpr (LK::EB == 4) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const uint32_t ad = lut_addr<B>(w, 32 * half + i, base_lane);
+                        asm("ld.shared.u32 %0, [%1];" : "=r"(a[i]) : "r"(ad));
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const uint32_t ad = lut_addr<B>(w, 16 * half + i, base_lane);
+                        asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a[2 * i]), "=r"(a[2 * i + 1]) : "r"(ad));
+                    }
+                }
+                tmem_st32(a_addr + 32 * half, a);
+            }
+            tmem_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&S.a_full[g][ab]));
+
+            s += kStreams;
+            if (s >= kStages) {
+                s -= kStages;
+                sph ^= 1;
+            }
+            ti += kStreams;
+            while (ti >= p.tiles_per_head) {
+                ti -= p.tiles_per_head;
+                ++h;
+            }
+        }
+    }
+};
+
+// Output threads (one warp per lane quadrant): for every tile of the range, in
+// order, the int32 sums -> scores of its keys for every query of the head.
+template <int NQ>
+struct Output {
+    static constexpr int N = 4 * NQ;
+
+    static __device__ void run(const TcParams &p, Smem &S, uint32_t tmem, int t0, int t1)
+    {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        int bsel0 = 1, bsel1 = 1, prev_h0 = -1, prev_h1 = -1;
+        int h = t0 / p.tiles_per_head, ti = t0 - h * p.tiles_per_head;
+        // norm of this thread's key, loaded one tile ahead
+        float nk = __ldg(p.norms + static_cast<int64_t>(h) * p.n + min(ti * kTileRows + r, p.n - 1));
+        int it = 0;
+        for (int tile = t0; tile < t1; ++tile, ++it) {
+            const int g = it & 1, k = it >> 1, ab = k & 1;
+            if (g == 0 && h != prev_h0) {
+                bsel0 ^= 1;
+                prev_h0 = h;
+            } else if (g == 1 && h != prev_h1) {
+                bsel1 ^= 1;
+                prev_h1 = h;
+            }
+            const int bs = g ? bsel1 : bsel0;
+            const int t = ti * kTileRows + r;
+            // next tile's key and norm
+            int hn = h, tin = ti + 1;
+            if (tin == p.tiles_per_head) {
+                tin = 0;
+                ++hn;
+            }
+            const bool more = tile + 1 < t1;
+            const float nk_next =
+                more ? __ldg(p.norms + static_cast<int64_t>(hn) * p.n + min(tin * kTileRows + r, p.n - 1)) : 0.0f;
+
+            if (!mbar_wait_warp(smem_u32(&S.d_full[g][ab]), (k >> 1) & 1)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                return;
+            }
+            tc_fence_after_sync();
+            float sc[NQ];
+#pragma unroll
+            for (int c = 0; c < N / 16; ++c) {
+                uint32_t acc[16];
+                tmem_ld16(tmem + lane_base + kDOff + (2 * g + ab) * kNMax + 16 * c, acc);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    sc[4 * c + e] = fmaf(128.0f, __int2float_rn(static_cast<int>(acc[4 * e])),
+                                         fmaf(1.0f / 16384.0f, __int2float_rn(static_cast<int>(acc[4 * e + 3])),
+                                              fmaf(1.0f / 128.0f, __int2float_rn(static_cast<int>(acc[4 * e + 2])),
+                                                   __int2float_rn(static_cast<int>(acc[4 * e + 1])))));
+            }
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&S.d_empty[g][ab]));
+            const float *inv = S.inv[g][bs];
+            if (t < p.n) {
+#pragma unroll
+                for (int qi = 0; qi < NQ; ++qi)
+                    if (qi < p.group)
+                        __stcs(p.scores + (static_cast<int64_t>(h) * p.group + qi) * p.n + t, nk * inv[qi] * sc[qi]);
+            }
+            nk = nk_next;
+            h = hn;
+            ti = tin;
+        }
+    }
+};
 
 template <int B, int NQ>
 __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_constant__ TcParams p)
@@ -260,14 +439,16 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
     static_assert(N <= kNMax && N * kK <= kBBytesMax, "B buffer too small for N");
     static_assert(kTileRows * P <= kStageBytes, "stage too small for a tile of packed rows");
     static_assert(LK::NF * 256 <= kLutBytes, "lookup table too large");
-    constexpr int NW = P / 4;                      // words of a packed row
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
-    uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-    uint8_t *sStage = base;                         // kStages x 8 KB
-    uint8_t *sLut = sStage + kStages * kStageBytes; // 64 KB
-    uint8_t *sB = sLut + kLutBytes;                 // 2 x 8 KB
-    Smem &S = *reinterpret_cast<Smem *>(sB + 2 * kBBytesMax);
+    const uint32_t base1k = (raw + 1023u) & ~1023u;
+    const uint32_t lut_pos = (base1k + 65535u) & ~65535u;
+    const bool rest_first = lut_pos - base1k >= static_cast<uint32_t>(kRestBytes);
+    const uint32_t rest_pos = rest_first ? base1k : lut_pos + kLutBytes;
+    uint8_t *sLut = smem_raw + (lut_pos - raw);
+    uint8_t *sStage = smem_raw + (rest_pos - raw);                  // kStages x 8 KB
+    uint8_t *sB = sStage + kStages * kStageBytes;                    // streams x 2 x 8 KB
+    Smem &S = *reinterpret_cast<Smem *>(sB + kStreams * 2 * kBBytesMax);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -277,16 +458,18 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&S.full[s]), 1);
-            mbar_init(smem_u32(&S.empty[s]), kWorkers);
+            mbar_init(smem_u32(&S.empty[s]), kGroupThreads);     // consumed by one stream
         }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(smem_u32(&S.a_full[a]), kWorkers);
-            mbar_init(smem_u32(&S.a_empty[a]), 1);
-            mbar_init(smem_u32(&S.d_full[a]), 1);
-            mbar_init(smem_u32(&S.d_empty[a]), kWorkers);
+        for (int g = 0; g < kStreams; ++g) {
+            for (int a = 0; a < 2; ++a) {
+                mbar_init(smem_u32(&S.a_full[g][a]), kGroupThreads);
+                mbar_init(smem_u32(&S.a_empty[g][a]), 1);
+                mbar_init(smem_u32(&S.d_full[g][a]), 1);
+                mbar_init(smem_u32(&S.d_empty[g][a]), kOutWarps * 32);
+            }
+            mbar_init(smem_u32(&S.wsync[g]), kGroupThreads);
         }
         mbar_init(smem_u32(&S.drain), 1);
-        mbar_init(smem_u32(&S.wsync), kWorkers);
         fence_mbar_init();
     }
     if (warp == kWarpTma && lane == 0) prefetch_tensormap(&p.tmap);
@@ -303,18 +486,25 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
     if (warp == kWarpTma) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            int it = 0;
+            int it = 0, s = 0;
+            uint32_t ph = 0;
+            int h = t0 / p.tiles_per_head, ti = t0 - h * p.tiles_per_head;
             for (int tile = t0; tile < t1; ++tile, ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
                 if (!mbar_wait(smem_u32(&S.empty[s]), ph ^ 1)) {
                     atomicOr(&g_status, kErrTimeoutDrain);
                     break;
                 }
-                const int h = tile / p.tiles_per_head, i = tile % p.tiles_per_head;
                 const uint32_t full = smem_u32(&S.full[s]);
                 mbar_arrive_expect_tx(full, kTileRows * P);
-                tma_load_2d(smem_u32(sStage + s * kStageBytes), &p.tmap, 0, h * p.n + i * kTileRows, full);
+                tma_load_2d(smem_u32(sStage + s * kStageBytes), &p.tmap, 0, h * p.n + ti * kTileRows, full);
+                if (++s == kStages) {
+                    s = 0;
+                    ph ^= 1;
+                }
+                if (++ti == p.tiles_per_head) {
+                    ti = 0;
+                    ++h;
+                }
             }
             for (int k = 0; k < kStages && k < it; ++k) {
                 const int j = it - 1 - k;
@@ -326,157 +516,54 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
         if (lane == 0) {
             const uint32_t id = idesc(kAccS32, kFmtS8, kFmtS8, 128, N);
             const uint32_t b0 = smem_u32(sB);
-            int it = 0, bsel = -1, prev_h = -1;
+            // per stream: head of its last tile and the B buffer it uses (scalars,
+            // so nothing lands in local memory)
+            int prev_h0 = -1, prev_h1 = -1, bsel0 = 1, bsel1 = 1;
+            int h = t0 / p.tiles_per_head, ti = t0 - h * p.tiles_per_head;
+            int it = 0;
             for (int tile = t0; tile < t1; ++tile, ++it) {
-                const int h = tile / p.tiles_per_head;
-                if (h != prev_h) {
-                    bsel ^= 1;
-                    prev_h = h;
-                    if (bsel < 0) bsel = 0;
+                const int g = it & 1, k = it >> 1;
+                if (g == 0 && h != prev_h0) {
+                    bsel0 ^= 1;
+                    prev_h0 = h;
+                } else if (g == 1 && h != prev_h1) {
+                    bsel1 ^= 1;
+                    prev_h1 = h;
                 }
-                const int ab = it & 1;
-                const uint32_t aph = (it >> 1) & 1;
-                if (!mbar_wait(smem_u32(&S.a_full[ab]), aph)) {
+                const int bs = g ? bsel1 : bsel0;
+                if (++ti == p.tiles_per_head) {
+                    ti = 0;
+                    ++h;
+                }
+                const int ab = k & 1;
+                const uint32_t aph = (k >> 1) & 1;
+                if (!mbar_wait(smem_u32(&S.a_full[g][ab]), aph)) {
                     atomicOr(&g_status, kErrTimeoutLoad);
                     break;
                 }
-                if (!mbar_wait(smem_u32(&S.d_empty[ab]), aph ^ 1)) {
+                if (!mbar_wait(smem_u32(&S.d_empty[g][ab]), aph ^ 1)) {
                     atomicOr(&g_status, kErrTimeoutDrain);
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t d = tmem + kDOff + ab * N;
-                const uint32_t a = tmem + kAOff + ab * kACols;
+                const uint32_t d = tmem + kDOff + (2 * g + ab) * kNMax;
+                const uint32_t a = tmem + (2 * g + ab) * kACols;
+                const uint32_t bb = b0 + (2 * g + bs) * kBBytesMax;
 #pragma unroll
-                for (int k = 0; k < kK / 32; ++k) {
-                    const uint64_t bd = desc_k_interleave(b0 + bsel * kBBytesMax + k * 256, 128, (kK / 16) * 128);
-                    mma_i8_ts(d, a + 8 * k, bd, id, k > 0);
+                for (int kk = 0; kk < kK / 32; ++kk) {
+                    const uint64_t bd = desc_k_interleave(bb + kk * 256, 128, (kK / 16) * 128);
+                    mma_i8_ts(d, a + 8 * kk, bd, id, kk > 0);
                 }
-                mma_commit(smem_u32(&S.a_empty[ab]));
-                mma_commit(smem_u32(&S.d_full[ab]));
+                mma_commit(smem_u32(&S.a_empty[g][ab]));
+                mma_commit(smem_u32(&S.d_full[g][ab]));
             }
             mma_commit(smem_u32(&S.drain));
             mbar_wait(smem_u32(&S.drain), 0);
         }
     } else {
         // ------------------------------------------------------------ workers
-        const int r = threadIdx.x;                  // key within the tile = tensor-memory lane
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t lane_off = static_cast<uint32_t>(lane * LK::EB);
-        const uint32_t lut0 = smem_u32(sLut);
-        int it = 0, bsel = -1, prev_h = -1;
-        int prev_tile = -1;
-        float prev_norm = 0.0f;
-        bool ok = true;
-        int sync_phase = 0;
-
-        auto output = [&](int tile, int itp, float nk) {
-            const int ab = itp & 1;
-            if (!mbar_wait_warp(smem_u32(&S.d_full[ab]), (itp >> 1) & 1)) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                return false;
-            }
-            tc_fence_after_sync();
-            uint32_t acc[16];
-            float sc[NQ];
-#pragma unroll
-            for (int c = 0; c < N / 16; ++c) {
-                tmem_ld16(tmem + lane_base + kDOff + ab * N + 16 * c, acc);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int g = 4 * c + e;
-                    const float v = fmaf(128.0f, __int2float_rn(static_cast<int>(acc[4 * e])),
-                                         fmaf(1.0f / 16384.0f, __int2float_rn(static_cast<int>(acc[4 * e + 3])),
-                                              fmaf(1.0f / 128.0f, __int2float_rn(static_cast<int>(acc[4 * e + 2])),
-                                                   __int2float_rn(static_cast<int>(acc[4 * e + 1])))));
-                    sc[g] = v;
-                }
-            }
-            tc_fence_before_sync();
-            mbar_arrive(smem_u32(&S.d_empty[ab]));
-            const int h = tile / p.tiles_per_head;
-            const int t = (tile % p.tiles_per_head) * kTileRows + r;
-            const int hb = ((tile / p.tiles_per_head) == prev_h) ? bsel : (bsel ^ 1);
-            if (t < p.n) {
-#pragma unroll
-                for (int g = 0; g < NQ; ++g)
-                    if (g < p.group)
-                        __stcs(p.scores + (static_cast<int64_t>(h) * p.group + g) * p.n + t, nk * S.inv[hb][g] * sc[g]);
-            }
-            return true;
-        };
-
-        for (int tile = t0; tile < t1; ++tile, ++it) {
-            const int h = tile / p.tiles_per_head;
-            const int t = (tile % p.tiles_per_head) * kTileRows + r;
-            // the packed row of this thread's key
-            const int s = it % kStages;
-            if (!mbar_wait_warp(smem_u32(&S.full[s]), (it / kStages) & 1)) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutLoad);
-                ok = false;
-                break;
-            }
-            uint32_t w[NW + 1];
-            {
-                const uint8_t *st = sStage + s * kStageBytes;
-#pragma unroll
-                for (int c = 0; c < P / 16; ++c) {
-                    const uint4 x = *reinterpret_cast<const uint4 *>(st + chunk_offset<P>(r, c));
-                    w[4 * c] = x.x; w[4 * c + 1] = x.y; w[4 * c + 2] = x.z; w[4 * c + 3] = x.w;
-                }
-                w[NW] = 0;
-            }
-            mbar_arrive(smem_u32(&S.empty[s]));
-            const float nk = (t < p.n) ? __ldg(p.norms + static_cast<int64_t>(h) * p.n + t) : 0.0f;
-
-            if (h != prev_h) {
-                bsel = (bsel < 0) ? 0 : (bsel ^ 1);
-                prev_h = h;
-                if (!build_b<B, NQ>(p, S, sB, bsel, h, sync_phase)) {
-                    if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
-                    ok = false;
-                    break;
-                }
-            }
-
-            // A = the digits of this key's centroids, into tensor memory
-            const int ab = it & 1;
-            if (!mbar_wait_warp(smem_u32(&S.a_empty[ab]), ((it >> 1) & 1) ^ 1)) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                ok = false;
-                break;
-            }
-            tc_fence_after_sync();
-#pragma unroll
-            for (int q4 = 0; q4 < kACols / 16; ++q4) {
-                uint32_t a[16];
-                if constexpr (LK::EB == 4) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint32_t ad = lut0 + lut_addr<B>(w, 16 * q4 + i, lane_off);
-                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[i]) : "r"(ad));
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t ad = lut0 + lut_addr<B>(w, 8 * q4 + i, lane_off);
-                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a[2 * i]), "=r"(a[2 * i + 1]) : "r"(ad));
-                    }
-                }
-                tmem_st16(tmem + lane_base + kAOff + ab * kACols + 16 * q4, a);
-            }
-            tmem_wait_st();
-            tc_fence_before_sync();
-            mbar_arrive(smem_u32(&S.a_full[ab]));
-
-            if (prev_tile >= 0 && !output(prev_tile, it - 1, prev_norm)) {
-                ok = false;
-                break;
-            }
-            prev_tile = tile;
-            prev_norm = nk;
-        }
-        if (ok && prev_tile >= 0) output(prev_tile, it - 1, prev_norm);
+        if (warp < kDecodeWarps) Decoder<B, NQ>::run(p, S, warp / 4, sStage, sB, lut_pos, tmem, t0, t1);
+        else Output<NQ>::run(p, S, tmem, t0, t1);
     }
 
     tc_fence_before_sync();
@@ -512,7 +599,7 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
 {
     constexpr int P = kD * B / 8;
     auto kernel = scores_tc_kernel<B, NQ>;
-    const size_t smem = 1024 + kStages * kStageBytes + kLutBytes + 2 * kBBytesMax + sizeof(Smem);
+    const size_t smem = kSmemRequest;
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

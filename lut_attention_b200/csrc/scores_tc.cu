@@ -65,6 +65,7 @@ constexpr int kDOff = kStreams * 2 * kACols;   // A buffers first, then D buffer
 constexpr int kBBytesMax = kNMax * kK; // one B buffer: N rows x K bytes
 constexpr int kStageBytes = kTileRows * 64;   // packed rows of one tile (P <= 64)
 constexpr int kLutBytes = 256 * 256;          // up to 256 fields x 256 bytes
+constexpr int kNormAhead = 8;                 // tiles of key norms in flight per output thread
 static_assert(kStages % kStreams == 0, "streams must own whole stages");
 static_assert(kDOff + kStreams * 2 * kNMax <= kTmemCols, "tensor memory budget");
 
@@ -99,15 +100,18 @@ struct TcParams {
 
 struct Smem {
     uint64_t full[kStages], empty[kStages];
-    uint64_t a_full[kStreams][2], a_empty[kStreams][2], d_full[kStreams][2], d_empty[kStreams][2];
+    // per stream and buffer: A written (decoders), products done (one commit:
+    // A may be overwritten and D may be read), D read (output threads)
+    uint64_t a_full[kStreams][2], mma_done[kStreams][2], d_empty[kStreams][2];
     uint64_t drain;
     uint64_t wsync[kStreams];          // the threads of one stream (query rotation steps)
     uint32_t tmem_base;
     float inv[kStreams][2][8];         // per stream, B buffer and query: 1 / (128 * S_q * S_c)
     float q[kStreams][8][kD];          // rotation scratch
     float qmax[kStreams][4][8];        // per stream warp and query: max |q''|
+    float norm_ring[kNormAhead + 1][kTileRows];   // key norms, kNormAhead tiles ahead
 };
-constexpr int kSmemBook = 12288;
+constexpr int kSmemBook = 16384;
 static_assert(sizeof(Smem) <= kSmemBook, "bookkeeping area too small");
 
 __device__ __forceinline__ float load_q(const void *q, int dtype, int64_t i)
@@ -307,6 +311,19 @@ struct Decoder {
             }
             mbar_arrive(smem_u32(&S.empty[s]));
 
+            // buffers of this stream's tile k - 2: its products are done (so A and
+            // the B buffer of two heads back are free) and its D has been read
+            const int ab = k & 1;
+            const uint32_t prev_phase = ((k >> 1) & 1) ^ 1;
+            if (!mbar_wait_warp(smem_u32(&S.mma_done[g][ab]), prev_phase)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                return;
+            }
+            if (!mbar_wait_warp(smem_u32(&S.d_empty[g][ab]), prev_phase)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                return;
+            }
+
             if (h != prev_h) {
                 bsel = (bsel < 0) ? 0 : (bsel ^ 1);
                 prev_h = h;
@@ -314,12 +331,6 @@ struct Decoder {
                     if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
                     return;
                 }
-            }
-
-            const int ab = k & 1;
-            if (!mbar_wait_warp(smem_u32(&S.a_empty[g][ab]), ((k >> 1) & 1) ^ 1)) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                return;
             }
             tc_fence_after_sync();
             const uint32_t a_addr = tmem + lane_base + (2 * g + ab) * kACols;
@@ -361,6 +372,11 @@ struct Decoder {
 
 // Output threads (one warp per lane quadrant): for every tile of the range, in
 // order, the int32 sums -> scores of its keys for every query of the head.
+// The key norms arrive kNormAhead tiles early through per-thread asynchronous
+// copies into a ring in shared memory; each thread reads only the slot it
+// filled itself, so its own commit groups order the reads and no barrier is
+// needed.  (A norm fetched only one tile ahead leaves the whole pipeline
+// waiting on one HBM round trip per tile.)
 template <int NQ>
 struct Output {
     static constexpr int N = 4 * NQ;
@@ -373,8 +389,24 @@ struct Output {
         const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
         int bsel0 = 1, bsel1 = 1, prev_h0 = -1, prev_h1 = -1;
         int h = t0 / p.tiles_per_head, ti = t0 - h * p.tiles_per_head;
-        // norm of this thread's key, loaded one tile ahead
-        float nk = __ldg(p.norms + static_cast<int64_t>(h) * p.n + min(ti * kTileRows + r, p.n - 1));
+
+        // prefetch cursor: (head, tile in head) of tile t0 + it + kNormAhead
+        int hp = h, tip = ti;
+        const uint32_t ring = smem_u32(&S.norm_ring[0][r]);
+        auto prefetch = [&](int slot, bool valid) {
+            if (valid)
+                cp_async_4(ring + slot * (kTileRows * 4),
+                           p.norms + static_cast<int64_t>(hp) * p.n + min(tip * kTileRows + r, p.n - 1));
+            cp_async_commit();
+            if (++tip == p.tiles_per_head) {
+                tip = 0;
+                ++hp;
+            }
+        };
+#pragma unroll 1
+        for (int j = 0; j < kNormAhead; ++j) prefetch(j, t0 + j < t1);
+        int rs = 0, ws = kNormAhead;      // ring slots of tile it and of tile it + kNormAhead
+
         int it = 0;
         for (int tile = t0; tile < t1; ++tile, ++it) {
             const int g = it & 1, k = it >> 1, ab = k & 1;
@@ -387,19 +419,17 @@ struct Output {
             }
             const int bs = g ? bsel1 : bsel0;
             const int t = ti * kTileRows + r;
-            // next tile's key and norm
-            int hn = h, tin = ti + 1;
-            if (tin == p.tiles_per_head) {
-                tin = 0;
-                ++hn;
-            }
-            const bool more = tile + 1 < t1;
-            const float nk_next =
-                more ? __ldg(p.norms + static_cast<int64_t>(hn) * p.n + min(tin * kTileRows + r, p.n - 1)) : 0.0f;
 
-            if (!mbar_wait_warp(smem_u32(&S.d_full[g][ab]), (k >> 1) & 1)) {
+            // this tile's norm (copies of the kNormAhead - 1 later tiles may still fly)
+            cp_async_wait<kNormAhead - 1>();
+            const float nk = S.norm_ring[rs][r];
+            prefetch(ws, tile + kNormAhead < t1);
+            rs = (rs == kNormAhead) ? 0 : rs + 1;
+            ws = (ws == kNormAhead) ? 0 : ws + 1;
+
+            if (!mbar_wait_warp(smem_u32(&S.mma_done[g][ab]), (k >> 1) & 1)) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                return;
+                break;
             }
             tc_fence_after_sync();
             float sc[NQ];
@@ -414,19 +444,25 @@ struct Output {
                                               fmaf(1.0f / 128.0f, __int2float_rn(static_cast<int>(acc[4 * e + 2])),
                                                    __int2float_rn(static_cast<int>(acc[4 * e + 1])))));
             }
+            // the query scales of this head's B buffer, read before D is released
+            // (the release lets the decoders rebuild that buffer two heads on)
+            float inv[NQ];
+#pragma unroll
+            for (int qi = 0; qi < NQ; ++qi) inv[qi] = S.inv[g][bs][qi];
             tc_fence_before_sync();
             mbar_arrive(smem_u32(&S.d_empty[g][ab]));
-            const float *inv = S.inv[g][bs];
             if (t < p.n) {
 #pragma unroll
                 for (int qi = 0; qi < NQ; ++qi)
                     if (qi < p.group)
                         __stcs(p.scores + (static_cast<int64_t>(h) * p.group + qi) * p.n + t, nk * inv[qi] * sc[qi]);
             }
-            nk = nk_next;
-            h = hn;
-            ti = tin;
+            if (++ti == p.tiles_per_head) {
+                ti = 0;
+                ++h;
+            }
         }
+        cp_async_wait<0>();
     }
 };
 
@@ -463,8 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
         for (int g = 0; g < kStreams; ++g) {
             for (int a = 0; a < 2; ++a) {
                 mbar_init(smem_u32(&S.a_full[g][a]), kGroupThreads);
-                mbar_init(smem_u32(&S.a_empty[g][a]), 1);
-                mbar_init(smem_u32(&S.d_full[g][a]), 1);
+                mbar_init(smem_u32(&S.mma_done[g][a]), 1);
                 mbar_init(smem_u32(&S.d_empty[g][a]), kOutWarps * 32);
             }
             mbar_init(smem_u32(&S.wsync[g]), kGroupThreads);
@@ -537,25 +572,20 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
                 }
                 const int ab = k & 1;
                 const uint32_t aph = (k >> 1) & 1;
+                // A of this tile written; the decoders saw its A and D buffers free
                 if (!mbar_wait(smem_u32(&S.a_full[g][ab]), aph)) {
                     atomicOr(&g_status, kErrTimeoutLoad);
-                    break;
-                }
-                if (!mbar_wait(smem_u32(&S.d_empty[g][ab]), aph ^ 1)) {
-                    atomicOr(&g_status, kErrTimeoutDrain);
                     break;
                 }
                 tc_fence_after_sync();
                 const uint32_t d = tmem + kDOff + (2 * g + ab) * kNMax;
                 const uint32_t a = tmem + (2 * g + ab) * kACols;
                 const uint32_t bb = b0 + (2 * g + bs) * kBBytesMax;
+                // K step kk reads B 256 bytes further on: +16 in the address field
+                const uint64_t bd = desc_k_interleave(bb, 128, (kK / 16) * 128);
 #pragma unroll
-                for (int kk = 0; kk < kK / 32; ++kk) {
-                    const uint64_t bd = desc_k_interleave(bb + kk * 256, 128, (kK / 16) * 128);
-                    mma_i8_ts(d, a + 8 * kk, bd, id, kk > 0);
-                }
-                mma_commit(smem_u32(&S.a_empty[g][ab]));
-                mma_commit(smem_u32(&S.d_full[g][ab]));
+                for (int kk = 0; kk < kK / 32; ++kk) mma_i8_ts(d, a + 8 * kk, bd + 16 * kk, id, kk > 0);
+                mma_commit(smem_u32(&S.mma_done[g][ab]));
             }
             mma_commit(smem_u32(&S.drain));
             mbar_wait(smem_u32(&S.drain), 0);

@@ -55,8 +55,11 @@ constexpr int kGroupThreads = 128;    // decoder threads of one stream (one per 
 constexpr int kDecodeWarps = kStreams * kGroupThreads / 32;
 constexpr int kOutWarps = 4;          // one per tensor-memory lane quadrant
 constexpr int kWorkWarps = kDecodeWarps + kOutWarps;
-constexpr int kThreads = (kWorkWarps + 2) * 32;
-constexpr int kWarpOut0 = kDecodeWarps, kWarpTma = kWorkWarps, kWarpMma = kWorkWarps + 1;
+// one producer warp and one MMA-issuing warp per stream: a tcgen05.mma issue
+// blocks while the tensor pipe is busy, so a single issuer would leave the
+// pipe idle during its own waits and commits; two issuers keep it fed
+constexpr int kThreads = (kWorkWarps + 1 + kStreams) * 32;
+constexpr int kWarpTma = kWorkWarps, kWarpMma0 = kWorkWarps + 1;
 constexpr int kK = 2 * kD;            // two digits per coordinate
 constexpr int kACols = kK / 4;        // tensor-memory columns of one A buffer
 constexpr int kTmemCols = 512;
@@ -103,13 +106,13 @@ struct Smem {
     // per stream and buffer: A written (decoders), products done (one commit:
     // A may be overwritten and D may be read), D read (output threads)
     uint64_t a_full[kStreams][2], mma_done[kStreams][2], d_empty[kStreams][2];
-    uint64_t drain;
+    uint64_t drain[kStreams];
     uint64_t wsync[kStreams];          // the threads of one stream (query rotation steps)
     uint32_t tmem_base;
     float inv[kStreams][2][8];         // per stream, B buffer and query: 1 / (128 * S_q * S_c)
     float q[kStreams][8][kD];          // rotation scratch
     float qmax[kStreams][4][8];        // per stream warp and query: max |q''|
-    float norm_ring[kNormAhead + 1][kTileRows];   // key norms, kNormAhead tiles ahead
+    float norm_ring[kNormAhead + 2][kTileRows];   // key norms, kNormAhead tiles ahead
 };
 constexpr int kSmemBook = 16384;
 static_assert(sizeof(Smem) <= kSmemBook, "bookkeeping area too small");
@@ -370,97 +373,131 @@ struct Decoder {
     }
 };
 
-// Output threads (one warp per lane quadrant): for every tile of the range, in
-// order, the int32 sums -> scores of its keys for every query of the head.
+// Output threads (one warp per lane quadrant): the int32 sums -> scores of the
+// keys of every tile of the range, for every query of the head.  Each pass
+// takes the two streams' tiles 2m and 2m+1 together, so the waits and tensor
+// memory loads of the pair overlap.
 // The key norms arrive kNormAhead tiles early through per-thread asynchronous
-// copies into a ring in shared memory; each thread reads only the slot it
+// copies into a ring in shared memory; each thread reads only the slots it
 // filled itself, so its own commit groups order the reads and no barrier is
 // needed.  (A norm fetched only one tile ahead leaves the whole pipeline
 // waiting on one HBM round trip per tile.)
 template <int NQ>
 struct Output {
     static constexpr int N = 4 * NQ;
+    static constexpr int kSlots = kNormAhead + 2;
+
+    // int32 digit sums of one key -> sum_j q''_j c_j * 128 * S_q * S_c per query
+    static __device__ __forceinline__ void load_sums(uint32_t taddr, float (&sc)[NQ])
+    {
+#pragma unroll
+        for (int c = 0; c < N / 16; ++c) {
+            uint32_t acc[16];
+            tmem_ld16(taddr + 16 * c, acc);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                sc[4 * c + e] = fmaf(128.0f, __int2float_rn(static_cast<int>(acc[4 * e])),
+                                     fmaf(1.0f / 16384.0f, __int2float_rn(static_cast<int>(acc[4 * e + 3])),
+                                          fmaf(1.0f / 128.0f, __int2float_rn(static_cast<int>(acc[4 * e + 2])),
+                                               __int2float_rn(static_cast<int>(acc[4 * e + 1])))));
+        }
+    }
+
+    static __device__ __forceinline__ void store(const TcParams &p, int h, int t, float nk, const float (&inv)[NQ],
+                                                 const float (&sc)[NQ])
+    {
+        if (t < p.n) {
+#pragma unroll
+            for (int qi = 0; qi < NQ; ++qi)
+                if (qi < p.group)
+                    __stcs(p.scores + (static_cast<int64_t>(h) * p.group + qi) * p.n + t, nk * inv[qi] * sc[qi]);
+        }
+    }
 
     static __device__ void run(const TcParams &p, Smem &S, uint32_t tmem, int t0, int t1)
     {
+        static_assert(kStreams == 2, "tiles are taken in pairs, one per stream");
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
-        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t dbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + kDOff;
         int bsel0 = 1, bsel1 = 1, prev_h0 = -1, prev_h1 = -1;
         int h = t0 / p.tiles_per_head, ti = t0 - h * p.tiles_per_head;
 
-        // prefetch cursor: (head, tile in head) of tile t0 + it + kNormAhead
+        // prefetch cursor: (head, tile in head) of the next tile whose norms to fetch
         int hp = h, tip = ti;
         const uint32_t ring = smem_u32(&S.norm_ring[0][r]);
-        auto prefetch = [&](int slot, bool valid) {
+        int ws = 0;
+        auto prefetch = [&](bool valid) {
             if (valid)
-                cp_async_4(ring + slot * (kTileRows * 4),
+                cp_async_4(ring + ws * (kTileRows * 4),
                            p.norms + static_cast<int64_t>(hp) * p.n + min(tip * kTileRows + r, p.n - 1));
             cp_async_commit();
+            ws = (ws == kSlots - 1) ? 0 : ws + 1;
             if (++tip == p.tiles_per_head) {
                 tip = 0;
                 ++hp;
             }
         };
 #pragma unroll 1
-        for (int j = 0; j < kNormAhead; ++j) prefetch(j, t0 + j < t1);
-        int rs = 0, ws = kNormAhead;      // ring slots of tile it and of tile it + kNormAhead
+        for (int j = 0; j < kNormAhead; ++j) prefetch(t0 + j < t1);
+        int rs = 0;                        // ring slot of tile `tile`
 
-        int it = 0;
-        for (int tile = t0; tile < t1; ++tile, ++it) {
-            const int g = it & 1, k = it >> 1, ab = k & 1;
-            if (g == 0 && h != prev_h0) {
-                bsel0 ^= 1;
-                prev_h0 = h;
-            } else if (g == 1 && h != prev_h1) {
-                bsel1 ^= 1;
-                prev_h1 = h;
-            }
-            const int bs = g ? bsel1 : bsel0;
-            const int t = ti * kTileRows + r;
-
-            // this tile's norm (copies of the kNormAhead - 1 later tiles may still fly)
-            cp_async_wait<kNormAhead - 1>();
-            const float nk = S.norm_ring[rs][r];
-            prefetch(ws, tile + kNormAhead < t1);
-            rs = (rs == kNormAhead) ? 0 : rs + 1;
-            ws = (ws == kNormAhead) ? 0 : ws + 1;
-
-            if (!mbar_wait_warp(smem_u32(&S.mma_done[g][ab]), (k >> 1) & 1)) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                break;
-            }
-            tc_fence_after_sync();
-            float sc[NQ];
-#pragma unroll
-            for (int c = 0; c < N / 16; ++c) {
-                uint32_t acc[16];
-                tmem_ld16(tmem + lane_base + kDOff + (2 * g + ab) * kNMax + 16 * c, acc);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    sc[4 * c + e] = fmaf(128.0f, __int2float_rn(static_cast<int>(acc[4 * e])),
-                                         fmaf(1.0f / 16384.0f, __int2float_rn(static_cast<int>(acc[4 * e + 3])),
-                                              fmaf(1.0f / 128.0f, __int2float_rn(static_cast<int>(acc[4 * e + 2])),
-                                                   __int2float_rn(static_cast<int>(acc[4 * e + 1])))));
-            }
-            // the query scales of this head's B buffer, read before D is released
-            // (the release lets the decoders rebuild that buffer two heads on)
-            float inv[NQ];
-#pragma unroll
-            for (int qi = 0; qi < NQ; ++qi) inv[qi] = S.inv[g][bs][qi];
-            tc_fence_before_sync();
-            mbar_arrive(smem_u32(&S.d_empty[g][ab]));
-            if (t < p.n) {
-#pragma unroll
-                for (int qi = 0; qi < NQ; ++qi)
-                    if (qi < p.group)
-                        __stcs(p.scores + (static_cast<int64_t>(h) * p.group + qi) * p.n + t, nk * inv[qi] * sc[qi]);
-            }
+        for (int tile = t0, k = 0; tile < t1; tile += 2, ++k) {
+            const bool two = tile + 1 < t1;
+            const int ab = k & 1;
+            const uint32_t ph = (k >> 1) & 1;
+            // heads of the pair and the B buffers (query scales) they use
+            const int h0 = h, i0 = ti;
             if (++ti == p.tiles_per_head) {
                 ti = 0;
                 ++h;
             }
+            const int h1 = h, i1 = ti;
+            if (++ti == p.tiles_per_head) {
+                ti = 0;
+                ++h;
+            }
+            if (h0 != prev_h0) {
+                bsel0 ^= 1;
+                prev_h0 = h0;
+            }
+            if (two && h1 != prev_h1) {
+                bsel1 ^= 1;
+                prev_h1 = h1;
+            }
+
+            // the pair's norms (slots rs, rs + 1); copies of later tiles may still fly
+            cp_async_wait<kNormAhead - 2>();
+            const float nk0 = S.norm_ring[rs][r];
+            const int rs1 = (rs == kSlots - 1) ? 0 : rs + 1;
+            const float nk1 = S.norm_ring[rs1][r];
+            rs = (rs1 == kSlots - 1) ? 0 : rs1 + 1;
+            prefetch(tile + kNormAhead < t1);
+            prefetch(tile + 1 + kNormAhead < t1);
+
+            if (!mbar_wait_warp(smem_u32(&S.mma_done[0][ab]), ph) ||
+                (two && !mbar_wait_warp(smem_u32(&S.mma_done[1][ab]), ph))) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                break;
+            }
+            tc_fence_after_sync();
+            float sc0[NQ], sc1[NQ];
+            load_sums(dbase + ab * kNMax, sc0);
+            if (two) load_sums(dbase + (2 + ab) * kNMax, sc1);
+            // the query scales of the pair's B buffers, read before D is released
+            // (the release lets the decoders rebuild a buffer two heads on)
+            float inv0[NQ], inv1[NQ];
+#pragma unroll
+            for (int qi = 0; qi < NQ; ++qi) {
+                inv0[qi] = S.inv[0][bsel0][qi];
+                inv1[qi] = S.inv[1][bsel1][qi];
+            }
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&S.d_empty[0][ab]));
+            if (two) mbar_arrive(smem_u32(&S.d_empty[1][ab]));
+            store(p, h0, i0 * kTileRows + r, nk0, inv0, sc0);
+            if (two) store(p, h1, i1 * kTileRows + r, nk1, inv1, sc1);
         }
         cp_async_wait<0>();
     }
@@ -504,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
             }
             mbar_init(smem_u32(&S.wsync[g]), kGroupThreads);
         }
-        mbar_init(smem_u32(&S.drain), 1);
+        for (int g = 0; g < kStreams; ++g) mbar_init(smem_u32(&S.drain[g]), 1);
         fence_mbar_init();
     }
     if (warp == kWarpTma && lane == 0) prefetch_tensormap(&p.tmap);
@@ -546,49 +583,45 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
                 mbar_wait(smem_u32(&S.full[j % kStages]), (j / kStages) & 1);
             }
         }
-    } else if (warp == kWarpMma) {
-        // --------------------------------------------------------------- MMA
+    } else if (warp >= kWarpMma0) {
+        // ------------------------------------------------- MMA, one per stream
         if (lane == 0) {
+            const int g = warp - kWarpMma0;
             const uint32_t id = idesc(kAccS32, kFmtS8, kFmtS8, 128, N);
-            const uint32_t b0 = smem_u32(sB);
-            // per stream: head of its last tile and the B buffer it uses (scalars,
-            // so nothing lands in local memory)
-            int prev_h0 = -1, prev_h1 = -1, bsel0 = 1, bsel1 = 1;
-            int h = t0 / p.tiles_per_head, ti = t0 - h * p.tiles_per_head;
-            int it = 0;
-            for (int tile = t0; tile < t1; ++tile, ++it) {
-                const int g = it & 1, k = it >> 1;
-                if (g == 0 && h != prev_h0) {
-                    bsel0 ^= 1;
-                    prev_h0 = h;
-                } else if (g == 1 && h != prev_h1) {
-                    bsel1 ^= 1;
-                    prev_h1 = h;
-                }
-                const int bs = g ? bsel1 : bsel0;
-                if (++ti == p.tiles_per_head) {
-                    ti = 0;
-                    ++h;
+            const uint32_t b0 = smem_u32(sB) + 2 * g * kBBytesMax;
+            const uint32_t a0 = tmem + 2 * g * kACols;
+            const uint32_t d0 = tmem + kDOff + 2 * g * kNMax;
+            // the stream's B buffer flips whenever its tiles enter a new head,
+            // exactly as the decoders flip it
+            int bsel = 1, prev_h = -1;
+            int h = (t0 + g) / p.tiles_per_head, ti = (t0 + g) - h * p.tiles_per_head;
+            int k = 0;
+            for (int tile = t0 + g; tile < t1; tile += kStreams, ++k) {
+                if (h != prev_h) {
+                    bsel ^= 1;
+                    prev_h = h;
                 }
                 const int ab = k & 1;
-                const uint32_t aph = (k >> 1) & 1;
                 // A of this tile written; the decoders saw its A and D buffers free
-                if (!mbar_wait(smem_u32(&S.a_full[g][ab]), aph)) {
+                if (!mbar_wait(smem_u32(&S.a_full[g][ab]), (k >> 1) & 1)) {
                     atomicOr(&g_status, kErrTimeoutLoad);
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t d = tmem + kDOff + (2 * g + ab) * kNMax;
-                const uint32_t a = tmem + (2 * g + ab) * kACols;
-                const uint32_t bb = b0 + (2 * g + bs) * kBBytesMax;
                 // K step kk reads B 256 bytes further on: +16 in the address field
-                const uint64_t bd = desc_k_interleave(bb, 128, (kK / 16) * 128);
+                const uint64_t bd = desc_k_interleave(b0 + bsel * kBBytesMax, 128, (kK / 16) * 128);
+                const uint32_t d = d0 + ab * kNMax, a = a0 + ab * kACols;
 #pragma unroll
                 for (int kk = 0; kk < kK / 32; ++kk) mma_i8_ts(d, a + 8 * kk, bd + 16 * kk, id, kk > 0);
                 mma_commit(smem_u32(&S.mma_done[g][ab]));
+                ti += kStreams;
+                while (ti >= p.tiles_per_head) {
+                    ti -= p.tiles_per_head;
+                    ++h;
+                }
             }
-            mma_commit(smem_u32(&S.drain));
-            mbar_wait(smem_u32(&S.drain), 0);
+            mma_commit(smem_u32(&S.drain[g]));
+            mbar_wait(smem_u32(&S.drain[g]), 0);
         }
     } else {
         // ------------------------------------------------------------ workers

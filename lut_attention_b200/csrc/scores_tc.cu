@@ -64,13 +64,18 @@ constexpr int kK = 2 * kD;            // two digits per coordinate
 constexpr int kACols = kK / 4;        // tensor-memory columns of one A buffer
 constexpr int kTmemCols = 512;
 constexpr int kNMax = 32;             // at most 8 queries x 4 digit columns
+constexpr int kDBufs = 4;             // D buffers per stream: the output may lag this many tiles
+constexpr int kInvSlots = 8;          // per-stream ring of query scales, one slot per head
 constexpr int kDOff = kStreams * 2 * kACols;   // A buffers first, then D buffers
 constexpr int kBBytesMax = kNMax * kK; // one B buffer: N rows x K bytes
 constexpr int kStageBytes = kTileRows * 64;   // packed rows of one tile (P <= 64)
 constexpr int kLutBytes = 256 * 256;          // up to 256 fields x 256 bytes
 constexpr int kNormAhead = 8;                 // tiles of key norms in flight per output thread
 static_assert(kStages % kStreams == 0, "streams must own whole stages");
-static_assert(kDOff + kStreams * 2 * kNMax <= kTmemCols, "tensor memory budget");
+static_assert(kDOff + kStreams * kDBufs * kNMax <= kTmemCols, "tensor memory budget");
+// a stream's output can be at most kDBufs + 1 tiles (so heads) behind its decoders
+static_assert(kInvSlots >= kDBufs + 2, "query-scale ring too short");
+static_assert((kInvSlots & (kInvSlots - 1)) == 0 && (kDBufs & (kDBufs - 1)) == 0, "ring sizes are powers of two");
 
 __device__ unsigned int g_status;
 
@@ -103,13 +108,14 @@ struct TcParams {
 
 struct Smem {
     uint64_t full[kStages], empty[kStages];
-    // per stream and buffer: A written (decoders), products done (one commit:
-    // A may be overwritten and D may be read), D read (output threads)
-    uint64_t a_full[kStreams][2], mma_done[kStreams][2], d_empty[kStreams][2];
+    // per stream and A buffer: A written (decoders), products done (A free)
+    uint64_t a_full[kStreams][2], mma_done[kStreams][2];
+    // per stream and D buffer: sums ready (MMA commit), sums read (output threads)
+    uint64_t d_full[kStreams][kDBufs], d_empty[kStreams][kDBufs];
     uint64_t drain[kStreams];
     uint64_t wsync[kStreams];          // the threads of one stream (query rotation steps)
     uint32_t tmem_base;
-    float inv[kStreams][2][8];         // per stream, B buffer and query: 1 / (128 * S_q * S_c)
+    float inv[kStreams][kInvSlots][8]; // per stream, head slot and query: 1 / (128 * S_q * S_c)
     float q[kStreams][8][kD];          // rotation scratch
     float qmax[kStreams][4][8];        // per stream warp and query: max |q''|
     float norm_ring[kNormAhead + 2][kTileRows];   // key norms, kNormAhead tiles ahead
@@ -292,7 +298,7 @@ struct Decoder {
         const int r = threadIdx.x & (kGroupThreads - 1);   // key within the tile = tensor-memory lane
         const uint32_t lane_base = static_cast<uint32_t>(r & ~31) << 16;
         const uint32_t base_lane = lut_base | static_cast<uint32_t>(lane * LK::EB);
-        int bsel = -1, prev_h = -1, sync_phase = 0;
+        int bsel = -1, prev_h = -1, hc = -1, sync_phase = 0;
         int h = (t0 + g) / p.tiles_per_head, ti = (t0 + g) - h * p.tiles_per_head;
         int s = g, k = 0;
         uint32_t sph = 0;
@@ -314,23 +320,20 @@ struct Decoder {
             }
             mbar_arrive(smem_u32(&S.empty[s]));
 
-            // buffers of this stream's tile k - 2: its products are done (so A and
-            // the B buffer of two heads back are free) and its D has been read
+            // the products of this stream's tile k - 2 are done, so its A buffer
+            // and the B buffer of two heads back are free
             const int ab = k & 1;
-            const uint32_t prev_phase = ((k >> 1) & 1) ^ 1;
-            if (!mbar_wait_warp(smem_u32(&S.mma_done[g][ab]), prev_phase)) {
+            if (!mbar_wait_warp(smem_u32(&S.mma_done[g][ab]), ((k >> 1) & 1) ^ 1)) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                return;
-            }
-            if (!mbar_wait_warp(smem_u32(&S.d_empty[g][ab]), prev_phase)) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
                 return;
             }
 
             if (h != prev_h) {
                 bsel = (bsel < 0) ? 0 : (bsel ^ 1);
                 prev_h = h;
-                if (!build_b<B, NQ>(p, S, g, sB + (2 * g + bsel) * kBBytesMax, S.inv[g][bsel], h, sync_phase)) {
+                ++hc;
+                if (!build_b<B, NQ>(p, S, g, sB + (2 * g + bsel) * kBBytesMax, S.inv[g][hc & (kInvSlots - 1)], h,
+                                    sync_phase)) {
                     if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
                     return;
                 }
@@ -421,7 +424,7 @@ struct Output {
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t dbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + kDOff;
-        int bsel0 = 1, bsel1 = 1, prev_h0 = -1, prev_h1 = -1;
+        int hc0 = -1, hc1 = -1, prev_h0 = -1, prev_h1 = -1;   // per stream: heads seen, last head
         int h = t0 / p.tiles_per_head, ti = t0 - h * p.tiles_per_head;
 
         // prefetch cursor: (head, tile in head) of the next tile whose norms to fetch
@@ -445,8 +448,8 @@ struct Output {
 
         for (int tile = t0, k = 0; tile < t1; tile += 2, ++k) {
             const bool two = tile + 1 < t1;
-            const int ab = k & 1;
-            const uint32_t ph = (k >> 1) & 1;
+            const int dk = k & (kDBufs - 1);
+            const uint32_t ph = (k / kDBufs) & 1;
             // heads of the pair and the B buffers (query scales) they use
             const int h0 = h, i0 = ti;
             if (++ti == p.tiles_per_head) {
@@ -459,11 +462,11 @@ struct Output {
                 ++h;
             }
             if (h0 != prev_h0) {
-                bsel0 ^= 1;
+                ++hc0;
                 prev_h0 = h0;
             }
             if (two && h1 != prev_h1) {
-                bsel1 ^= 1;
+                ++hc1;
                 prev_h1 = h1;
             }
 
@@ -476,26 +479,26 @@ struct Output {
             prefetch(tile + kNormAhead < t1);
             prefetch(tile + 1 + kNormAhead < t1);
 
-            if (!mbar_wait_warp(smem_u32(&S.mma_done[0][ab]), ph) ||
-                (two && !mbar_wait_warp(smem_u32(&S.mma_done[1][ab]), ph))) {
+            if (!mbar_wait_warp(smem_u32(&S.d_full[0][dk]), ph) ||
+                (two && !mbar_wait_warp(smem_u32(&S.d_full[1][dk]), ph))) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
                 break;
             }
             tc_fence_after_sync();
             float sc0[NQ], sc1[NQ];
-            load_sums(dbase + ab * kNMax, sc0);
-            if (two) load_sums(dbase + (2 + ab) * kNMax, sc1);
-            // the query scales of the pair's B buffers, read before D is released
-            // (the release lets the decoders rebuild a buffer two heads on)
+            load_sums(dbase + dk * kNMax, sc0);
+            if (two) load_sums(dbase + (kDBufs + dk) * kNMax, sc1);
+            // the query scales of the pair's heads, read before D is released
+            // (the release lets the decoders reuse a head slot kInvSlots heads on)
             float inv0[NQ], inv1[NQ];
 #pragma unroll
             for (int qi = 0; qi < NQ; ++qi) {
-                inv0[qi] = S.inv[0][bsel0][qi];
-                inv1[qi] = S.inv[1][bsel1][qi];
+                inv0[qi] = S.inv[0][hc0 & (kInvSlots - 1)][qi];
+                inv1[qi] = S.inv[1][hc1 & (kInvSlots - 1)][qi];
             }
             tc_fence_before_sync();
-            mbar_arrive(smem_u32(&S.d_empty[0][ab]));
-            if (two) mbar_arrive(smem_u32(&S.d_empty[1][ab]));
+            mbar_arrive(smem_u32(&S.d_empty[0][dk]));
+            if (two) mbar_arrive(smem_u32(&S.d_empty[1][dk]));
             store(p, h0, i0 * kTileRows + r, nk0, inv0, sc0);
             if (two) store(p, h1, i1 * kTileRows + r, nk1, inv1, sc1);
         }
@@ -537,6 +540,9 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
             for (int a = 0; a < 2; ++a) {
                 mbar_init(smem_u32(&S.a_full[g][a]), kGroupThreads);
                 mbar_init(smem_u32(&S.mma_done[g][a]), 1);
+            }
+            for (int a = 0; a < kDBufs; ++a) {
+                mbar_init(smem_u32(&S.d_full[g][a]), 1);
                 mbar_init(smem_u32(&S.d_empty[g][a]), kOutWarps * 32);
             }
             mbar_init(smem_u32(&S.wsync[g]), kGroupThreads);
@@ -590,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
             const uint32_t id = idesc(kAccS32, kFmtS8, kFmtS8, 128, N);
             const uint32_t b0 = smem_u32(sB) + 2 * g * kBBytesMax;
             const uint32_t a0 = tmem + 2 * g * kACols;
-            const uint32_t d0 = tmem + kDOff + 2 * g * kNMax;
+            const uint32_t d0 = tmem + kDOff + g * kDBufs * kNMax;
             // the stream's B buffer flips whenever its tiles enter a new head,
             // exactly as the decoders flip it
             int bsel = 1, prev_h = -1;
@@ -601,19 +607,24 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
                     bsel ^= 1;
                     prev_h = h;
                 }
-                const int ab = k & 1;
-                // A of this tile written; the decoders saw its A and D buffers free
+                const int ab = k & 1, dk = k & (kDBufs - 1);
+                // A of this tile written, and the sums of tile k - kDBufs read out of D
                 if (!mbar_wait(smem_u32(&S.a_full[g][ab]), (k >> 1) & 1)) {
                     atomicOr(&g_status, kErrTimeoutLoad);
+                    break;
+                }
+                if (!mbar_wait(smem_u32(&S.d_empty[g][dk]), ((k / kDBufs) & 1) ^ 1)) {
+                    atomicOr(&g_status, kErrTimeoutDrain);
                     break;
                 }
                 tc_fence_after_sync();
                 // K step kk reads B 256 bytes further on: +16 in the address field
                 const uint64_t bd = desc_k_interleave(b0 + bsel * kBBytesMax, 128, (kK / 16) * 128);
-                const uint32_t d = d0 + ab * kNMax, a = a0 + ab * kACols;
+                const uint32_t d = d0 + dk * kNMax, a = a0 + ab * kACols;
 #pragma unroll
                 for (int kk = 0; kk < kK / 32; ++kk) mma_i8_ts(d, a + 8 * kk, bd + 16 * kk, id, kk > 0);
                 mma_commit(smem_u32(&S.mma_done[g][ab]));
+                mma_commit(smem_u32(&S.d_full[g][dk]));
                 ti += kStreams;
                 while (ti >= p.tiles_per_head) {
                     ti -= p.tiles_per_head;

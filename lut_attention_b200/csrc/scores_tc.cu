@@ -25,15 +25,23 @@
 // codes from a table replicated per lane (address = field * 256 + lane * entry
 // size), which is conflict-free in shared memory.
 //
-// One CTA per SM, persistent over a contiguous range of 128-key tiles:
-//   warp 4 (TMA) : packed index tiles HBM -> shared memory (6 stages);
-//   warp 5 (MMA) : 8 tcgen05.mma (M=128, N=16|32, K=32) per tile;
-//   warps 0-3    : one thread per key: read its packed row, look up its digits,
-//                  store them to tensor memory (A); for the previous tile read
-//                  the int32 sums (D), scale by the key norm, store the scores.
-// Whenever the range enters a new KV head the worker warps rotate that head's
-// queries (sign flip, Walsh-Hadamard butterflies, 1/d) and write its digits
-// into the other of two B buffers.
+// One CTA per SM, persistent over a contiguous range of 128-key tiles, which it
+// deals round-robin to S tile streams (S = 3 for up to 4 queries per KV head,
+// else 2).  Per stream:
+//   4 worker warps : one thread per key (= tensor-memory lane).  For tile k:
+//                    read the packed row, look up its digits, store them to A
+//                    in tensor memory; then, once the products of tile k - 2
+//                    are done, read its int32 sums (D), scale them by the key
+//                    norm and the query scale, store the scores.  On entering a
+//                    new KV head they rotate its queries (sign flip,
+//                    Walsh-Hadamard butterflies, 1/d) and write their digits
+//                    into the other of the stream's two B buffers.
+//   1 MMA warp     : 8 tcgen05.mma (M = 128, N = 4G, K = 32) per tile and one
+//                    commit, which frees A and publishes D at once.
+// plus one TMA warp loading packed tiles HBM -> shared memory (6 stages).
+// A tcgen05.mma issue blocks while the tensor pipe works, and a tile's 8
+// products take longer than its decode, so every stream has its own issuer:
+// together they keep the pipe fed while each waits for its own workers.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -49,33 +57,32 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTileRows = 128;
-constexpr int kStages = 6;            // even: each stream owns every other stage
-constexpr int kStreams = 2;           // tile streams: even and odd tiles of a CTA's range
-constexpr int kGroupThreads = 128;    // decoder threads of one stream (one per key of a tile)
-constexpr int kDecodeWarps = kStreams * kGroupThreads / 32;
-constexpr int kOutWarps = 4;          // one per tensor-memory lane quadrant
-constexpr int kWorkWarps = kDecodeWarps + kOutWarps;
-// one producer warp and one MMA-issuing warp per stream: a tcgen05.mma issue
-// blocks while the tensor pipe is busy, so a single issuer would leave the
-// pipe idle during its own waits and commits; two issuers keep it fed
-constexpr int kThreads = (kWorkWarps + 1 + kStreams) * 32;
-constexpr int kWarpTma = kWorkWarps, kWarpMma0 = kWorkWarps + 1;
+constexpr int kStages = 6;            // a multiple of every stream count: a stream owns whole stages
+constexpr int kGroupThreads = 128;    // worker threads of one stream (one per key of a tile)
 constexpr int kK = 2 * kD;            // two digits per coordinate
 constexpr int kACols = kK / 4;        // tensor-memory columns of one A buffer
 constexpr int kTmemCols = 512;
-constexpr int kNMax = 32;             // at most 8 queries x 4 digit columns
-constexpr int kDBufs = 4;             // D buffers per stream: the output may lag this many tiles
-constexpr int kInvSlots = 8;          // per-stream ring of query scales, one slot per head
-constexpr int kDOff = kStreams * 2 * kACols;   // A buffers first, then D buffers
-constexpr int kBBytesMax = kNMax * kK; // one B buffer: N rows x K bytes
 constexpr int kStageBytes = kTileRows * 64;   // packed rows of one tile (P <= 64)
 constexpr int kLutBytes = 256 * 256;          // up to 256 fields x 256 bytes
-constexpr int kNormAhead = 8;                 // tiles of key norms in flight per output thread
-static_assert(kStages % kStreams == 0, "streams must own whole stages");
-static_assert(kDOff + kStreams * kDBufs * kNMax <= kTmemCols, "tensor memory budget");
-// a stream's output can be at most kDBufs + 1 tiles (so heads) behind its decoders
-static_assert(kInvSlots >= kDBufs + 2, "query-scale ring too short");
-static_assert((kInvSlots & (kInvSlots - 1)) == 0 && (kDBufs & (kDBufs - 1)) == 0, "ring sizes are powers of two");
+constexpr int kInvSlots = 8;          // per-stream ring of query scales, one slot per head
+constexpr int kNormSlots = 4;         // per-thread ring of key norms (tile k is read at k + 2)
+constexpr int kBBytesMax = 32 * kK;   // one B buffer at most: 8 queries x 4 digit rows x K bytes
+
+// launch shape for NQ query columns per KV head (G <= NQ)
+template <int NQ>
+struct Cfg {
+    static constexpr int N = 4 * NQ;                  // B rows = D columns
+    static constexpr int S = (NQ <= 4) ? 3 : 2;       // tile streams
+    static constexpr int kWorkerWarps = 4 * S;
+    static constexpr int kWarpTma = kWorkerWarps;
+    static constexpr int kWarpMma0 = kWorkerWarps + 1;
+    static constexpr int kThreads = (kWorkerWarps + 1 + S) * 32;
+    static constexpr int kDOff = S * 2 * kACols;      // A buffers first, then D buffers
+    static constexpr int kBBytes = N * kK;
+    static_assert(kStages % S == 0, "streams must own whole stages");
+    static_assert(kDOff + S * 2 * N <= kTmemCols, "tensor memory budget");
+    static_assert(kBBytes <= kBBytesMax, "B buffer");
+};
 
 __device__ unsigned int g_status;
 
@@ -85,7 +92,6 @@ struct Lookup {
     static constexpr int C = (B >= 3) ? 2 : 4;
     static constexpr int FB = C * B;              // 8, 6, 8, 4
     static constexpr int EB = 2 * C;              // entry bytes: C hi digits, C lo digits
-    static constexpr int NL = kD / C;             // lookups per row
     static constexpr int NF = 1 << FB;            // table fields
 };
 
@@ -106,19 +112,19 @@ struct TcParams {
     int8_t lo[kMaxLevels];
 };
 
+constexpr int kMaxStreams = 3;
 struct Smem {
     uint64_t full[kStages], empty[kStages];
-    // per stream and A buffer: A written (decoders), products done (A free)
-    uint64_t a_full[kStreams][2], mma_done[kStreams][2];
-    // per stream and D buffer: sums ready (MMA commit), sums read (output threads)
-    uint64_t d_full[kStreams][kDBufs], d_empty[kStreams][kDBufs];
-    uint64_t drain[kStreams];
-    uint64_t wsync[kStreams];          // the threads of one stream (query rotation steps)
+    // per stream and buffer: A written (workers); products done (one commit: A
+    // may be overwritten, D may be read)
+    uint64_t a_full[kMaxStreams][2], mma_done[kMaxStreams][2];
+    uint64_t drain[kMaxStreams];
+    uint64_t wsync[kMaxStreams];       // the threads of one stream (query rotation steps)
     uint32_t tmem_base;
-    float inv[kStreams][kInvSlots][8]; // per stream, head slot and query: 1 / (128 * S_q * S_c)
-    float q[kStreams][8][kD];          // rotation scratch
-    float qmax[kStreams][4][8];        // per stream warp and query: max |q''|
-    float norm_ring[kNormAhead + 2][kTileRows];   // key norms, kNormAhead tiles ahead
+    float inv[kMaxStreams][kInvSlots][8];   // per stream, head slot and query: 1 / (128 * S_q * S_c)
+    float q[2048];                           // rotation scratch: S * NQ <= 16 query rows of d floats
+    float qmax[kMaxStreams][4][8];           // per stream, warp and query: max |q''|
+    float norm_ring[kMaxStreams][kNormSlots][kTileRows];
 };
 constexpr int kSmemBook = 16384;
 static_assert(sizeof(Smem) <= kSmemBook, "bookkeeping area too small");
@@ -155,7 +161,7 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
 {
     using LK = Lookup<B>;
     const int tid = threadIdx.x & (kGroupThreads - 1);
-    float(*q)[kD] = S.q[g];
+    float(*q)[kD] = reinterpret_cast<float(*)[kD]>(S.q + g * NQ * kD);
     const float sg = p.signs[tid] < 0 ? -1.0f : 1.0f;
 #pragma unroll
     for (int qi = 0; qi < NQ; ++qi)
@@ -218,12 +224,11 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
 
 // table entry of one field value: C hi digits then C lo digits, replicated for
 // the 32 lanes (entry (field, lane) at field * 256 + lane * EB)
-template <int B>
+template <int B, int kWorkers>
 __device__ void build_lut(const TcParams &p, uint8_t *lut)
 {
     using LK = Lookup<B>;
     constexpr uint32_t mask = (1u << B) - 1u;
-    constexpr int kWorkers = kWorkWarps * 32;    // every worker thread helps
     for (int e = threadIdx.x; e < LK::NF * 32; e += kWorkers) {
         const int field = e / 32, ln = e % 32;
         uint8_t bytes[LK::EB];
@@ -278,35 +283,76 @@ __device__ __forceinline__ uint32_t lut_addr(const uint32_t *w, int l, uint32_t 
 // Dynamic shared memory: the table on a 64 KB boundary of the shared window
 // (so one PRMT forms a full address), the rest below it when the gap is large
 // enough, else after it.
-constexpr int kRestBytes = kStages * kStageBytes + kStreams * 2 * kBBytesMax + kSmemBook;
+constexpr int kBRegion = 32768;       // two B buffers per stream, for every stream
+constexpr int kRestBytes = kStages * kStageBytes + kBRegion + kSmemBook;
 constexpr size_t kSmemRequest = 1024 + 65536 + kLutBytes + kRestBytes;
 static_assert(kSmemRequest <= 232448, "shared memory per block");
+static_assert(Cfg<8>::S * 2 * Cfg<8>::kBBytes <= kBRegion && Cfg<4>::S * 2 * Cfg<4>::kBBytes <= kBRegion,
+              "B buffers of every stream fit");
 
-// Decoder threads of tile stream g (local tiles g, g+2, ...): one thread per
-// key, packed row -> table lookups -> A in tensor memory.  They also rotate the
-// queries of every new KV head into the stream's B buffers.
+// Worker threads of tile stream g (local tiles k = 0, 1, ... are the CTA's
+// tiles t0 + g + S*k): one thread per key of a tile.
 template <int B, int NQ>
-struct Decoder {
+struct Worker {
     using LK = Lookup<B>;
+    using C = Cfg<NQ>;
     static constexpr int P = kD * B / 8;
     static constexpr int NW = P / 4;
+
+    // int32 digit sums of one key -> sum_j q''_j c_j * 128 * S_q * S_c per query
+    static __device__ __forceinline__ void load_sums(uint32_t taddr, float (&sc)[NQ])
+    {
+#pragma unroll
+        for (int c = 0; c < C::N / 16; ++c) {
+            uint32_t acc[16];
+            tmem_ld16(taddr + 16 * c, acc);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                sc[4 * c + e] = fmaf(128.0f, __int2float_rn(static_cast<int>(acc[4 * e])),
+                                     fmaf(1.0f / 16384.0f, __int2float_rn(static_cast<int>(acc[4 * e + 3])),
+                                          fmaf(1.0f / 128.0f, __int2float_rn(static_cast<int>(acc[4 * e + 2])),
+                                               __int2float_rn(static_cast<int>(acc[4 * e + 1])))));
+        }
+    }
+
+    // scores of this thread's key in a finished tile: D of buffer `ab`, key
+    // norm from ring slot `slot`, query scales from head slot `hslot`
+    static __device__ __forceinline__ void emit(const TcParams &p, const Smem &S, int g, uint32_t tmem_lane,
+                                                int ab, int slot, int hslot, int h, int t, int r)
+    {
+        float sc[NQ];
+        load_sums(tmem_lane + C::kDOff + (2 * g + ab) * C::N, sc);
+        const float nk = S.norm_ring[g][slot][r];
+        if (t < p.n) {
+#pragma unroll
+            for (int qi = 0; qi < NQ; ++qi)
+                if (qi < p.group)
+                    __stcs(p.scores + (static_cast<int64_t>(h) * p.group + qi) * p.n + t,
+                           nk * S.inv[g][hslot][qi] * sc[qi]);
+        }
+    }
 
     static __device__ void run(const TcParams &p, Smem &S, int g, uint8_t *sStage, uint8_t *sB, uint32_t lut_base,
                                uint32_t tmem, int t0, int t1)
     {
         const int lane = threadIdx.x & 31;
         const int r = threadIdx.x & (kGroupThreads - 1);   // key within the tile = tensor-memory lane
-        const uint32_t lane_base = static_cast<uint32_t>(r & ~31) << 16;
+        const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(r & ~31) << 16);
         const uint32_t base_lane = lut_base | static_cast<uint32_t>(lane * LK::EB);
+        const uint32_t ring = smem_u32(&S.norm_ring[g][0][r]);
         int bsel = -1, prev_h = -1, hc = -1, sync_phase = 0;
         int h = (t0 + g) / p.tiles_per_head, ti = (t0 + g) - h * p.tiles_per_head;
+        // (head, key offset, head slot) of tiles k - 1 and k - 2, whose scores are still due
+        int h1 = 0, t1k = 0, hs1 = 0, h2 = 0, t2k = 0, hs2 = 0;
         int s = g, k = 0;
         uint32_t sph = 0;
+        bool ok = true;
 
-        for (int tile = t0 + g; tile < t1; tile += kStreams, ++k) {
+        for (int tile = t0 + g; tile < t1; tile += C::S, ++k) {
             if (!mbar_wait_warp(smem_u32(&S.full[s]), sph)) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutLoad);
-                return;
+                ok = false;
+                break;
             }
             uint32_t w[NW + 1];
             {
@@ -319,27 +365,38 @@ struct Decoder {
                 w[NW] = 0;
             }
             mbar_arrive(smem_u32(&S.empty[s]));
+            // this tile's key norm, read two tiles from now
+            cp_async_4(ring + (k & (kNormSlots - 1)) * (kTileRows * 4),
+                       p.norms + static_cast<int64_t>(h) * p.n + min(ti * kTileRows + r, p.n - 1));
+            cp_async_commit();
 
-            // the products of this stream's tile k - 2 are done, so its A buffer
-            // and the B buffer of two heads back are free
+            // products of tile k - 2 done: its D is readable, its A buffer and the
+            // B buffer of two heads back are free
             const int ab = k & 1;
             if (!mbar_wait_warp(smem_u32(&S.mma_done[g][ab]), ((k >> 1) & 1) ^ 1)) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                return;
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            if (k >= 2) {
+                cp_async_wait<2>();          // the norm copy of tile k - 2 has landed
+                emit(p, S, g, tmem_lane, ab, (k - 2) & (kNormSlots - 1), hs2, h2, t2k + r, r);
             }
 
             if (h != prev_h) {
                 bsel = (bsel < 0) ? 0 : (bsel ^ 1);
                 prev_h = h;
                 ++hc;
-                if (!build_b<B, NQ>(p, S, g, sB + (2 * g + bsel) * kBBytesMax, S.inv[g][hc & (kInvSlots - 1)], h,
+                if (!build_b<B, NQ>(p, S, g, sB + (2 * g + bsel) * C::kBBytes, S.inv[g][hc & (kInvSlots - 1)], h,
                                     sync_phase)) {
                     if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
-                    return;
+                    ok = false;
+                    break;
                 }
             }
-            tc_fence_after_sync();
-            const uint32_t a_addr = tmem + lane_base + (2 * g + ab) * kACols;
+
+            const uint32_t a_addr = tmem_lane + (2 * g + ab) * kACols;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t a[32];
@@ -362,157 +419,44 @@ struct Decoder {
             tc_fence_before_sync();
             mbar_arrive(smem_u32(&S.a_full[g][ab]));
 
-            s += kStreams;
+            h2 = h1; t2k = t1k; hs2 = hs1;
+            h1 = h; t1k = ti * kTileRows; hs1 = hc & (kInvSlots - 1);
+            s += C::S;
             if (s >= kStages) {
                 s -= kStages;
                 sph ^= 1;
             }
-            ti += kStreams;
+            ti += C::S;
             while (ti >= p.tiles_per_head) {
                 ti -= p.tiles_per_head;
                 ++h;
             }
         }
-    }
-};
 
-// Output threads (one warp per lane quadrant): the int32 sums -> scores of the
-// keys of every tile of the range, for every query of the head.  Each pass
-// takes the two streams' tiles 2m and 2m+1 together, so the waits and tensor
-// memory loads of the pair overlap.
-// The key norms arrive kNormAhead tiles early through per-thread asynchronous
-// copies into a ring in shared memory; each thread reads only the slots it
-// filled itself, so its own commit groups order the reads and no barrier is
-// needed.  (A norm fetched only one tile ahead leaves the whole pipeline
-// waiting on one HBM round trip per tile.)
-template <int NQ>
-struct Output {
-    static constexpr int N = 4 * NQ;
-    static constexpr int kSlots = kNormAhead + 2;
-
-    // int32 digit sums of one key -> sum_j q''_j c_j * 128 * S_q * S_c per query
-    static __device__ __forceinline__ void load_sums(uint32_t taddr, float (&sc)[NQ])
-    {
-#pragma unroll
-        for (int c = 0; c < N / 16; ++c) {
-            uint32_t acc[16];
-            tmem_ld16(taddr + 16 * c, acc);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                sc[4 * c + e] = fmaf(128.0f, __int2float_rn(static_cast<int>(acc[4 * e])),
-                                     fmaf(1.0f / 16384.0f, __int2float_rn(static_cast<int>(acc[4 * e + 3])),
-                                          fmaf(1.0f / 128.0f, __int2float_rn(static_cast<int>(acc[4 * e + 2])),
-                                               __int2float_rn(static_cast<int>(acc[4 * e + 1])))));
-        }
-    }
-
-    static __device__ __forceinline__ void store(const TcParams &p, int h, int t, float nk, const float (&inv)[NQ],
-                                                 const float (&sc)[NQ])
-    {
-        if (t < p.n) {
-#pragma unroll
-            for (int qi = 0; qi < NQ; ++qi)
-                if (qi < p.group)
-                    __stcs(p.scores + (static_cast<int64_t>(h) * p.group + qi) * p.n + t, nk * inv[qi] * sc[qi]);
-        }
-    }
-
-    static __device__ void run(const TcParams &p, Smem &S, uint32_t tmem, int t0, int t1)
-    {
-        static_assert(kStreams == 2, "tiles are taken in pairs, one per stream");
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-        const int quad = warp & 3;
-        const int r = quad * 32 + lane;
-        const uint32_t dbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + kDOff;
-        int hc0 = -1, hc1 = -1, prev_h0 = -1, prev_h1 = -1;   // per stream: heads seen, last head
-        int h = t0 / p.tiles_per_head, ti = t0 - h * p.tiles_per_head;
-
-        // prefetch cursor: (head, tile in head) of the next tile whose norms to fetch
-        int hp = h, tip = ti;
-        const uint32_t ring = smem_u32(&S.norm_ring[0][r]);
-        int ws = 0;
-        auto prefetch = [&](bool valid) {
-            if (valid)
-                cp_async_4(ring + ws * (kTileRows * 4),
-                           p.norms + static_cast<int64_t>(hp) * p.n + min(tip * kTileRows + r, p.n - 1));
-            cp_async_commit();
-            ws = (ws == kSlots - 1) ? 0 : ws + 1;
-            if (++tip == p.tiles_per_head) {
-                tip = 0;
-                ++hp;
+        // the last two tiles' scores
+        if (ok) {
+            cp_async_wait<0>();
+            for (int j = (k >= 2 ? k - 2 : 0); j < k; ++j) {
+                const bool last = (j == k - 1);
+                if (!mbar_wait_warp(smem_u32(&S.mma_done[g][j & 1]), (j >> 1) & 1)) {
+                    if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                    break;
+                }
+                tc_fence_after_sync();
+                emit(p, S, g, tmem_lane, j & 1, j & (kNormSlots - 1), last ? hs1 : hs2, last ? h1 : h2,
+                     (last ? t1k : t2k) + r, r);
             }
-        };
-#pragma unroll 1
-        for (int j = 0; j < kNormAhead; ++j) prefetch(t0 + j < t1);
-        int rs = 0;                        // ring slot of tile `tile`
-
-        for (int tile = t0, k = 0; tile < t1; tile += 2, ++k) {
-            const bool two = tile + 1 < t1;
-            const int dk = k & (kDBufs - 1);
-            const uint32_t ph = (k / kDBufs) & 1;
-            // heads of the pair and the B buffers (query scales) they use
-            const int h0 = h, i0 = ti;
-            if (++ti == p.tiles_per_head) {
-                ti = 0;
-                ++h;
-            }
-            const int h1 = h, i1 = ti;
-            if (++ti == p.tiles_per_head) {
-                ti = 0;
-                ++h;
-            }
-            if (h0 != prev_h0) {
-                ++hc0;
-                prev_h0 = h0;
-            }
-            if (two && h1 != prev_h1) {
-                ++hc1;
-                prev_h1 = h1;
-            }
-
-            // the pair's norms (slots rs, rs + 1); copies of later tiles may still fly
-            cp_async_wait<kNormAhead - 2>();
-            const float nk0 = S.norm_ring[rs][r];
-            const int rs1 = (rs == kSlots - 1) ? 0 : rs + 1;
-            const float nk1 = S.norm_ring[rs1][r];
-            rs = (rs1 == kSlots - 1) ? 0 : rs1 + 1;
-            prefetch(tile + kNormAhead < t1);
-            prefetch(tile + 1 + kNormAhead < t1);
-
-            if (!mbar_wait_warp(smem_u32(&S.d_full[0][dk]), ph) ||
-                (two && !mbar_wait_warp(smem_u32(&S.d_full[1][dk]), ph))) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                break;
-            }
-            tc_fence_after_sync();
-            float sc0[NQ], sc1[NQ];
-            load_sums(dbase + dk * kNMax, sc0);
-            if (two) load_sums(dbase + (kDBufs + dk) * kNMax, sc1);
-            // the query scales of the pair's heads, read before D is released
-            // (the release lets the decoders reuse a head slot kInvSlots heads on)
-            float inv0[NQ], inv1[NQ];
-#pragma unroll
-            for (int qi = 0; qi < NQ; ++qi) {
-                inv0[qi] = S.inv[0][hc0 & (kInvSlots - 1)][qi];
-                inv1[qi] = S.inv[1][hc1 & (kInvSlots - 1)][qi];
-            }
-            tc_fence_before_sync();
-            mbar_arrive(smem_u32(&S.d_empty[0][dk]));
-            if (two) mbar_arrive(smem_u32(&S.d_empty[1][dk]));
-            store(p, h0, i0 * kTileRows + r, nk0, inv0, sc0);
-            if (two) store(p, h1, i1 * kTileRows + r, nk1, inv1, sc1);
         }
         cp_async_wait<0>();
     }
 };
 
 template <int B, int NQ>
-__global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_constant__ TcParams p)
+__global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const __grid_constant__ TcParams p)
 {
     using LK = Lookup<B>;
+    using C = Cfg<NQ>;
     constexpr int P = kD * B / 8;
-    constexpr int N = 4 * NQ;
-    static_assert(N <= kNMax && N * kK <= kBBytesMax, "B buffer too small for N");
     static_assert(kTileRows * P <= kStageBytes, "stage too small for a tile of packed rows");
     static_assert(LK::NF * 256 <= kLutBytes, "lookup table too large");
     extern __shared__ uint8_t smem_raw[];
@@ -523,8 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
     const uint32_t rest_pos = rest_first ? base1k : lut_pos + kLutBytes;
     uint8_t *sLut = smem_raw + (lut_pos - raw);
     uint8_t *sStage = smem_raw + (rest_pos - raw);                  // kStages x 8 KB
-    uint8_t *sB = sStage + kStages * kStageBytes;                    // streams x 2 x 8 KB
-    Smem &S = *reinterpret_cast<Smem *>(sB + kStreams * 2 * kBBytesMax);
+    uint8_t *sB = sStage + kStages * kStageBytes;                    // S streams x 2 B buffers
+    Smem &S = *reinterpret_cast<Smem *>(sB + kBRegion);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -536,22 +480,18 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
             mbar_init(smem_u32(&S.full[s]), 1);
             mbar_init(smem_u32(&S.empty[s]), kGroupThreads);     // consumed by one stream
         }
-        for (int g = 0; g < kStreams; ++g) {
+        for (int g = 0; g < C::S; ++g) {
             for (int a = 0; a < 2; ++a) {
                 mbar_init(smem_u32(&S.a_full[g][a]), kGroupThreads);
                 mbar_init(smem_u32(&S.mma_done[g][a]), 1);
             }
-            for (int a = 0; a < kDBufs; ++a) {
-                mbar_init(smem_u32(&S.d_full[g][a]), 1);
-                mbar_init(smem_u32(&S.d_empty[g][a]), kOutWarps * 32);
-            }
             mbar_init(smem_u32(&S.wsync[g]), kGroupThreads);
+            mbar_init(smem_u32(&S.drain[g]), 1);
         }
-        for (int g = 0; g < kStreams; ++g) mbar_init(smem_u32(&S.drain[g]), 1);
         fence_mbar_init();
     }
-    if (warp == kWarpTma && lane == 0) prefetch_tensormap(&p.tmap);
-    if (warp < kWorkWarps) build_lut<B>(p, sLut);
+    if (warp == C::kWarpTma && lane == 0) prefetch_tensormap(&p.tmap);
+    if (warp < C::kWorkerWarps) build_lut<B, C::kWorkerWarps * 32>(p, sLut);
     if (warp == 0) {
         tmem_alloc(smem_u32(&S.tmem_base), kTmemCols);
         tmem_relinquish();
@@ -561,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
     tc_fence_after_sync();
     const uint32_t tmem = S.tmem_base;
 
-    if (warp == kWarpTma) {
+    if (warp == C::kWarpTma) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
             int it = 0, s = 0;
@@ -584,48 +524,45 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
                     ++h;
                 }
             }
+            // every load issued has landed before the CTA may exit
             for (int k = 0; k < kStages && k < it; ++k) {
                 const int j = it - 1 - k;
                 mbar_wait(smem_u32(&S.full[j % kStages]), (j / kStages) & 1);
             }
         }
-    } else if (warp >= kWarpMma0) {
+    } else if (warp >= C::kWarpMma0) {
         // ------------------------------------------------- MMA, one per stream
         if (lane == 0) {
-            const int g = warp - kWarpMma0;
-            const uint32_t id = idesc(kAccS32, kFmtS8, kFmtS8, 128, N);
-            const uint32_t b0 = smem_u32(sB) + 2 * g * kBBytesMax;
+            const int g = warp - C::kWarpMma0;
+            const uint32_t id = idesc(kAccS32, kFmtS8, kFmtS8, 128, C::N);
+            const uint32_t b0 = smem_u32(sB) + 2 * g * C::kBBytes;
             const uint32_t a0 = tmem + 2 * g * kACols;
-            const uint32_t d0 = tmem + kDOff + g * kDBufs * kNMax;
+            const uint32_t d0 = tmem + C::kDOff + 2 * g * C::N;
             // the stream's B buffer flips whenever its tiles enter a new head,
-            // exactly as the decoders flip it
+            // exactly as the workers flip it
             int bsel = 1, prev_h = -1;
             int h = (t0 + g) / p.tiles_per_head, ti = (t0 + g) - h * p.tiles_per_head;
             int k = 0;
-            for (int tile = t0 + g; tile < t1; tile += kStreams, ++k) {
+            for (int tile = t0 + g; tile < t1; tile += C::S, ++k) {
                 if (h != prev_h) {
                     bsel ^= 1;
                     prev_h = h;
                 }
-                const int ab = k & 1, dk = k & (kDBufs - 1);
-                // A of this tile written, and the sums of tile k - kDBufs read out of D
+                const int ab = k & 1;
+                // A of this tile written (which also means the workers have read
+                // the D of tile k - 2 out of this buffer)
                 if (!mbar_wait(smem_u32(&S.a_full[g][ab]), (k >> 1) & 1)) {
                     atomicOr(&g_status, kErrTimeoutLoad);
                     break;
                 }
-                if (!mbar_wait(smem_u32(&S.d_empty[g][dk]), ((k / kDBufs) & 1) ^ 1)) {
-                    atomicOr(&g_status, kErrTimeoutDrain);
-                    break;
-                }
                 tc_fence_after_sync();
                 // K step kk reads B 256 bytes further on: +16 in the address field
-                const uint64_t bd = desc_k_interleave(b0 + bsel * kBBytesMax, 128, (kK / 16) * 128);
-                const uint32_t d = d0 + dk * kNMax, a = a0 + ab * kACols;
+                const uint64_t bd = desc_k_interleave(b0 + bsel * C::kBBytes, 128, (kK / 16) * 128);
+                const uint32_t d = d0 + ab * C::N, a = a0 + ab * kACols;
 #pragma unroll
                 for (int kk = 0; kk < kK / 32; ++kk) mma_i8_ts(d, a + 8 * kk, bd + 16 * kk, id, kk > 0);
                 mma_commit(smem_u32(&S.mma_done[g][ab]));
-                mma_commit(smem_u32(&S.d_full[g][dk]));
-                ti += kStreams;
+                ti += C::S;
                 while (ti >= p.tiles_per_head) {
                     ti -= p.tiles_per_head;
                     ++h;
@@ -635,9 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
             mbar_wait(smem_u32(&S.drain[g]), 0);
         }
     } else {
-        // ------------------------------------------------------------ workers
-        if (warp < kDecodeWarps) Decoder<B, NQ>::run(p, S, warp / 4, sStage, sB, lut_pos, tmem, t0, t1);
-        else Output<NQ>::run(p, S, tmem, t0, t1);
+        // ----------------------------------------------------------- workers
+        Worker<B, NQ>::run(p, S, warp / 4, sStage, sB, lut_pos, tmem, t0, t1);
     }
 
     tc_fence_before_sync();
@@ -720,7 +656,7 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
         p.lo[i] = static_cast<int8_t>(vi - 128 * hi);
     }
     const int used = (p.total_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
-    kernel<<<used, kThreads, smem, stream>>>(p);
+    kernel<<<used, Cfg<NQ>::kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -761,3 +697,4 @@ unsigned int scores_tc_status(bool clear)
 }
 
 }  // namespace axr
+

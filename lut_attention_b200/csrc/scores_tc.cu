@@ -299,37 +299,49 @@ struct Worker {
     static constexpr int P = kD * B / 8;
     static constexpr int NW = P / 4;
 
-    // int32 digit sums of one key -> sum_j q''_j c_j * 128 * S_q * S_c per query
-    static __device__ __forceinline__ void load_sums(uint32_t taddr, float (&sc)[NQ])
+    static constexpr int NL = C::N / 16;      // 16-column loads of one D buffer
+
+    // scores of this thread's key from its int32 digit sums.  D columns 4q .. 4q+3
+    // of query q carry weights 128, 1, 1/128, 1/128^2; the pairs are joined in
+    // int32 first (|128 c0 + c1| < 1.4e8, |128 c2 + c3| < 2.1e8), so two
+    // conversions serve a query.  The key norm is in ring slot `slot`; the
+    // query scales of the stream's head number `hc` (slot hc mod kInvSlots) are
+    // kept in `inv` while that head lasts.
+    static __device__ __forceinline__ void store_sums(const TcParams &p, const Smem &S, int g,
+                                                      const uint32_t (&acc)[NL][16], int slot, int hc, int h,
+                                                      int t, int r, int &inv_hc, float (&inv)[NQ])
     {
+        if (hc != inv_hc) {
+            inv_hc = hc;
 #pragma unroll
-        for (int c = 0; c < C::N / 16; ++c) {
-            uint32_t acc[16];
-            tmem_ld16(taddr + 16 * c, acc);
+            for (int qi = 0; qi < NQ; ++qi) inv[qi] = S.inv[g][hc & (kInvSlots - 1)][qi];
+        }
+        const float nk = S.norm_ring[g][slot][r];
+        if (t < p.n) {
+            float *dst = p.scores + static_cast<int64_t>(h) * p.group * p.n + t;
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                sc[4 * c + e] = fmaf(128.0f, __int2float_rn(static_cast<int>(acc[4 * e])),
-                                     fmaf(1.0f / 16384.0f, __int2float_rn(static_cast<int>(acc[4 * e + 3])),
-                                          fmaf(1.0f / 128.0f, __int2float_rn(static_cast<int>(acc[4 * e + 2])),
-                                               __int2float_rn(static_cast<int>(acc[4 * e + 1])))));
+            for (int qi = 0; qi < NQ; ++qi) {
+                const int *x = reinterpret_cast<const int *>(&acc[qi / 4][4 * (qi % 4)]);
+                const float hi = __int2float_rn(x[0] * 128 + x[1]);
+                const float lo = __int2float_rn(x[2] * 128 + x[3]);
+                if (qi < p.group) {
+                    __stcs(dst, nk * inv[qi] * fmaf(lo, 1.0f / 16384.0f, hi));
+                    dst += p.n;
+                }
+            }
         }
     }
 
-    // scores of this thread's key in a finished tile: D of buffer `ab`, key
-    // norm from ring slot `slot`, query scales from head slot `hslot`
-    static __device__ __forceinline__ void emit(const TcParams &p, const Smem &S, int g, uint32_t tmem_lane,
-                                                int ab, int slot, int hslot, int h, int t, int r)
+    static __device__ __forceinline__ void load_issue(uint32_t taddr, uint32_t (&acc)[NL][16])
     {
-        float sc[NQ];
-        load_sums(tmem_lane + C::kDOff + (2 * g + ab) * C::N, sc);
-        const float nk = S.norm_ring[g][slot][r];
-        if (t < p.n) {
 #pragma unroll
-            for (int qi = 0; qi < NQ; ++qi)
-                if (qi < p.group)
-                    __stcs(p.scores + (static_cast<int64_t>(h) * p.group + qi) * p.n + t,
-                           nk * S.inv[g][hslot][qi] * sc[qi]);
-        }
+        for (int c = 0; c < NL; ++c) tmem_ld16_issue(taddr + 16 * c, acc[c]);
+    }
+
+    static __device__ __forceinline__ void load_wait(uint32_t (&acc)[NL][16])
+    {
+#pragma unroll
+        for (int c = 0; c < NL; ++c) tmem_wait_ld_pass(acc[c]);
     }
 
     static __device__ void run(const TcParams &p, Smem &S, int g, uint8_t *sStage, uint8_t *sB, uint32_t lut_base,
@@ -342,11 +354,14 @@ struct Worker {
         const uint32_t ring = smem_u32(&S.norm_ring[g][0][r]);
         int bsel = -1, prev_h = -1, hc = -1, sync_phase = 0;
         int h = (t0 + g) / p.tiles_per_head, ti = (t0 + g) - h * p.tiles_per_head;
-        // (head, key offset, head slot) of tiles k - 1 and k - 2, whose scores are still due
+        // (head, key offset, stream head number) of tiles k - 1 and k - 2, whose scores are still due
         int h1 = 0, t1k = 0, hs1 = 0, h2 = 0, t2k = 0, hs2 = 0;
         int s = g, k = 0;
         uint32_t sph = 0;
         bool ok = true;
+        uint32_t acc[NL][16] = {};          // sums of tile k - 2, loaded while tile k decodes
+        int inv_hc = -1;                    // head number whose query scales `inv` holds
+        float inv[NQ];
 
         for (int tile = t0 + g; tile < t1; tile += C::S, ++k) {
             if (!mbar_wait_warp(smem_u32(&S.full[s]), sph)) {
@@ -379,10 +394,7 @@ struct Worker {
                 break;
             }
             tc_fence_after_sync();
-            if (k >= 2) {
-                cp_async_wait<2>();          // the norm copy of tile k - 2 has landed
-                emit(p, S, g, tmem_lane, ab, (k - 2) & (kNormSlots - 1), hs2, h2, t2k + r, r);
-            }
+            if (k >= 2) load_issue(tmem_lane + C::kDOff + (2 * g + ab) * C::N, acc);
 
             if (h != prev_h) {
                 bsel = (bsel < 0) ? 0 : (bsel ^ 1);
@@ -396,31 +408,39 @@ struct Worker {
                 }
             }
 
+            // lookup l fills A columns l (4-byte entries) or 2l, 2l+1 (8-byte entries)
             const uint32_t a_addr = tmem_lane + (2 * g + ab) * kACols;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t a[32];
+            for (int qt = 0; qt < 4; ++qt) {
+                uint32_t a[16];
                 if constexpr (LK::EB == 4) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const uint32_t ad = lut_addr<B>(w, 32 * half + i, base_lane);
+                    for (int i = 0; i < 16; ++i) {
+                        const uint32_t ad = lut_addr<B>(w, 16 * qt + i, base_lane);
                         asm("ld.shared.u32 %0, [%1];" : "=r"(a[i]) : "r"(ad));
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint32_t ad = lut_addr<B>(w, 16 * half + i, base_lane);
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t ad = lut_addr<B>(w, 8 * qt + i, base_lane);
                         asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a[2 * i]), "=r"(a[2 * i + 1]) : "r"(ad));
                     }
                 }
-                tmem_st32(a_addr + 32 * half, a);
+                tmem_st16(a_addr + 16 * qt, a);
             }
             tmem_wait_st();
+            // the products of tile k overwrite D of tile k - 2: its sums must be in
+            // registers before A is published
+            if (k >= 2) load_wait(acc);
             tc_fence_before_sync();
             mbar_arrive(smem_u32(&S.a_full[g][ab]));
+            if (k >= 2) {
+                cp_async_wait<2>();          // the norm copy of tile k - 2 has landed
+                store_sums(p, S, g, acc, (k - 2) & (kNormSlots - 1), hs2, h2, t2k + r, r, inv_hc, inv);
+            }
 
             h2 = h1; t2k = t1k; hs2 = hs1;
-            h1 = h; t1k = ti * kTileRows; hs1 = hc & (kInvSlots - 1);
+            h1 = h; t1k = ti * kTileRows; hs1 = hc;
             s += C::S;
             if (s >= kStages) {
                 s -= kStages;
@@ -443,8 +463,10 @@ struct Worker {
                     break;
                 }
                 tc_fence_after_sync();
-                emit(p, S, g, tmem_lane, j & 1, j & (kNormSlots - 1), last ? hs1 : hs2, last ? h1 : h2,
-                     (last ? t1k : t2k) + r, r);
+                load_issue(tmem_lane + C::kDOff + (2 * g + (j & 1)) * C::N, acc);
+                load_wait(acc);
+                store_sums(p, S, g, acc, j & (kNormSlots - 1), last ? hs1 : hs2, last ? h1 : h2,
+                           (last ? t1k : t2k) + r, r, inv_hc, inv);
             }
         }
         cp_async_wait<0>();

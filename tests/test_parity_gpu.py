@@ -81,11 +81,14 @@ def test_scores_parity_groups_and_query_dtypes(group, qdtype):
 
 
 @pytest.mark.parametrize("b", [2, 3, 4])
-@pytest.mark.parametrize("heads,n,group", [(64, 3001, 4), (50, 100, 2), (3, 131, 8), (200, 77, 1)])
+@pytest.mark.parametrize("heads,n,group", [(64, 3001, 4), (50, 100, 2), (3, 131, 8), (200, 77, 1),
+                                           (4096, 100, 4), (3000, 64, 8)])
 def test_scores_tile_ranges_cross_heads(heads, n, group, b):
     """d = 128 reads run on the tensor-core kernel, whose CTAs walk contiguous
     ranges of 128-key tiles: ranges cross KV heads (the query digits are rebuilt
-    mid-range) and, for n < 128, one tile spans several heads."""
+    mid-range) and, for n < 128, every tile is a head of its own.  The last two
+    shapes give each CTA about 28 and 21 such tiles, so every tile stream passes
+    through more heads than the kernel keeps query scales for at once."""
     d = 128
     packed, norms = workloads.make_random_packed(heads, n, d, b, seed=heads + n + b, device=DEV)
     wl = workloads.GQA_DECODE_128K.with_(batch=1, kv_heads=heads, group=group, T=n)

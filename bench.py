@@ -92,6 +92,14 @@ def kernel_source_hash(name: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+def kernel_file(kind: str, wl: workloads.Workload) -> str:
+    """Source file of the kernel the library runs for this workload (api.cu takes the
+    tensor-core kernels at d = 128, for the write path with bf16/f16 keys)."""
+    if kind == "quantize_keys":
+        return "quantize_keys_tc.cu" if wl.d == 128 and wl.dtype in ("bf16", "f16") else "quantize_keys.cu"
+    return "scores_tc.cu" if wl.d == 128 else "scores.cu"
+
+
 def profiled_traffic(kernel_file: str, workload: str, b: int):
     """DRAM bytes per launch from the committed ncu summary, when that summary was
     taken on the current kernel source (its hash line matches); else None."""
@@ -403,7 +411,7 @@ def main():
     }
     dominant = "quantize_keys" if t_write >= t_read else "scores"
     dk = kernels[dominant]
-    src = "quantize_keys.cu" if dominant == "quantize_keys" else "scores.cu"
+    src = kernel_file(dominant, wl)
     line = {
         "metric": "lut_attention_scores_per_s",
         "value": scores_per_step / (ms_per_step * 1e-3),
@@ -420,7 +428,7 @@ def main():
         "config": config_dict(wl, world),
         "keys_per_s": keys_per_step / (ms_per_step * 1e-3),
         "kernels": kernels,
-        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dk["gbs"], "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": dominant, "source": src, "achieved": dk["gbs"], "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": dk["gbs"] / peak,
                      "frac_of_8tbs": dk["gbs"] / NOMINAL_HBM_GBS,
                      "traffic": profiled_traffic(src, wl.name, wl.b)},

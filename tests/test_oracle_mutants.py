@@ -1,0 +1,134 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the oracle's C source (on the CPU,
+in a temporary directory), builds it as a separate module, and runs the pins of
+test_oracle_pins.py against it: at least one pin must fail.  An unmodified copy
+must pass them all, which shows the harness itself is sound.
+"""
+import importlib.util
+import os
+import shutil
+import sys
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ORACLE_DIR = os.path.join(os.path.dirname(HERE), "oracle")
+
+
+def _load_pins():
+    spec = importlib.util.spec_from_file_location("oracle_pins_for_mutants",
+                                                  os.path.join(HERE, "test_oracle_pins.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+PINS = _load_pins()
+
+# (pin, keyword arguments): one representative parameter set per pin
+PIN_CALLS = [
+    ("test_hadamard_sylvester_recursion_and_scipy", {}),
+    ("test_rotation_is_orthonormal_hadamard_times_signs", {"d": 64}),
+    ("test_rotation_rejects_bad_signs", {}),
+    ("test_lloyd_max_one_bit_closed_form", {}),
+    ("test_lloyd_max_conditions_by_quadrature", {"b": 3}),
+    ("test_lloyd_max_matches_classical_table_and_is_a_minimum", {"b": 4}),
+    ("test_codebook_scaling_symmetry_and_boundaries", {"d": 128, "b": 3}),
+    ("test_codebook_is_data_independent", {}),
+    ("test_packing_hand_worked_examples", {}),
+    ("test_pack_roundtrip_and_bit_positions", {"d": 16, "b": 3}),
+    ("test_rotated_unit_keys_have_unit_norm_and_variance_one_over_d", {}),
+    ("test_basis_vector_closed_form", {"b": 2}),
+    ("test_zero_key", {}),
+    ("test_brute_force_nearest_codeword_d8", {"b": 2}),
+    ("test_quantization_mse_matches_lloyd_max", {"b": 4}),
+    ("test_margins_are_distances_to_decision_points", {}),
+    ("test_lut_scores_equal_dequantized_dot", {"d": 64, "b": 3, "group": 2}),
+    ("test_scores_brute_force_d8", {}),
+]
+
+# name -> (text in oracle.c, replacement): one plausible mistake each
+MUTANTS = {
+    "sign_flip_dropped": (
+        "R[(size_t)i * d + j] *= (double)signs[j] * inv_sqrt_d;",
+        "R[(size_t)i * d + j] *= inv_sqrt_d;"),
+    "signs_applied_to_rows": (
+        "R[(size_t)i * d + j] *= (double)signs[j] * inv_sqrt_d;",
+        "R[(size_t)i * d + j] *= (double)signs[i] * inv_sqrt_d;"),
+    "rotation_not_normalised": (
+        "R[(size_t)i * d + j] *= (double)signs[j] * inv_sqrt_d;",
+        "R[(size_t)i * d + j] *= (double)signs[j];"),
+    "codebook_scaled_by_1_over_d": (
+        "const double sigma = 1.0 / sqrt((double)d);",
+        "const double sigma = 1.0 / (double)d;"),
+    "centroid_rule_replaced_by_cell_midpoint": (
+        "next[i] = std_normal_conditional_mean(lo, hi);",
+        "next[i] = (i == 0) ? hi - 1.0 : (i == L - 1) ? lo + 1.0 : 0.5 * (lo + hi);"),
+    "ties_to_upper_index": (
+        "if (dist < best_dist) {",
+        "if (dist <= best_dist) {"),
+    "msb_first_packing": (
+        "if ((codes[j] >> i) & 1) row[bit / 8] |= (uint8_t)(1u << (bit % 8));",
+        "if ((codes[j] >> i) & 1) row[bit / 8] |= (uint8_t)(1u << (7 - bit % 8));"),
+    "temperature_dropped": (
+        "out[t] = (double)norms[(int64_t)h * n + t] * s * inv_sqrt_d;",
+        "out[t] = (double)norms[(int64_t)h * n + t] * s;"),
+    "query_reads_wrong_kv_head": (
+        "unpack_row(packed + ((int64_t)h * n + t) * P, d, b, codes);\n                double s = 0.0;",
+        "unpack_row(packed + ((int64_t)((h * group + g) % heads) * n + t) * P, d, b, codes);\n"
+        "                double s = 0.0;"),
+    "squared_norm_stored": (
+        "const float norm = (float)sqrt(ss);",
+        "const float norm = (float)ss;"),
+    "boundary_at_lower_centroid": (
+        "boundaries[i] = (float)(0.5 * ((double)centroids[i] + (double)centroids[i + 1]));",
+        "boundaries[i] = centroids[i];"),
+}
+
+# the MSB-first mutant changes packing on both sides, as a consistent mistake would
+UNPACK_MSB = ("v |= (unsigned)((row[bit / 8] >> (bit % 8)) & 1) << i;",
+              "v |= (unsigned)((row[bit / 8] >> (7 - bit % 8)) & 1) << i;")
+
+
+def _build_copy(tmp_path, name, edits):
+    pkg = tmp_path / f"oracle_{name}"
+    pkg.mkdir()
+    src = open(os.path.join(ORACLE_DIR, "oracle.c")).read()
+    for old, new in edits:
+        assert src.count(old) == 1, f"{name}: edit target not found once: {old}"
+        src = src.replace(old, new)
+    (pkg / "oracle.c").write_text(src)
+    shutil.copy(os.path.join(ORACLE_DIR, "__init__.py"), pkg / "__init__.py")
+    modname = f"oracle_copy_{name}"
+    spec = importlib.util.spec_from_file_location(modname, pkg / "__init__.py",
+                                                  submodule_search_locations=[str(pkg)])
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[modname] = mod
+    spec.loader.exec_module(mod)
+    mod.build(force=True)
+    return mod
+
+
+def _failing_pins(monkeypatch, mod):
+    monkeypatch.setattr(PINS, "oracle", mod)
+    failed = []
+    for pin, kw in PIN_CALLS:
+        try:
+            getattr(PINS, pin)(**kw)
+        except Exception as e:          # an assertion, or the oracle rejecting its inputs
+            failed.append((pin, type(e).__name__))
+    return failed
+
+
+def test_unmodified_copy_passes_every_pin(tmp_path, monkeypatch):
+    mod = _build_copy(tmp_path, "unmodified", [])
+    assert _failing_pins(monkeypatch, mod) == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_fails_a_pin(tmp_path, monkeypatch, name):
+    edits = [MUTANTS[name]] + ([UNPACK_MSB] if name == "msb_first_packing" else [])
+    mod = _build_copy(tmp_path, name, edits)
+    failed = _failing_pins(monkeypatch, mod)
+    assert failed, f"no pin catches the planted mistake {name}"

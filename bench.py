@@ -92,6 +92,20 @@ def kernel_source_hash(name: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+def max_over_ranks(values, world: int, device) -> list:
+    """Element-wise maximum of per-rank timings (ms) over all ranks: the job is as
+    slow as its slowest rank.  Every rank must call it, in the same order."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_scores_per_s(wl: workloads.Workload, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank scores its own batch each step."""
+    return wl.heads * wl.group * wl.T * world / (ms_per_step * 1e-3)
+
+
 def kernel_file(kind: str, wl: workloads.Workload) -> str:
     """Source file of the kernel the library runs for this workload (api.cu takes the
     tensor-core kernels at d = 128, for the write path with bf16/f16 keys)."""
@@ -378,11 +392,7 @@ def main():
     t_write = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     t_read = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
 
-    # max over ranks
-    t = torch.tensor([elapsed_ms, t_write, t_read], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, t_write, t_read = t.tolist()
+    elapsed_ms, t_write, t_read = max_over_ranks([elapsed_ms, t_write, t_read], world, device)
     ms_per_step = elapsed_ms / args.steps
 
     # end to end through the public API with host buffers
@@ -394,7 +404,6 @@ def main():
             dist.destroy_process_group()
         return
 
-    scores_per_step = wl.heads * wl.group * wl.T * world
     keys_per_step = wl.rows * world
     peak, peak_kind = measured_peak()
     write_gbs = algo["write"] / (t_write * 1e-3) / 1e9
@@ -414,7 +423,7 @@ def main():
     src = kernel_file(dominant, wl)
     line = {
         "metric": "lut_attention_scores_per_s",
-        "value": scores_per_step / (ms_per_step * 1e-3),
+        "value": job_scores_per_s(wl, world, ms_per_step),
         "unit": "scores/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -473,11 +482,8 @@ def run_e2e(wl, path, device, steps, world):
         step()
     b.record(stream)
     torch.cuda.synchronize(device)
-    ms = torch.tensor([a.elapsed_time(b) / steps], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    ms = ms.item()
-    return {"value": wl.heads * wl.group * wl.T * world / (ms * 1e-3), "unit": "scores/s",
+    ms = max_over_ranks([a.elapsed_time(b) / steps], world, device)[0]
+    return {"value": job_scores_per_s(wl, world, ms), "unit": "scores/s",
             "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 

@@ -76,16 +76,14 @@ struct Smem {
     float ss[2][2][kTileRows];     // [accumulator][column half][key]: partial sums of y^2
 };
 
-// Quantize one rotated coordinate y (bucket table at shared address tab, bias
-// folded so that the entry address is bits(f) * 8 + bias) and add its code into
-// the packed words at bit offset O.  Codes occupy disjoint bit fields, so adding
-// the bucket's base and then the compare bit is the same as or-ing the code.
+// Add the code of one coordinate into the packed words at bit offset O, given its
+// bucket value g and the bits of f = round(g) + 1.5 * 2^23 (bucket table at
+// shared address tab, bias folded so that the entry address is bits(f) * 8 +
+// bias).  Codes occupy disjoint bit fields, so adding the bucket's base and then
+// the compare bit is the same as or-ing the code.
 template <int B, int O, bool kClamp>
-__device__ __forceinline__ void quantize_one(float y, float a, float g_off, float off_magic, uint32_t tab,
-                                             uint32_t bias, uint32_t *w)
+__device__ __forceinline__ void place_code(float g, float f, uint32_t tab, uint32_t bias, uint32_t *w)
 {
-    const float g = fmaf(y, a, g_off);
-    const float f = fmaf(y, a, off_magic);          // round(g) sits in the low bits of f
     uint32_t addr;
     if constexpr (kClamp) {
         const uint32_t bucket = min(__float_as_uint(f) - kMagicBits, static_cast<uint32_t>(kMaxBuckets - 1));
@@ -107,13 +105,20 @@ __device__ __forceinline__ void quantize_one(float y, float a, float g_off, floa
     }
 }
 
+// Quantize coordinates C0 + E, C0 + E + 1 (two at a time: one paired FMA gives
+// both bucket values g = y a + g_off, one more both f = y a + g_off + 1.5 * 2^23,
+// rounded exactly as two scalar FMAs would be).
 template <int B, int C0, int E, bool kClamp>
-__device__ __forceinline__ void quantize_chunk(const uint32_t (&v)[32], float a, float g_off, float off_magic,
+__device__ __forceinline__ void quantize_chunk(const uint32_t (&v)[32], float2 a2, float2 goff2, float2 offm2,
                                                uint32_t tab, uint32_t bias, uint32_t *w)
 {
     if constexpr (E < 32) {
-        quantize_one<B, (C0 + E) * B, kClamp>(__uint_as_float(v[E]), a, g_off, off_magic, tab, bias, w);
-        quantize_chunk<B, C0, E + 1, kClamp>(v, a, g_off, off_magic, tab, bias, w);
+        const float2 y = make_float2(__uint_as_float(v[E]), __uint_as_float(v[E + 1]));
+        const float2 g = __ffma2_rn(y, a2, goff2);
+        const float2 f = __ffma2_rn(y, a2, offm2);
+        place_code<B, (C0 + E) * B, kClamp>(g.x, f.x, tab, bias, w);
+        place_code<B, (C0 + E + 1) * B, kClamp>(g.y, f.y, tab, bias, w);
+        quantize_chunk<B, C0, E + 2, kClamp>(v, a2, goff2, offm2, tab, bias, w);
     }
 }
 
@@ -261,16 +266,21 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const uint32_t col_addr = tmem + lane_base + acc * kD + half * kHalfCols;
             // pass 1: this half's sum of y^2 (four interleaved partial sums); the
             // pair adds both halves in a fixed order
-            float part4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            // (partial sums 0,1 and 2,3 in paired FMAs: coordinates e = 0, 1 mod 4 and 2, 3 mod 4)
+            float2 p01 = make_float2(0.0f, 0.0f), p23 = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int c = 0; c < kHalfCols / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(col_addr + 32 * c, v);
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    part4[e & 3] = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), part4[e & 3]);
+                for (int e = 0; e < 32; e += 4) {
+                    const float2 x01 = make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                    const float2 x23 = make_float2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                    p01 = __ffma2_rn(x01, x01, p01);
+                    p23 = __ffma2_rn(x23, x23, p23);
+                }
             }
-            S.ss[acc][half][key] = (part4[0] + part4[1]) + (part4[2] + part4[3]);
+            S.ss[acc][half][key] = (p01.x + p01.y) + (p23.x + p23.y);
             mbar_arrive(smem_u32(&S.pair[acc][quad]));
             if (!mbar_wait_warp(smem_u32(&S.pair[acc][quad]), aph)) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
@@ -290,16 +300,17 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const bool finite = ss <= 3.402823466e38f;
             const bool clamp = !(ss >= 1e-36f);
             const float a = (finite && ss > 0.0f) ? p.g_scale / sqrtf(ss) : 0.0f;
-            const float g_off = p.g_off;
-            const float off_magic = g_off + kMagic;
+            const float2 a2 = make_float2(a, a);
+            const float2 goff2 = make_float2(p.g_off, p.g_off);
+            const float2 offm2 = make_float2(p.g_off + kMagic, p.g_off + kMagic);
             {
                 uint32_t v[32];
                 tmem_ld32(col_addr, v);
-                if (finite && !clamp) quantize_chunk<B, 0, 0, false>(v, a, g_off, off_magic, tab_u32, tab_bias, w);
-                else if (finite) quantize_chunk<B, 0, 0, true>(v, a, g_off, off_magic, tab_u32, tab_bias, w);
+                if (finite && !clamp) quantize_chunk<B, 0, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 0, 0, true>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
                 tmem_ld32(col_addr + 32, v);
-                if (finite && !clamp) quantize_chunk<B, 32, 0, false>(v, a, g_off, off_magic, tab_u32, tab_bias, w);
-                else if (finite) quantize_chunk<B, 32, 0, true>(v, a, g_off, off_magic, tab_u32, tab_bias, w);
+                if (finite && !clamp) quantize_chunk<B, 32, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 32, 0, true>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
             }
             if (!finite) {
 #pragma unroll

@@ -62,10 +62,15 @@ constexpr int kGroupThreads = 128;    // worker threads of one stream (one per k
 constexpr int kK = 2 * kD;            // two digits per coordinate
 constexpr int kACols = kK / 4;        // tensor-memory columns of one A buffer
 constexpr int kTmemCols = 512;
-constexpr int kStageBytes = kTileRows * 64;   // packed rows of one tile (P <= 64)
+// One stage: the packed rows of a tile (P <= 64 bytes each), then its key norms.
+// The norms come as a TMA box that starts on a 16-byte boundary at or below the
+// tile's first norm, so it holds 128 + 3 floats; its offset in the box is
+// (first norm index + nshift) mod 4.
+constexpr int kStageCodeBytes = kTileRows * 64;
+constexpr int kNormBox = kTileRows + 4;
+constexpr int kStageBytes = kStageCodeBytes + 1024;   // keeps every stage 512-byte aligned
 constexpr int kLutBytes = 256 * 256;          // up to 256 fields x 256 bytes
 constexpr int kInvSlots = 8;          // per-stream ring of query scales, one slot per head
-constexpr int kNormSlots = 4;         // per-thread ring of key norms (tile k is read at k + 2)
 constexpr int kBBytesMax = 32 * kK;   // one B buffer at most: 8 queries x 4 digit rows x K bytes
 
 // launch shape for NQ query columns per KV head (G <= NQ)
@@ -97,9 +102,10 @@ struct Lookup {
 
 struct TcParams {
     CUtensorMap tmap;          // packed rows as a [heads*n, P] byte tensor, box P x 128
+    CUtensorMap nmap;          // key norms as a 1-D fp32 tensor from a 16-byte boundary, box kNormBox
     const void *q;
     int qdtype;
-    const float *norms;
+    int nshift;                // norms[0] is element nshift of nmap
     const int8_t *signs;
     float *scores;
     int n;                     // keys per head
@@ -124,9 +130,8 @@ struct Smem {
     float inv[kMaxStreams][kInvSlots][8];   // per stream, head slot and query: 1 / (128 * S_q * S_c)
     float q[2048];                           // rotation scratch: S * NQ <= 16 query rows of d floats
     float qmax[kMaxStreams][4][8];           // per stream, warp and query: max |q''|
-    float norm_ring[kMaxStreams][kNormSlots][kTileRows];
 };
-constexpr int kSmemBook = 16384;
+constexpr int kSmemBook = 10240;
 static_assert(sizeof(Smem) <= kSmemBook, "bookkeeping area too small");
 
 __device__ __forceinline__ float load_q(const void *q, int dtype, int64_t i)
@@ -304,19 +309,18 @@ struct Worker {
     // scores of this thread's key from its int32 digit sums.  D columns 4q .. 4q+3
     // of query q carry weights 128, 1, 1/128, 1/128^2; the pairs are joined in
     // int32 first (|128 c0 + c1| < 1.4e8, |128 c2 + c3| < 2.1e8), so two
-    // conversions serve a query.  The key norm is in ring slot `slot`; the
-    // query scales of the stream's head number `hc` (slot hc mod kInvSlots) are
-    // kept in `inv` while that head lasts.
+    // conversions serve a query.  nk is the key norm; the query scales of the
+    // stream's head number `hc` (slot hc mod kInvSlots) are kept in `inv` while
+    // that head lasts.
     static __device__ __forceinline__ void store_sums(const TcParams &p, const Smem &S, int g,
-                                                      const uint32_t (&acc)[NL][16], int slot, int hc, int h,
-                                                      int t, int r, int &inv_hc, float (&inv)[NQ])
+                                                      const uint32_t (&acc)[NL][16], float nk, int hc, int h,
+                                                      int t, int &inv_hc, float (&inv)[NQ])
     {
         if (hc != inv_hc) {
             inv_hc = hc;
 #pragma unroll
             for (int qi = 0; qi < NQ; ++qi) inv[qi] = S.inv[g][hc & (kInvSlots - 1)][qi];
         }
-        const float nk = S.norm_ring[g][slot][r];
         if (t < p.n) {
             float *dst = p.scores + static_cast<int64_t>(h) * p.group * p.n + t;
 #pragma unroll
@@ -351,11 +355,12 @@ struct Worker {
         const int r = threadIdx.x & (kGroupThreads - 1);   // key within the tile = tensor-memory lane
         const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(r & ~31) << 16);
         const uint32_t base_lane = lut_base | static_cast<uint32_t>(lane * LK::EB);
-        const uint32_t ring = smem_u32(&S.norm_ring[g][0][r]);
         int bsel = -1, prev_h = -1, hc = -1, sync_phase = 0;
         int h = (t0 + g) / p.tiles_per_head, ti = (t0 + g) - h * p.tiles_per_head;
-        // (head, key offset, stream head number) of tiles k - 1 and k - 2, whose scores are still due
+        // (head, key offset, stream head number, key norm) of tiles k - 1 and k - 2,
+        // whose scores are still due
         int h1 = 0, t1k = 0, hs1 = 0, h2 = 0, t2k = 0, hs2 = 0;
+        float nk1 = 0.0f, nk2 = 0.0f;
         int s = g, k = 0;
         uint32_t sph = 0;
         bool ok = true;
@@ -379,11 +384,10 @@ struct Worker {
                 }
                 w[NW] = 0;
             }
+            // this tile's key norm (its scores are due two tiles from now)
+            const float nk = reinterpret_cast<const float *>(sStage + s * kStageBytes + kStageCodeBytes)
+                [((h * p.n + ti * kTileRows + p.nshift) & 3) + r];
             mbar_arrive(smem_u32(&S.empty[s]));
-            // this tile's key norm, read two tiles from now
-            cp_async_4(ring + (k & (kNormSlots - 1)) * (kTileRows * 4),
-                       p.norms + static_cast<int64_t>(h) * p.n + min(ti * kTileRows + r, p.n - 1));
-            cp_async_commit();
 
             // products of tile k - 2 done: its D is readable, its A buffer and the
             // B buffer of two heads back are free
@@ -434,13 +438,10 @@ struct Worker {
             if (k >= 2) load_wait(acc);
             tc_fence_before_sync();
             mbar_arrive(smem_u32(&S.a_full[g][ab]));
-            if (k >= 2) {
-                cp_async_wait<2>();          // the norm copy of tile k - 2 has landed
-                store_sums(p, S, g, acc, (k - 2) & (kNormSlots - 1), hs2, h2, t2k + r, r, inv_hc, inv);
-            }
+            if (k >= 2) store_sums(p, S, g, acc, nk2, hs2, h2, t2k + r, inv_hc, inv);
 
-            h2 = h1; t2k = t1k; hs2 = hs1;
-            h1 = h; t1k = ti * kTileRows; hs1 = hc;
+            h2 = h1; t2k = t1k; hs2 = hs1; nk2 = nk1;
+            h1 = h; t1k = ti * kTileRows; hs1 = hc; nk1 = nk;
             s += C::S;
             if (s >= kStages) {
                 s -= kStages;
@@ -455,7 +456,6 @@ struct Worker {
 
         // the last two tiles' scores
         if (ok) {
-            cp_async_wait<0>();
             for (int j = (k >= 2 ? k - 2 : 0); j < k; ++j) {
                 const bool last = (j == k - 1);
                 if (!mbar_wait_warp(smem_u32(&S.mma_done[g][j & 1]), (j >> 1) & 1)) {
@@ -465,11 +465,10 @@ struct Worker {
                 tc_fence_after_sync();
                 load_issue(tmem_lane + C::kDOff + (2 * g + (j & 1)) * C::N, acc);
                 load_wait(acc);
-                store_sums(p, S, g, acc, j & (kNormSlots - 1), last ? hs1 : hs2, last ? h1 : h2,
-                           (last ? t1k : t2k) + r, r, inv_hc, inv);
+                store_sums(p, S, g, acc, last ? nk1 : nk2, last ? hs1 : hs2, last ? h1 : h2,
+                           (last ? t1k : t2k) + r, inv_hc, inv);
             }
         }
-        cp_async_wait<0>();
     }
 };
 
@@ -479,7 +478,8 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const _
     using LK = Lookup<B>;
     using C = Cfg<NQ>;
     constexpr int P = kD * B / 8;
-    static_assert(kTileRows * P <= kStageBytes, "stage too small for a tile of packed rows");
+    static_assert(kTileRows * P <= kStageCodeBytes && kStageCodeBytes + kNormBox * 4 <= kStageBytes,
+                  "stage too small for a tile of packed rows and its norms");
     static_assert(LK::NF * 256 <= kLutBytes, "lookup table too large");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -512,7 +512,10 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const _
         }
         fence_mbar_init();
     }
-    if (warp == C::kWarpTma && lane == 0) prefetch_tensormap(&p.tmap);
+    if (warp == C::kWarpTma && lane == 0) {
+        prefetch_tensormap(&p.tmap);
+        prefetch_tensormap(&p.nmap);
+    }
     if (warp < C::kWorkerWarps) build_lut<B, C::kWorkerWarps * 32>(p, sLut);
     if (warp == 0) {
         tmem_alloc(smem_u32(&S.tmem_base), kTmemCols);
@@ -535,8 +538,11 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const _
                     break;
                 }
                 const uint32_t full = smem_u32(&S.full[s]);
-                mbar_arrive_expect_tx(full, kTileRows * P);
-                tma_load_2d(smem_u32(sStage + s * kStageBytes), &p.tmap, 0, h * p.n + ti * kTileRows, full);
+                const int row = h * p.n + ti * kTileRows;
+                mbar_arrive_expect_tx(full, kTileRows * P + kNormBox * 4);
+                tma_load_2d(smem_u32(sStage + s * kStageBytes), &p.tmap, 0, row, full);
+                tma_load_1d(smem_u32(sStage + s * kStageBytes + kStageCodeBytes), &p.nmap, (row + p.nshift) & ~3,
+                            full);
                 if (++s == kStages) {
                     s = 0;
                     ph ^= 1;
@@ -653,9 +659,22 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    // norms as a 1-D fp32 tensor whose base is the 16-byte boundary at or below
+    // a.norms (TMA wants an aligned base and element offsets that are multiples
+    // of 4 floats); boxes running past the end read zeros
+    const uintptr_t nbase = reinterpret_cast<uintptr_t>(a.norms) & ~static_cast<uintptr_t>(15);
+    p.nshift = static_cast<int>((reinterpret_cast<uintptr_t>(a.norms) - nbase) / sizeof(float));
+    const cuuint64_t ndims[1] = {static_cast<cuuint64_t>(a.heads) * static_cast<cuuint64_t>(a.n) +
+                                 static_cast<cuuint64_t>(p.nshift)};
+    const cuuint64_t nstrides[1] = {0};      // unused for one dimension
+    const cuuint32_t nbox[1] = {kNormBox};
+    const cuuint32_t nestr[1] = {1};
+    r = enc(&p.nmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, reinterpret_cast<void *>(nbase), ndims, nstrides, nbox,
+            nestr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     p.q = a.q;
     p.qdtype = a.qdtype;
-    p.norms = a.norms;
     p.signs = a.signs;
     p.scores = a.scores;
     p.n = static_cast<int>(a.n);

@@ -98,6 +98,23 @@ def test_scores_tile_ranges_cross_heads(heads, n, group, b):
     assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
 
 
+@pytest.mark.parametrize("offset", [0, 1, 2, 3])
+def test_scores_norms_at_any_4_byte_offset(offset):
+    """The tensor-core read kernel loads key norms by TMA from the 16-byte boundary
+    at or below the norms pointer; a norms buffer that starts 4, 8 or 12 bytes past
+    such a boundary must give the same scores."""
+    d, b, heads, n, group = 128, 4, 5, 1000, 4
+    packed, norms = workloads.make_random_packed(heads, n, d, b, seed=41 + offset, device=DEV)
+    store = torch.zeros(heads * n + 4, dtype=torch.float32, device=DEV)
+    shifted = store[offset:offset + heads * n].view(heads, n)
+    shifted.copy_(norms)
+    wl = workloads.GQA_DECODE_128K.with_(batch=1, kv_heads=heads, group=group, T=n)
+    q = workloads.make_queries(wl, DEV)
+    s = workloads.make_signs(wl).to(DEV)
+    out = gpu_scores(q, packed, shifted, group, b, s)
+    assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
+
+
 def test_scores_group8_wide_head():
     d, b, heads, n, group = 512, 2, 1, 700, 8
     packed, norms = workloads.make_random_packed(heads, n, d, b, seed=5, device=DEV)

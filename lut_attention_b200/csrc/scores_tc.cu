@@ -29,10 +29,11 @@
 // deals round-robin to S tile streams (S = 3 for up to 4 queries per KV head,
 // else 2).  Per stream:
 //   4 worker warps : one thread per key (= tensor-memory lane).  For tile k:
-//                    read the packed row, look up its digits, store them to A
-//                    in tensor memory; then, once the products of tile k - 2
-//                    are done, read its int32 sums (D), scale them by the key
-//                    norm and the query scale, store the scores.  On entering a
+//                    read the packed row and the key norm; once the products
+//                    of tile k - 2 are done, read its int32 sums (D), scale
+//                    them by the key norm and the query scale and store the
+//                    scores; then look up tile k's digits and store them to
+//                    A in the same buffer.  On entering a
 //                    new KV head they rotate its queries (sign flip,
 //                    Walsh-Hadamard butterflies, 1/d) and write their digits
 //                    into the other of the stream's two B buffers.
@@ -336,16 +337,11 @@ struct Worker {
         }
     }
 
-    static __device__ __forceinline__ void load_issue(uint32_t taddr, uint32_t (&acc)[NL][16])
+    // int32 digit sums of this thread's key out of D (load and wait)
+    static __device__ __forceinline__ void load_sums(uint32_t taddr, uint32_t (&acc)[NL][16])
     {
 #pragma unroll
-        for (int c = 0; c < NL; ++c) tmem_ld16_issue(taddr + 16 * c, acc[c]);
-    }
-
-    static __device__ __forceinline__ void load_wait(uint32_t (&acc)[NL][16])
-    {
-#pragma unroll
-        for (int c = 0; c < NL; ++c) tmem_wait_ld_pass(acc[c]);
+        for (int c = 0; c < NL; ++c) tmem_ld16(taddr + 16 * c, acc[c]);
     }
 
     static __device__ void run(const TcParams &p, Smem &S, int g, uint8_t *sStage, uint8_t *sB, uint32_t lut_base,
@@ -364,7 +360,6 @@ struct Worker {
         int s = g, k = 0;
         uint32_t sph = 0;
         bool ok = true;
-        uint32_t acc[NL][16] = {};          // sums of tile k - 2, loaded while tile k decodes
         int inv_hc = -1;                    // head number whose query scales `inv` holds
         float inv[NQ];
 
@@ -398,7 +393,12 @@ struct Worker {
                 break;
             }
             tc_fence_after_sync();
-            if (k >= 2) load_issue(tmem_lane + C::kDOff + (2 * g + ab) * C::N, acc);
+            // scores of tile k - 2, read out of D before tile k's products may overwrite it
+            if (k >= 2) {
+                uint32_t acc[NL][16];
+                load_sums(tmem_lane + C::kDOff + (2 * g + ab) * C::N, acc);
+                store_sums(p, S, g, acc, nk2, hs2, h2, t2k + r, inv_hc, inv);
+            }
 
             if (h != prev_h) {
                 bsel = (bsel < 0) ? 0 : (bsel ^ 1);
@@ -433,12 +433,8 @@ struct Worker {
                 tmem_st16(a_addr + 16 * qt, a);
             }
             tmem_wait_st();
-            // the products of tile k overwrite D of tile k - 2: its sums must be in
-            // registers before A is published
-            if (k >= 2) load_wait(acc);
             tc_fence_before_sync();
             mbar_arrive(smem_u32(&S.a_full[g][ab]));
-            if (k >= 2) store_sums(p, S, g, acc, nk2, hs2, h2, t2k + r, inv_hc, inv);
 
             h2 = h1; t2k = t1k; hs2 = hs1; nk2 = nk1;
             h1 = h; t1k = ti * kTileRows; hs1 = hc; nk1 = nk;
@@ -463,8 +459,8 @@ struct Worker {
                     break;
                 }
                 tc_fence_after_sync();
-                load_issue(tmem_lane + C::kDOff + (2 * g + (j & 1)) * C::N, acc);
-                load_wait(acc);
+                uint32_t acc[NL][16];
+                load_sums(tmem_lane + C::kDOff + (2 * g + (j & 1)) * C::N, acc);
                 store_sums(p, S, g, acc, last ? nk1 : nk2, last ? hs1 : hs2, last ? h1 : h2,
                            (last ? t1k : t2k) + r, inv_hc, inv);
             }

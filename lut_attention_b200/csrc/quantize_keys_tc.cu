@@ -9,13 +9,16 @@
 // a butterfly transform, without spending CUDA-core instructions on it.
 //
 // One CTA per SM, persistent over 128-key tiles:
-//   warp 8 (TMA)  : streams key tiles HBM -> shared memory (4-stage ring,
+//   warp 16 (TMA) : streams key tiles HBM -> shared memory (4-stage ring,
 //                   128-byte swizzle, one 32 KB tile per stage);
-//   warp 9 (MMA)  : 8 tcgen05.mma (M=128, N=128, K=16) per tile into one of two
+//   warp 17 (MMA) : 8 tcgen05.mma (M=128, N=128, K=16) per tile into one of two
 //                   128-column fp32 accumulators in tensor memory;
-//   warps 0-7     : two warps per 32 keys (a tensor-memory lane quadrant), one
-//                   per half of the 128 columns: read y, exchange the partial
-//                   sums of y^2 (= d ||k||^2 in total), quantize, pack, store.
+//   warps 0-15    : two epilogue groups of 8 warps, group e draining
+//                   accumulator e (the CTA's even or odd tiles), so two tiles are
+//                   in the epilogue at once.  In a group, two warps per 32 keys
+//                   (a tensor-memory lane quadrant), one per half of the 128
+//                   columns: read y, exchange the partial sums of y^2
+//                   (= d ||k||^2 in total), quantize, pack, store.
 // Quantization: u = y / sqrt(sum y^2); with g = u * G_SCALE + G_OFF every
 // bucket [j - 0.5, j + 0.5) of g holds at most one decision boundary, so
 //     idx = base[j] + (g > tau[j]),   j = round(g)
@@ -45,7 +48,8 @@ constexpr int kStages = 4;
 constexpr int kABytes = kTileRows * kD * 2;     // one tile of keys, 32 KB
 constexpr int kBBytes = kD * kD * 2;            // H diag(s), 32 KB
 constexpr int kHalfBytes = kTileRows * 128;     // one 64-element K block of a tile
-constexpr int kEpiWarps = 8;
+constexpr int kGroupWarps = 8;                  // one epilogue group: two warps per lane quadrant
+constexpr int kEpiWarps = 2 * kGroupWarps;      // two groups, one per accumulator
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kTmemCols = 256;                  // two 128-column accumulators
 constexpr int kWarpTma = kEpiWarps, kWarpMma = kEpiWarps + 1;
@@ -145,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&S.acc_full[a]), 1);
-            mbar_init(smem_u32(&S.acc_empty[a]), kEpiWarps * 32);   // every epilogue thread
+            mbar_init(smem_u32(&S.acc_empty[a]), kGroupWarps * 32);   // the group that drains it
         }
         mbar_init(smem_u32(&S.drain), 1);
         for (int a = 0; a < 2; ++a)
@@ -248,16 +252,19 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         // ---------------------------------------------------------- epilogue
         constexpr int kHalfCols = kD / 2;
         constexpr int NWH = NW / 2;                  // packed words per half row
-        const int quad = warp & 3, half = warp >> 2;
+        // group e drains accumulator e: the CTA's tiles 2m + e, so two tiles are
+        // in the epilogue at once
+        const int grp = warp / kGroupWarps;
+        const int quad = warp & 3, half = (warp >> 2) & 1;
         const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
         const int key = quad * 32 + lane;            // key within the tile
         constexpr uint32_t kCentral = (1u << (B - 1)) - 1u;
         const uint32_t tab_u32 = smem_u32(sTab);
         const uint32_t tab_bias = tab_u32 - kMagicBits * 8u;     // wraps mod 2^32 by design
         int it = 0;
-        for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
-            const int acc = it & 1;
-            const uint32_t aph = (it >> 1) & 1;
+        const int acc = grp;
+        for (int t = blockIdx.x + grp * gridDim.x; t < p.ntiles; t += 2 * gridDim.x, ++it) {
+            const uint32_t aph = it & 1;
             if (!mbar_wait_warp(smem_u32(&S.acc_full[acc]), aph)) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
                 break;

@@ -114,6 +114,30 @@ int axr_scores(const void *q, int qdtype, const uint8_t *idx, const float *norms
                float *scores, axr_stream stream);
 
 /*
+ * One decode step on a key cache (AXELRAM abstract: keys are quantized once, when
+ * written; every read is a table lookup on the stored indices).  For every KV
+ * head h the new key k_new[h] is quantized exactly as axr_quantize_keys would
+ * and stored in slot `pos` of that head's cache; then every query head scores
+ * keys 0 .. pos of its KV head exactly as axr_scores would.
+ *
+ * k_new   device, heads x d row-major, element type kdtype; 16-byte aligned.
+ * q       device, (heads*group) x d row-major, element type qdtype; 16-byte aligned.
+ * idx     device, heads x capacity x P bytes (P = d*b/8): the packed cache, head h
+ *         at rows [h*capacity, (h+1)*capacity); 16-byte aligned.  Rows < pos hold
+ *         earlier keys; row pos is overwritten; rows > pos are neither read for
+ *         scores nor written.
+ * norms   device float[heads * capacity], laid out like idx; row pos is overwritten.
+ * capacity  keys each head's cache holds, >= 1; 0 <= pos < capacity (else AXR_EINVAL).
+ * scores  device float[(heads*group) * (pos+1)] output; row h*group+g holds the
+ *         pos+1 scores of that query head (row stride pos+1).
+ * The two parts are enqueued on `stream` in order; the call is asynchronous like
+ * the others.
+ */
+int axr_append_scores(const void *k_new, int kdtype, const void *q, int qdtype, uint8_t *idx,
+                      float *norms, int64_t capacity, int64_t pos, int heads, int group, int d, int b,
+                      const int8_t *signs, float *scores, axr_stream stream);
+
+/*
  * Device-side status of the tensor-core kernels (no counterpart in the method;
  * a diagnostic).  Every wait inside those kernels is bounded; a wait that runs
  * out records a bit here instead of hanging: 1 = a tile load never arrived,

@@ -7,6 +7,7 @@ load the library; the first call does, and raises if it has not been built.
 """
 from .axr import (  # noqa: F401
     AxrError,
+    axr_append_scores,
     axr_device_status,
     axr_make_codebook,
     axr_quantize_keys,
@@ -17,6 +18,7 @@ from .axr import (  # noqa: F401
 
 __all__ = [
     "AxrError",
+    "axr_append_scores",
     "axr_device_status",
     "axr_make_codebook",
     "axr_quantize_keys",

@@ -27,6 +27,7 @@ SIGNATURES = {
     "axr_make_codebook": (_I32, [_I32, _I32, _P, _P]),
     "axr_quantize_keys": (_I32, [_P, _I32, _I64, _I32, _I32, _P, _P, _P, _P]),
     "axr_scores": (_I32, [_P, _I32, _P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
+    "axr_append_scores": (_I32, [_P, _I32, _P, _I32, _P, _P, _I64, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
     "axr_status_string": (ctypes.c_char_p, [_I32]),
     "axr_last_error": (ctypes.c_char_p, []),
     "axr_version": (_I32, []),
@@ -152,6 +153,43 @@ def axr_scores(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, group: i
                               heads, group, d, b, signs.data_ptr(), scores.data_ptr(),
                               _stream_handle(stream))
     _raise(rc, "axr_scores")
+    return scores
+
+
+def axr_append_scores(k_new: torch.Tensor, q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, pos: int,
+                      group: int, b: int, signs: torch.Tensor, scores: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """One decode step on a key cache: quantize the new key of every KV head
+    (k_new (heads, d)) into slot ``pos`` of idx (heads, capacity, d*b/8) and norms
+    (heads, capacity), then score the query heads q (heads*group, d) against keys
+    0 .. pos.  Returns scores (heads*group, pos+1) fp32."""
+    for t, name in ((k_new, "k_new"), (q, "q"), (idx, "idx"), (norms, "norms"), (signs, "signs")):
+        _require_cuda(t, name)
+    if k_new.dtype not in _DTYPE_CODE or q.dtype not in _DTYPE_CODE:
+        raise ValueError("k_new and q must be float32, float16 or bfloat16")
+    if idx.dtype != torch.uint8 or norms.dtype != torch.float32 or signs.dtype != torch.int8:
+        raise ValueError("idx must be uint8, norms float32, signs int8")
+    heads, d = k_new.shape
+    hg, dq = q.shape
+    if dq != d or group < 1 or hg != heads * group:
+        raise ValueError(f"q must be ({heads}*{group}, {d})")
+    if idx.dim() != 3 or idx.shape[0] != heads or idx.shape[2] != packed_row_bytes(d, b):
+        raise ValueError(f"idx must be (heads={heads}, capacity, {packed_row_bytes(d, b)})")
+    capacity = idx.shape[1]
+    if tuple(norms.shape) != (heads, capacity):
+        raise ValueError(f"norms must be ({heads}, {capacity})")
+    if not 0 <= pos < capacity:
+        raise ValueError(f"pos={pos} is outside the cache [0, {capacity})")
+    if scores is None:
+        scores = torch.empty((hg, pos + 1), dtype=torch.float32, device=q.device)
+    _require_cuda(scores, "scores")
+    if scores.numel() < hg * (pos + 1) or scores.dtype != torch.float32:
+        raise ValueError("scores must be float32 with (heads*group)*(pos+1) elements")
+    rc = library().axr_append_scores(k_new.data_ptr(), _DTYPE_CODE[k_new.dtype], q.data_ptr(),
+                                     _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), capacity, pos,
+                                     heads, group, d, b, signs.data_ptr(), scores.data_ptr(),
+                                     _stream_handle(stream))
+    _raise(rc, "axr_append_scores")
     return scores
 
 

@@ -152,9 +152,50 @@ extern "C" int axr_scores(const void *q, int qdtype, const uint8_t *idx, const f
     if ((rc = check_device_ptr(scores, 4, "scores")) != AXR_OK) return rc;
 
     ScoresArgs a{q, qdtype, idx, norms, n, heads, group, d, b, signs, scores, Codebook{}};
+    a.head_stride = n;
     if (!get_codebook(d, b, &a.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
     cudaError_t e = scores_tc_supported(a) ? launch_scores_tc(a, reinterpret_cast<cudaStream_t>(stream))
                                            : launch_scores(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "scores launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+extern "C" int axr_append_scores(const void *k_new, int kdtype, const void *q, int qdtype, uint8_t *idx,
+                                 float *norms, int64_t capacity, int64_t pos, int heads, int group, int d, int b,
+                                 const int8_t *signs, float *scores, axr_stream stream)
+{
+    int rc = check_shape(d, b);
+    if (rc != AXR_OK) return rc;
+    if (elem_size(kdtype) == 0) return fail(AXR_EINVAL, "kdtype=%d is not an axr_dtype", kdtype);
+    if (elem_size(qdtype) == 0) return fail(AXR_EINVAL, "qdtype=%d is not an axr_dtype", qdtype);
+    if (heads < 1) return fail(AXR_EINVAL, "heads=%d must be >= 1", heads);
+    if (group < 1) return fail(AXR_EINVAL, "group=%d must be >= 1", group);
+    if (group > kMaxGroup) return fail(AXR_EUNSUPPORTED, "group=%d: at most %d", group, kMaxGroup);
+    if (capacity < 1) return fail(AXR_EINVAL, "capacity=%lld must be >= 1", (long long)capacity);
+    if (capacity > (int64_t)INT32_MAX)
+        return fail(AXR_EUNSUPPORTED, "capacity=%lld: at most 2^31-1 keys per head", (long long)capacity);
+    if (pos < 0 || pos >= capacity)
+        return fail(AXR_EINVAL, "pos=%lld is outside the cache [0, %lld)", (long long)pos, (long long)capacity);
+    if ((rc = check_device_ptr(k_new, 16, "k_new")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(q, 16, "q")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(idx, 16, "idx")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(norms, 4, "norms")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(signs, 1, "signs")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(scores, 4, "scores")) != AXR_OK) return rc;
+
+    Codebook cb;
+    if (!get_codebook(d, b, &cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // the new key of KV head h goes to cache row h * capacity + pos
+    QuantizeArgs qa{k_new, kdtype, heads, d, b, signs, idx, norms, cb};
+    qa.out_stride = capacity;
+    qa.out_offset = pos;
+    cudaError_t e = launch_quantize_keys(qa, st);
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "append launch: %s", cudaGetErrorString(e));
+    // then every query head against keys 0 .. pos of its KV head
+    ScoresArgs sa{q, qdtype, idx, norms, pos + 1, heads, group, d, b, signs, scores, cb};
+    sa.head_stride = capacity;
+    e = scores_tc_supported(sa) ? launch_scores_tc(sa, st) : launch_scores(sa, st);
     if (e != cudaSuccess) return fail(AXR_ECUDA, "scores launch: %s", cudaGetErrorString(e));
     return ok();
 }

@@ -48,6 +48,11 @@ struct QuantizeArgs {
     uint8_t *idx;
     float *norms;
     Codebook cb;
+    // key r is stored at row r * out_stride + out_offset of idx and norms
+    // (1 and 0 for a dense batch; a cache's capacity and the write slot when one
+    // key per head is appended)
+    int64_t out_stride = 1;
+    int64_t out_offset = 0;
 };
 
 struct ScoresArgs {
@@ -63,6 +68,7 @@ struct ScoresArgs {
     const int8_t *signs;
     float *scores;
     Codebook cb;
+    int64_t head_stride = 0;   // rows between KV heads in idx and norms (n for a dense cache)
 };
 
 // Kernel launchers (quantize_keys.cu, scores.cu).  They return cudaSuccess or

@@ -35,6 +35,8 @@ struct QParams {
     const int8_t *signs;
     uint8_t *idx;
     float *norms;
+    int64_t out_stride;        // key r goes to row r * out_stride + out_offset
+    int64_t out_offset;
     float bnd[kMaxLevels - 1];
 };
 
@@ -200,18 +202,26 @@ __global__ void __launch_bounds__(kThreads) quantize_keys_kernel(QParams p)
         }
         __syncwarp();
 
-        // the warp step's rows are contiguous in idx: write them out
         const int64_t first = s * RW;
-        uint8_t *dst = p.idx + first * P;
         const int64_t rows_here = (p.n - first < RW) ? (p.n - first) : RW;
-        if (rows_here == RW) {
-            if (lane < WBYTES / 16)
-                __stcs(reinterpret_cast<uint4 *>(dst) + lane, reinterpret_cast<const uint4 *>(stage)[lane]);
+        if (p.out_stride == 1 && p.out_offset == 0) {
+            // the warp step's rows are contiguous in idx: write them out
+            uint8_t *dst = p.idx + first * P;
+            if (rows_here == RW) {
+                if (lane < WBYTES / 16)
+                    __stcs(reinterpret_cast<uint4 *>(dst) + lane, reinterpret_cast<const uint4 *>(stage)[lane]);
+            } else {
+                const int nbytes = static_cast<int>(rows_here) * P;
+                for (int i = lane; i < nbytes; i += 32) dst[i] = stage[i];
+            }
         } else {
-            const int nbytes = static_cast<int>(rows_here) * P;
-            for (int i = lane; i < nbytes; i += 32) dst[i] = stage[i];
+            // rows land out_stride rows apart (one key appended per cache head)
+            for (int i = lane; i < static_cast<int>(rows_here) * P; i += 32) {
+                const int64_t rr = first + i / P;
+                p.idx[(rr * p.out_stride + p.out_offset) * P + i % P] = stage[i];
+            }
         }
-        if (valid && t == 0) __stcs(p.norms + row, norm);
+        if (valid && t == 0) __stcs(p.norms + row * p.out_stride + p.out_offset, norm);
         __syncwarp();
     }
 }
@@ -240,6 +250,8 @@ cudaError_t launch_typed(const QuantizeArgs &a, cudaStream_t stream)
     p.signs = a.signs;
     p.idx = a.idx;
     p.norms = a.norms;
+    p.out_stride = a.out_stride;
+    p.out_offset = a.out_offset;
     for (int i = 0; i < kMaxLevels - 1; ++i) p.bnd[i] = a.cb.boundaries[i];
     kernel<<<grid, kThreads, 0, stream>>>(p);
     return cudaGetLastError();

@@ -433,7 +433,8 @@ cudaError_t launch_typed(const QuantizeArgs &a, const BucketTable &tab, cudaStre
 
 bool quantize_tc_supported(const QuantizeArgs &a)
 {
-    return a.d == kD && (a.kdtype == AXR_BF16 || a.kdtype == AXR_F16) && a.n > 0 &&
+    return a.d == kD && (a.kdtype == AXR_BF16 || a.kdtype == AXR_F16) && a.n > 0 && a.out_stride == 1 &&
+           a.out_offset == 0 &&
            a.n <= static_cast<int64_t>(0x7fffffff) - kTileRows && encode_tiled() != nullptr;
 }
 

@@ -33,6 +33,7 @@ struct SParams {
     const uint8_t *idx;
     const float *norms;
     int n;
+    int64_t head_stride;       // rows between KV heads in idx and norms
     int group;
     const int8_t *signs;
     float *scores;
@@ -162,8 +163,8 @@ __global__ void __launch_bounds__(kThreads) scores_kernel(SParams p)
     const int n = p.n;
     const int tile0 = blockIdx.x * kTile;
     const int tile1 = (n - tile0 < kTile) ? n : tile0 + kTile;
-    const uint8_t *idx_h = p.idx + static_cast<int64_t>(h) * n * P;
-    const float *norms_h = p.norms + static_cast<int64_t>(h) * n;
+    const uint8_t *idx_h = p.idx + static_cast<int64_t>(h) * p.head_stride * P;
+    const float *norms_h = p.norms + static_cast<int64_t>(h) * p.head_stride;
 
     for (int r0 = tile0 + warp * RS; r0 < tile1; r0 += kWarps * RS) {
         const int r = r0 + slot;
@@ -202,6 +203,7 @@ cudaError_t launch_dbg(const ScoresArgs &a, cudaStream_t stream)
     p.idx = a.idx;
     p.norms = a.norms;
     p.n = static_cast<int>(a.n);
+    p.head_stride = a.head_stride;
     p.group = a.group;
     p.signs = a.signs;
     p.scores = a.scores;

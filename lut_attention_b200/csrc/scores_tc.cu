@@ -110,6 +110,7 @@ struct TcParams {
     const int8_t *signs;
     float *scores;
     int n;                     // keys per head
+    int head_stride;           // rows between KV heads in the packed rows and norms (>= n)
     int group;
     int tiles_per_head;
     int total_tiles;
@@ -381,7 +382,7 @@ struct Worker {
             }
             // this tile's key norm (its scores are due two tiles from now)
             const float nk = reinterpret_cast<const float *>(sStage + s * kStageBytes + kStageCodeBytes)
-                [((h * p.n + ti * kTileRows + p.nshift) & 3) + r];
+                [((h * p.head_stride + ti * kTileRows + p.nshift) & 3) + r];
             mbar_arrive(smem_u32(&S.empty[s]));
 
             // products of tile k - 2 done: its D is readable, its A buffer and the
@@ -534,7 +535,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const _
                     break;
                 }
                 const uint32_t full = smem_u32(&S.full[s]);
-                const int row = h * p.n + ti * kTileRows;
+                const int row = h * p.head_stride + ti * kTileRows;
                 mbar_arrive_expect_tx(full, kTileRows * P + kNormBox * 4);
                 tma_load_2d(smem_u32(sStage + s * kStageBytes), &p.tmap, 0, row, full);
                 tma_load_1d(smem_u32(sStage + s * kStageBytes + kStageCodeBytes), &p.nmap, (row + p.nshift) & ~3,
@@ -645,7 +646,7 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     if (!enc) return cudaErrorNotSupported;
     TcParams p{};
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(P),
-                                static_cast<cuuint64_t>(a.heads) * static_cast<cuuint64_t>(a.n)};
+                                static_cast<cuuint64_t>(a.heads) * static_cast<cuuint64_t>(a.head_stride)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(P)};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(P), kTileRows};
     const cuuint32_t estr[2] = {1, 1};
@@ -660,7 +661,7 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     // of 4 floats); boxes running past the end read zeros
     const uintptr_t nbase = reinterpret_cast<uintptr_t>(a.norms) & ~static_cast<uintptr_t>(15);
     p.nshift = static_cast<int>((reinterpret_cast<uintptr_t>(a.norms) - nbase) / sizeof(float));
-    const cuuint64_t ndims[1] = {static_cast<cuuint64_t>(a.heads) * static_cast<cuuint64_t>(a.n) +
+    const cuuint64_t ndims[1] = {static_cast<cuuint64_t>(a.heads) * static_cast<cuuint64_t>(a.head_stride) +
                                  static_cast<cuuint64_t>(p.nshift)};
     const cuuint64_t nstrides[1] = {0};      // unused for one dimension
     const cuuint32_t nbox[1] = {kNormBox};
@@ -674,6 +675,7 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     p.signs = a.signs;
     p.scores = a.scores;
     p.n = static_cast<int>(a.n);
+    p.head_stride = static_cast<int>(a.head_stride);
     p.group = a.group;
     p.tiles_per_head = static_cast<int>((a.n + kTileRows - 1) / kTileRows);
     p.total_tiles = p.tiles_per_head * a.heads;
@@ -708,7 +710,7 @@ cudaError_t launch_b(const ScoresArgs &a, cudaStream_t stream)
 bool scores_tc_supported(const ScoresArgs &a)
 {
     return a.d == kD && a.b >= 1 && a.b <= 4 && a.group <= 8 && a.n > 0 &&
-           static_cast<int64_t>(a.heads) * a.n < (static_cast<int64_t>(1) << 31) - kTileRows &&
+           static_cast<int64_t>(a.heads) * a.head_stride < (static_cast<int64_t>(1) << 31) - kTileRows &&
            encode_tiled() != nullptr;
 }
 

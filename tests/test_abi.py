@@ -91,6 +91,23 @@ def test_scores_argument_errors(axr_lib):
     assert s(p, 2, p, p, 10, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL       # host memory
 
 
+def test_append_argument_errors(axr_lib):
+    f = axr_lib.axr_append_scores
+    host = np.zeros(4096, np.uint8)
+    p = host.ctypes.data
+    # (k_new, kdtype, q, qdtype, idx, norms, capacity, pos, heads, group, d, b, signs, scores, stream)
+    assert f(p, 2, p, 2, p, p, 16, 16, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL        # pos == capacity
+    assert f(p, 2, p, 2, p, p, 16, -1, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL        # pos < 0
+    assert f(p, 2, p, 2, p, p, 0, 0, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL          # empty cache
+    assert f(p, 2, p, 2, p, p, 16, 3, 0, 1, 128, 4, p, p, None) == axr.AXR_EINVAL         # heads < 1
+    assert f(p, 2, p, 2, p, p, 16, 3, 1, 9, 128, 4, p, p, None) == axr.AXR_EUNSUPPORTED   # group > 8
+    assert f(p, 2, p, 2, p, p, 16, 3, 1, 1, 96, 4, p, p, None) == axr.AXR_EUNSUPPORTED    # d
+    assert f(p, 5, p, 2, p, p, 16, 3, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL         # key dtype
+    assert f(p, 2, p, 7, p, p, 16, 3, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL         # query dtype
+    assert f(p + 4, 2, p, 2, p, p, 16, 3, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL     # misaligned k_new
+    assert f(p, 2, p, 2, p, p, 16, 3, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL         # host memory
+
+
 def test_binding_refuses_cpu_tensors():
     """No CPU path: the binding raises instead of computing on the host."""
     K = torch.zeros(4, 128)

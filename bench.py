@@ -236,6 +236,36 @@ class Path:
                        scores=self.scores)
 
 
+def run_decode_step(path: Path, steps: int) -> dict:
+    """The decode step the cache serves: append one key per KV head at the last
+    slot (pos = T - 1) and score every query head against all T keys
+    (axr_append_scores), timed against scoring the same T keys alone."""
+    wl = path.wl
+    k_new = path.K[:, -1].contiguous()
+    pos = wl.T - 1
+
+    def append():
+        axr.axr_append_scores(k_new, path.q, path.idx[0], path.norms[0], pos, wl.group, wl.b, path.signs,
+                              scores=path.scores)
+
+    def time_ms(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    t_step = time_ms(append)
+    t_scores = time_ms(lambda: path.score(0))
+    return {"ms": t_step, "scores_only_ms": t_scores, "context": wl.T,
+            "queries": wl.heads * wl.group, "keys_appended": wl.heads}
+
+
 def run_cpu_baseline(wl: workloads.Workload, target_s: float):
     """The oracle, as it stands (single thread), on a bounded sample of the
     workload: consecutive chunks of keys of one KV head (drawn by the workload's
@@ -397,6 +427,7 @@ def main():
 
     # end to end through the public API with host buffers
     e2e = run_e2e(wl, path, device, args.e2e_steps, world)
+    decode_step = run_decode_step(path, 200)
     clocks.stop()
 
     if rank != 0:
@@ -444,6 +475,7 @@ def main():
         "gpu_launches": 2 * args.steps,
         "clocks": clocks.summary(),
         "e2e": e2e,
+        "decode_step": decode_step,
         "cpu_baseline": cpu_baseline,
     }
     print(json.dumps(line), flush=True)

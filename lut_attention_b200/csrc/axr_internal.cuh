@@ -69,6 +69,14 @@ struct ScoresArgs {
     float *scores;
     Codebook cb;
     int64_t head_stride = 0;   // rows between KV heads in idx and norms (n for a dense cache)
+    // decode step fused into the read (tensor-core path): quantize k_new[h] into
+    // row append_pos (= n - 1) of head h of idx_out / norms_out (the same cache)
+    // before scoring it
+    const void *k_new = nullptr;
+    int kdtype = 0;
+    int64_t append_pos = -1;
+    uint8_t *idx_out = nullptr;
+    float *norms_out = nullptr;
 };
 
 // Kernel launchers (quantize_keys.cu, scores.cu).  They return cudaSuccess or

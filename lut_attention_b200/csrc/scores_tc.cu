@@ -118,6 +118,14 @@ struct TcParams {
     float inv_sc;              // 1 / (128 * S_c)
     int8_t hi[kMaxLevels];     // centroid digits
     int8_t lo[kMaxLevels];
+    // decode step: the key of KV head h in k_new (heads x 128, kdtype) is quantized
+    // into row append_pos of that head (the last key scored) before it is read
+    int append_pos;            // -1: no key to append
+    int kdtype;
+    const void *k_new;
+    uint8_t *idx_out;          // the packed rows and norms, writable
+    float *norms_out;
+    float bnd[kMaxLevels - 1]; // codebook decision boundaries (unit-vector scale)
 };
 
 constexpr int kMaxStreams = 3;
@@ -132,6 +140,7 @@ struct Smem {
     float inv[kMaxStreams][kInvSlots][8];   // per stream, head slot and query: 1 / (128 * S_q * S_c)
     float q[2048];                           // rotation scratch: S * NQ <= 16 query rows of d floats
     float qmax[kMaxStreams][4][8];           // per stream, warp and query: max |q''|
+    uint32_t arow[kMaxStreams][17];          // per stream: packed row of an appended key
 };
 constexpr int kSmemBook = 10240;
 static_assert(sizeof(Smem) <= kSmemBook, "bookkeeping area too small");
@@ -227,6 +236,53 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
     }
     fence_proxy_async_smem();
     return stream_sync(S, g, phase);
+}
+
+// Decode step: quantize the appended key of KV head h, exactly as the write path
+// defines it (sign flip, Walsh-Hadamard, norm, nearest centroid, packing), with
+// the stream's 128 threads (thread j owns coordinate j).  Stores its codes and
+// norm in the cache and leaves the packed row in S.arow[g] and the norm in *norm.
+template <int B, int NQ>
+__device__ bool append_key(const TcParams &p, Smem &S, int g, int h, float *norm, int &phase)
+{
+    constexpr int P = kD * B / 8;
+    constexpr int L = 1 << B;
+    const int tid = threadIdx.x & (kGroupThreads - 1);
+    float *y = S.q + g * NQ * kD;
+    const float x = (p.signs[tid] < 0 ? -1.0f : 1.0f) *
+                    load_q(p.k_new, p.kdtype, static_cast<int64_t>(h) * kD + tid);
+    y[tid] = x;
+    float ss = x * x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((tid & 31) == 0) S.qmax[g][tid >> 5][0] = ss;
+    if (tid <= P / 4) S.arow[g][tid] = 0u;
+    if (!stream_sync(S, g, phase)) return false;
+    for (int hh = 1; hh < kD; hh <<= 1) {
+        if (tid < kD / 2) {
+            const int i = (tid / hh) * 2 * hh + (tid % hh);
+            const float a = y[i], c = y[i + hh];
+            y[i] = a + c;
+            y[i + hh] = a - c;
+        }
+        if (!stream_sync(S, g, phase)) return false;
+    }
+    const float nk = sqrtf((S.qmax[g][0][0] + S.qmax[g][1][0]) + (S.qmax[g][2][0] + S.qmax[g][3][0]));
+    // u = y / (sqrt(d) ||k||); idx = number of boundaries below u (a zero key has
+    // u = 0 and takes the central index)
+    const float u = (nk > 0.0f) ? y[tid] / (sqrtf(static_cast<float>(kD)) * nk) : 0.0f;
+    uint32_t code = 0;
+#pragma unroll
+    for (int i = 0; i < L - 1; ++i) code += (u > p.bnd[i]) ? 1u : 0u;
+    const int bit = tid * B;
+    atomicOr(&S.arow[g][bit >> 5], code << (bit & 31));
+    if ((bit & 31) + B > 32) atomicOr(&S.arow[g][(bit >> 5) + 1], code >> (32 - (bit & 31)));
+    if (!stream_sync(S, g, phase)) return false;
+    const int64_t row = static_cast<int64_t>(h) * p.head_stride + p.append_pos;
+    if (tid < P / 4) reinterpret_cast<uint32_t *>(p.idx_out + row * P)[tid] = S.arow[g][tid];
+    if (tid == 0) p.norms_out[row] = nk;
+    *norm = nk;
+    return true;
 }
 
 // table entry of one field value: C hi digits then C lo digits, replicated for
@@ -381,7 +437,7 @@ struct Worker {
                 w[NW] = 0;
             }
             // this tile's key norm (its scores are due two tiles from now)
-            const float nk = reinterpret_cast<const float *>(sStage + s * kStageBytes + kStageCodeBytes)
+            float nk = reinterpret_cast<const float *>(sStage + s * kStageBytes + kStageCodeBytes)
                 [((h * p.head_stride + ti * kTileRows + p.nshift) & 3) + r];
             mbar_arrive(smem_u32(&S.empty[s]));
 
@@ -410,6 +466,21 @@ struct Worker {
                     if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
                     ok = false;
                     break;
+                }
+            }
+            // decode step: this head's last tile holds the appended key, whose row
+            // the stage has only as it was before this launch
+            if (p.append_pos >= 0 && ti == (p.append_pos >> 7)) {
+                float nka;
+                if (!append_key<B, NQ>(p, S, g, h, &nka, sync_phase)) {
+                    if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                    ok = false;
+                    break;
+                }
+                if (r == (p.append_pos & (kTileRows - 1))) {
+#pragma unroll
+                    for (int i = 0; i < NW; ++i) w[i] = S.arow[g][i];
+                    nk = nka;
                 }
             }
 
@@ -676,6 +747,12 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     p.scores = a.scores;
     p.n = static_cast<int>(a.n);
     p.head_stride = static_cast<int>(a.head_stride);
+    p.append_pos = a.k_new ? static_cast<int>(a.append_pos) : -1;
+    p.kdtype = a.kdtype;
+    p.k_new = a.k_new;
+    p.idx_out = a.idx_out;
+    p.norms_out = a.norms_out;
+    for (int i = 0; i < kMaxLevels - 1; ++i) p.bnd[i] = a.cb.boundaries[i];
     p.group = a.group;
     p.tiles_per_head = static_cast<int>((a.n + kTileRows - 1) / kTileRows);
     p.total_tiles = p.tiles_per_head * a.heads;

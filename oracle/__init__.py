@@ -193,3 +193,32 @@ def dequant_scores(q, packed, norms, group: int, b: int, signs) -> np.ndarray:
     _check(_load().oracle_dequant_scores(_ptr(q), _ptr(packed), _ptr(norms), n, heads, group, d,
                                          b, _ptr(_signs(signs, d)), _ptr(out)), "dequant_scores")
     return out
+
+
+def attention_from_scores(s: np.ndarray, V: np.ndarray, group: int) -> np.ndarray:
+    """Decode attention after the scores (fp64): for query head h*group + g,
+    p = softmax(s[h*group + g, :]) over the n keys of KV head h, and the output
+    is sum_t p_t V[h, t, :].  s: (heads*group, n); V: (heads, n, d) as stored.
+
+    The pages define the scores only; softmax over a query's scores and the
+    weighted sum of the value rows is the standard attention that consumes them.
+    The values are read as given (not quantized).
+    """
+    s = np.asarray(s, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    heads, n, d = V.shape
+    if s.shape != (heads * group, n):
+        raise ValueError(f"scores must be ({heads * group}, {n})")
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    p /= p.sum(axis=1, keepdims=True)
+    out = np.empty((heads * group, d), dtype=np.float64)
+    for h in range(heads):
+        out[h * group:(h + 1) * group] = p[h * group:(h + 1) * group] @ V[h]
+    return out
+
+
+def attention(q, packed, norms, V, group: int, b: int, signs) -> np.ndarray:
+    """Decode attention on the quantized keys: softmax of the LUT scores
+    (:func:`scores`) times the value rows, (heads*group, d) fp64."""
+    return attention_from_scores(scores(q, packed, norms, group, b, signs), V, group)

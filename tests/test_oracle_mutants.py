@@ -7,7 +7,6 @@ must pass them all, which shows the harness itself is sound.
 """
 import importlib.util
 import os
-import shutil
 import sys
 
 import pytest
@@ -46,6 +45,10 @@ PIN_CALLS = [
     ("test_margins_are_distances_to_decision_points", {}),
     ("test_lut_scores_equal_dequantized_dot", {"d": 64, "b": 3, "group": 2}),
     ("test_scores_brute_force_d8", {}),
+    ("test_attention_of_equal_scores_is_the_mean_value_row", {}),
+    ("test_attention_single_key_returns_its_value_row", {}),
+    ("test_attention_brute_force_on_dequantized_keys", {}),
+    ("test_attention_is_linear_in_values_and_shift_free_in_scores", {}),
 ]
 
 # name -> (text in oracle.c, replacement): one plausible mistake each
@@ -86,12 +89,22 @@ MUTANTS = {
         "boundaries[i] = centroids[i];"),
 }
 
+# mistakes in the Python half of the oracle (__init__.py): name -> (text, replacement)
+PY_MUTANTS = {
+    "attention_reads_wrong_value_head": (
+        "out[h * group:(h + 1) * group] = p[h * group:(h + 1) * group] @ V[h]",
+        "out[h * group:(h + 1) * group] = p[h * group:(h + 1) * group] @ V[(h + 1) % heads]"),
+    "softmax_not_normalised": (
+        "    p /= p.sum(axis=1, keepdims=True)\n",
+        ""),
+}
+
 # the MSB-first mutant changes packing on both sides, as a consistent mistake would
 UNPACK_MSB = ("v |= (unsigned)((row[bit / 8] >> (bit % 8)) & 1) << i;",
               "v |= (unsigned)((row[bit / 8] >> (7 - bit % 8)) & 1) << i;")
 
 
-def _build_copy(tmp_path, name, edits):
+def _build_copy(tmp_path, name, edits, py_edits=()):
     pkg = tmp_path / f"oracle_{name}"
     pkg.mkdir()
     src = open(os.path.join(ORACLE_DIR, "oracle.c")).read()
@@ -99,7 +112,11 @@ def _build_copy(tmp_path, name, edits):
         assert src.count(old) == 1, f"{name}: edit target not found once: {old}"
         src = src.replace(old, new)
     (pkg / "oracle.c").write_text(src)
-    shutil.copy(os.path.join(ORACLE_DIR, "__init__.py"), pkg / "__init__.py")
+    py = open(os.path.join(ORACLE_DIR, "__init__.py")).read()
+    for old, new in py_edits:
+        assert py.count(old) == 1, f"{name}: edit target not found once: {old}"
+        py = py.replace(old, new)
+    (pkg / "__init__.py").write_text(py)
     modname = f"oracle_copy_{name}"
     spec = importlib.util.spec_from_file_location(modname, pkg / "__init__.py",
                                                   submodule_search_locations=[str(pkg)])
@@ -130,5 +147,12 @@ def test_unmodified_copy_passes_every_pin(tmp_path, monkeypatch):
 def test_planted_mistake_fails_a_pin(tmp_path, monkeypatch, name):
     edits = [MUTANTS[name]] + ([UNPACK_MSB] if name == "msb_first_packing" else [])
     mod = _build_copy(tmp_path, name, edits)
+    failed = _failing_pins(monkeypatch, mod)
+    assert failed, f"no pin catches the planted mistake {name}"
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_planted_mistake_in_the_python_half_fails_a_pin(tmp_path, monkeypatch, name):
+    mod = _build_copy(tmp_path, name, [], [PY_MUTANTS[name]])
     failed = _failing_pins(monkeypatch, mod)
     assert failed, f"no pin catches the planted mistake {name}"

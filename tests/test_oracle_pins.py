@@ -368,3 +368,59 @@ def test_workloads_deterministic_and_shaped():
         assert torch.isfinite(k.float()).all()
         q = workloads.make_queries(small)
         assert q.shape == (small.heads * w.group, w.d)
+
+
+# ---------------------------------------------------------------- attention --
+
+def test_attention_of_equal_scores_is_the_mean_value_row():
+    """q = 0 gives every key the score 0, so the softmax is uniform."""
+    d, b, heads, n, group = 16, 3, 2, 37, 2
+    rng = np.random.default_rng(5)
+    s = _rng_signs(d, 5)
+    packed, norms, _ = oracle.quantize(rng.standard_normal((heads * n, d)), b, s)
+    V = rng.standard_normal((heads, n, d))
+    out = oracle.attention(np.zeros((heads * group, d)), packed.reshape(heads, n, -1), norms.reshape(heads, n),
+                           V, group, b, s)
+    for h in range(heads):
+        for g in range(group):
+            assert np.allclose(out[h * group + g], V[h].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_attention_single_key_returns_its_value_row():
+    d, b = 8, 2
+    s = _rng_signs(d, 6)
+    packed, norms, _ = oracle.quantize(np.arange(1.0, d + 1.0)[None], b, s)
+    V = np.arange(d, dtype=np.float64)[None, None] * 0.5
+    out = oracle.attention(np.ones((3, d)), packed[None], norms[None], V, 3, b, s)
+    assert np.array_equal(out, np.repeat(V[0], 3, axis=0))
+
+
+def test_attention_brute_force_on_dequantized_keys():
+    """Independent of the oracle's numpy path: scores on dequantized,
+    inverse-rotated keys, then softmax and the weighted sum in plain loops."""
+    d, b, heads, n, group = 8, 2, 2, 5, 2
+    rng = np.random.default_rng(7)
+    s = _rng_signs(d, 7)
+    K = rng.standard_normal((heads * n, d)) * 3.0
+    packed, norms, _ = oracle.quantize(K, b, s)
+    packed, norms = packed.reshape(heads, n, -1), norms.reshape(heads, n)
+    q = rng.standard_normal((heads * group, d))
+    V = rng.standard_normal((heads, n, d))
+    sd = oracle.dequant_scores(q, packed, norms, group, b, s)
+    got = oracle.attention(q, packed, norms, V, group, b, s)
+    for row in range(heads * group):
+        h = row // group
+        w = [math.exp(sd[row, t]) for t in range(n)]
+        tot = sum(w)
+        for j in range(d):
+            exp_v = sum(w[t] * V[h, t, j] for t in range(n)) / tot
+            assert abs(got[row, j] - exp_v) <= 1e-12 * (1.0 + abs(exp_v))
+
+
+def test_attention_is_linear_in_values_and_shift_free_in_scores():
+    rng = np.random.default_rng(8)
+    s = rng.standard_normal((6, 40)) * 4.0
+    V = rng.standard_normal((3, 40, 8))
+    a = oracle.attention_from_scores(s, V, 2)
+    assert np.allclose(oracle.attention_from_scores(s + 123.0, V, 2), a, rtol=1e-13, atol=1e-13)
+    assert np.allclose(oracle.attention_from_scores(s, 2.5 * V - 1.0, 2), 2.5 * a - 1.0, rtol=1e-13, atol=1e-13)

@@ -266,6 +266,38 @@ def run_decode_step(path: Path, steps: int) -> dict:
             "queries": wl.heads * wl.group, "keys_appended": wl.heads}
 
 
+def run_attention(path: Path, steps: int) -> dict:
+    """Decode attention on the cache (axr_attention: scores, then the softmax of
+    every query head's scores and the weighted sum of bf16 value rows)."""
+    wl = path.wl
+    g = torch.Generator(device=path.K.device).manual_seed(4242)
+    V = torch.randn((wl.heads, wl.T, wl.d), generator=g, device=path.K.device).to(torch.bfloat16)
+    ws = torch.empty(axr.axr_attention_workspace_bytes(wl.T, wl.heads, wl.group, wl.d), dtype=torch.uint8,
+                     device=path.K.device)
+    out = torch.empty((wl.heads * wl.group, wl.d), dtype=torch.float32, device=path.K.device)
+
+    def step():
+        axr.axr_attention(path.q, path.idx[0], path.norms[0], V, wl.group, wl.b, path.signs, scores=path.scores,
+                          workspace=ws, out=out)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    # per key: packed row + norm + scores written and read back + bf16 value row
+    per_key = wl.d * wl.b // 8 + 4 + 8 * wl.group + 2 * wl.d
+    byts = wl.rows * per_key
+    del V, ws
+    return {"ms": ms, "algo_bytes": byts, "gbs": byts / (ms * 1e-3) / 1e9, "bytes_per_key": per_key,
+            "value_dtype": "bf16", "launches": 3}
+
+
 def run_cpu_baseline(wl: workloads.Workload, target_s: float):
     """The oracle, as it stands (single thread), on a bounded sample of the
     workload: consecutive chunks of keys of one KV head (drawn by the workload's
@@ -428,6 +460,7 @@ def main():
     # end to end through the public API with host buffers
     e2e = run_e2e(wl, path, device, args.e2e_steps, world)
     decode_step = run_decode_step(path, 200)
+    attention = run_attention(path, 100)
     clocks.stop()
 
     if rank != 0:
@@ -476,6 +509,7 @@ def main():
         "clocks": clocks.summary(),
         "e2e": e2e,
         "decode_step": decode_step,
+        "attention": attention,
         "cpu_baseline": cpu_baseline,
     }
     print(json.dumps(line), flush=True)

@@ -138,6 +138,30 @@ int axr_append_scores(const void *k_new, int kdtype, const void *q, int qdtype, 
                       const int8_t *signs, float *scores, axr_stream stream);
 
 /*
+ * Decode attention on the quantized keys.  The pages define the scores only; this
+ * is the standard attention that consumes them: for query head h*group + g,
+ *   p = softmax over t of scores[h*group + g, t]     (t = 0 .. n-1)
+ *   out[h*group + g, :] = sum_t p_t * V[h, t, :]
+ * with the scores exactly as axr_scores computes them (they are also returned).
+ * The values are read as stored (not quantized).
+ *
+ * q, idx, norms, signs as for axr_scores (16/16/4/1-byte aligned).
+ * V          device, heads x n x d row-major, element type vdtype; 16-byte aligned.
+ * scores     device float[(heads*group) * n] output (the scores); 16-byte aligned.
+ * workspace  device scratch of at least axr_attention_workspace_bytes(...) bytes,
+ *            16-byte aligned, owned by the caller; its contents on entry do not
+ *            matter and on exit are unspecified.  Calls that share a workspace
+ *            must not overlap in time.
+ * out        device float[(heads*group) * d] output.
+ * d must be a power of two in [32, 512]; n >= 1.  Three kernels are enqueued on
+ * `stream` in order (scores, per-chunk partial softmax sums, their merge).
+ */
+int axr_attention_workspace_bytes(int64_t n, int heads, int group, int d, int64_t *bytes);
+int axr_attention(const void *q, int qdtype, const uint8_t *idx, const float *norms, const void *V, int vdtype,
+                  int64_t n, int heads, int group, int d, int b, const int8_t *signs, float *scores,
+                  void *workspace, int64_t workspace_bytes, float *out, axr_stream stream);
+
+/*
  * Device-side status of the tensor-core kernels (no counterpart in the method;
  * a diagnostic).  Every wait inside those kernels is bounded; a wait that runs
  * out records a bit here instead of hanging: 1 = a tile load never arrived,

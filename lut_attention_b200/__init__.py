@@ -8,6 +8,8 @@ load the library; the first call does, and raises if it has not been built.
 from .axr import (  # noqa: F401
     AxrError,
     axr_append_scores,
+    axr_attention,
+    axr_attention_workspace_bytes,
     axr_device_status,
     axr_make_codebook,
     axr_quantize_keys,
@@ -19,6 +21,8 @@ from .axr import (  # noqa: F401
 __all__ = [
     "AxrError",
     "axr_append_scores",
+    "axr_attention",
+    "axr_attention_workspace_bytes",
     "axr_device_status",
     "axr_make_codebook",
     "axr_quantize_keys",

@@ -28,6 +28,8 @@ SIGNATURES = {
     "axr_quantize_keys": (_I32, [_P, _I32, _I64, _I32, _I32, _P, _P, _P, _P]),
     "axr_scores": (_I32, [_P, _I32, _P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
     "axr_append_scores": (_I32, [_P, _I32, _P, _I32, _P, _P, _I64, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
+    "axr_attention_workspace_bytes": (_I32, [_I64, _I32, _I32, _I32, _P]),
+    "axr_attention": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _I64, _P, _P]),
     "axr_status_string": (ctypes.c_char_p, [_I32]),
     "axr_last_error": (ctypes.c_char_p, []),
     "axr_version": (_I32, []),
@@ -191,6 +193,56 @@ def axr_append_scores(k_new: torch.Tensor, q: torch.Tensor, idx: torch.Tensor, n
                                      _stream_handle(stream))
     _raise(rc, "axr_append_scores")
     return scores
+
+
+def axr_attention_workspace_bytes(n: int, heads: int, group: int, d: int) -> int:
+    """Scratch bytes axr_attention needs for this shape."""
+    out = ctypes.c_int64(0)
+    _raise(library().axr_attention_workspace_bytes(n, heads, group, d, ctypes.byref(out)),
+           "axr_attention_workspace_bytes")
+    return out.value
+
+
+def axr_attention(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, V: torch.Tensor, group: int, b: int,
+                  signs: torch.Tensor, scores: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                  out: torch.Tensor | None = None, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Decode attention on packed keys idx (heads, n, d*b/8) with norms (heads, n)
+    and values V (heads, n, d): returns (out (heads*group, d) fp32, scores
+    (heads*group, n) fp32).  A workspace is allocated when none is given."""
+    for t, name in ((q, "q"), (idx, "idx"), (norms, "norms"), (V, "V"), (signs, "signs")):
+        _require_cuda(t, name)
+    if q.dtype not in _DTYPE_CODE or V.dtype not in _DTYPE_CODE:
+        raise ValueError("q and V must be float32, float16 or bfloat16")
+    if idx.dtype != torch.uint8 or norms.dtype != torch.float32 or signs.dtype != torch.int8:
+        raise ValueError("idx must be uint8, norms float32, signs int8")
+    hg, d = q.shape
+    if group < 1 or hg % group:
+        raise ValueError("q must have heads*group rows")
+    heads = hg // group
+    if idx.dim() != 3 or idx.shape[0] != heads or idx.shape[2] != packed_row_bytes(d, b):
+        raise ValueError(f"idx must be (heads={heads}, n, {packed_row_bytes(d, b)})")
+    n = idx.shape[1]
+    if tuple(norms.shape) != (heads, n) or tuple(V.shape) != (heads, n, d):
+        raise ValueError(f"norms must be ({heads}, {n}) and V ({heads}, {n}, {d})")
+    if scores is None:
+        scores = torch.empty((hg, n), dtype=torch.float32, device=q.device)
+    if out is None:
+        out = torch.empty((hg, d), dtype=torch.float32, device=q.device)
+    need = axr_attention_workspace_bytes(n, heads, group, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    for t, name in ((scores, "scores"), (out, "out"), (workspace, "workspace")):
+        _require_cuda(t, name)
+    if scores.numel() < hg * n or out.numel() < hg * d or scores.dtype != torch.float32 \
+            or out.dtype != torch.float32:
+        raise ValueError("scores and out must be float32 and large enough")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = library().axr_attention(q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(),
+                                 V.data_ptr(), _DTYPE_CODE[V.dtype], n, heads, group, d, b, signs.data_ptr(),
+                                 scores.data_ptr(), workspace.data_ptr(), ws_bytes, out.data_ptr(),
+                                 _stream_handle(stream))
+    _raise(rc, "axr_attention")
+    return out, scores
 
 
 def axr_device_status(clear: bool = True) -> int:

@@ -211,6 +211,55 @@ extern "C" int axr_append_scores(const void *k_new, int kdtype, const void *q, i
     return ok();
 }
 
+extern "C" int axr_attention_workspace_bytes(int64_t n, int heads, int group, int d, int64_t *bytes)
+{
+    if (!bytes) return fail(AXR_EINVAL, "bytes is NULL");
+    if (!pow2_in_range(d) || d < 32) return fail(AXR_EUNSUPPORTED, "d=%d: attention needs a power of two in [32, 512]", d);
+    if (n < 0 || heads < 1 || group < 1) return fail(AXR_EINVAL, "n, heads or group out of range");
+    if (group > kMaxGroup) return fail(AXR_EUNSUPPORTED, "group=%d: at most %d", group, kMaxGroup);
+    *bytes = n == 0 ? 0 : attention_workspace_bytes(n, heads, group, d);
+    return ok();
+}
+
+extern "C" int axr_attention(const void *q, int qdtype, const uint8_t *idx, const float *norms, const void *V,
+                             int vdtype, int64_t n, int heads, int group, int d, int b, const int8_t *signs,
+                             float *scores, void *workspace, int64_t workspace_bytes, float *out,
+                             axr_stream stream)
+{
+    int rc = check_shape(d, b);
+    if (rc != AXR_OK) return rc;
+    if (d < 32) return fail(AXR_EUNSUPPORTED, "d=%d: attention needs d >= 32", d);
+    if (elem_size(qdtype) == 0) return fail(AXR_EINVAL, "qdtype=%d is not an axr_dtype", qdtype);
+    if (elem_size(vdtype) == 0) return fail(AXR_EINVAL, "vdtype=%d is not an axr_dtype", vdtype);
+    if (n < 1) return fail(AXR_EINVAL, "n=%lld: attention needs at least one key", (long long)n);
+    if (heads < 1) return fail(AXR_EINVAL, "heads=%d must be >= 1", heads);
+    if (group < 1) return fail(AXR_EINVAL, "group=%d must be >= 1", group);
+    if (group > kMaxGroup) return fail(AXR_EUNSUPPORTED, "group=%d: at most %d", group, kMaxGroup);
+    if (n > (int64_t)INT32_MAX) return fail(AXR_EUNSUPPORTED, "n=%lld: at most 2^31-1 keys per head", (long long)n);
+    const int64_t need = attention_workspace_bytes(n, heads, group, d);
+    if (workspace_bytes < need)
+        return fail(AXR_EINVAL, "workspace_bytes=%lld: needs %lld", (long long)workspace_bytes, (long long)need);
+    if ((rc = check_device_ptr(q, 16, "q")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(idx, 16, "idx")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(norms, 4, "norms")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(V, 16, "V")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(signs, 1, "signs")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(scores, 16, "scores")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(workspace, 16, "workspace")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(out, 4, "out")) != AXR_OK) return rc;
+
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    ScoresArgs sa{q, qdtype, idx, norms, n, heads, group, d, b, signs, scores, Codebook{}};
+    sa.head_stride = n;
+    if (!get_codebook(d, b, &sa.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
+    cudaError_t e = scores_tc_supported(sa) ? launch_scores_tc(sa, st) : launch_scores(sa, st);
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "scores launch: %s", cudaGetErrorString(e));
+    AttentionArgs aa{scores, V, vdtype, n, heads, group, d, workspace, out};
+    e = launch_attention(aa, st);
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "attention launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 extern "C" const char *axr_status_string(int status)
 {
     switch (status) {

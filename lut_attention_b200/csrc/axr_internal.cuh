@@ -94,6 +94,23 @@ bool scores_tc_supported(const ScoresArgs &a);
 cudaError_t launch_scores_tc(const ScoresArgs &a, cudaStream_t stream);
 unsigned int scores_tc_status(bool clear);
 
+// Decode attention after the scores (attention.cu): softmax over each query
+// head's n scores, weighted sum of its KV head's value rows.
+struct AttentionArgs {
+    const float *scores;       // (heads*group, n), already computed
+    const void *V;             // (heads, n, d), vdtype
+    int vdtype;
+    int64_t n;
+    int heads;
+    int group;
+    int d;
+    void *workspace;           // attention_workspace_bytes(n, heads, group, d)
+    float *out;                // (heads*group, d)
+};
+int attention_splits(int64_t n, int group);
+int64_t attention_workspace_bytes(int64_t n, int heads, int group, int d);
+cudaError_t launch_attention(const AttentionArgs &a, cudaStream_t stream);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

@@ -108,6 +108,23 @@ def test_append_argument_errors(axr_lib):
     assert f(p, 2, p, 2, p, p, 16, 3, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL         # host memory
 
 
+def test_attention_workspace_and_argument_errors(axr_lib):
+    # 32 heads x 64 chunks of 1024 keys x 4 queries x (128 + 2) floats
+    assert axr.axr_attention_workspace_bytes(131072, 32, 4, 128) == 32 * 128 * 4 * 130 * 4
+    assert axr.axr_attention_workspace_bytes(1, 1, 3, 64) == 1 * 1 * 4 * 66 * 4      # group padded to 4
+    out = ctypes.c_int64(0)
+    assert axr_lib.axr_attention_workspace_bytes(100, 1, 1, 16, ctypes.byref(out)) == axr.AXR_EUNSUPPORTED
+    f = axr_lib.axr_attention
+    host = np.zeros(4096, np.uint8)
+    p = host.ctypes.data
+    # (q, qdt, idx, norms, V, vdt, n, heads, group, d, b, signs, scores, ws, ws_bytes, out, stream)
+    assert f(p, 2, p, p, p, 2, 0, 1, 1, 128, 4, p, p, p, 1 << 20, p, None) == axr.AXR_EINVAL       # n = 0
+    assert f(p, 2, p, p, p, 2, 10, 1, 1, 16, 4, p, p, p, 1 << 20, p, None) == axr.AXR_EUNSUPPORTED  # d < 32
+    assert f(p, 2, p, p, p, 9, 10, 1, 1, 128, 4, p, p, p, 1 << 20, p, None) == axr.AXR_EINVAL      # V dtype
+    assert f(p, 2, p, p, p, 2, 10, 1, 1, 128, 4, p, p, p, 8, p, None) == axr.AXR_EINVAL            # workspace
+    assert f(p, 2, p, p, p, 2, 10, 1, 1, 128, 4, p, p, p, 1 << 20, p, None) == axr.AXR_EINVAL      # host memory
+
+
 def test_binding_refuses_cpu_tensors():
     """No CPU path: the binding raises instead of computing on the host."""
     K = torch.zeros(4, 128)

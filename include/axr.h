@@ -162,6 +162,33 @@ int axr_attention(const void *q, int qdtype, const uint8_t *idx, const float *no
                   void *workspace, int64_t workspace_bytes, float *out, axr_stream stream);
 
 /*
+ * axr_attention without a workspace argument: the same computation, with the
+ * partial sums kept in a fixed 16 MiB scratch area that the library carries in
+ * device memory (one per device).  The method has no counterpart to this call;
+ * it exists for callers that cannot hand the library device memory of their own:
+ * a plain C program with no device allocator at hand, code that runs with a fixed
+ * device-memory budget that must not grow, or a latency-bound decode loop that
+ * cannot afford the synchronisation an allocation may cause.
+ *
+ * Arguments as for axr_attention, less workspace and workspace_bytes.
+ * Limit: shapes whose axr_attention_workspace_bytes exceed 16 MiB (16777216
+ *   bytes) return AXR_EUNSUPPORTED with nothing enqueued; 131072 keys x 32 KV heads
+ *   x 4 queries per head at d = 128 need 8.5 MB.
+ * Set-up: the first call on a device looks up the scratch address there (with
+ *   that device current), and the first call for a (d, b) pair solves its
+ *   codebook on the host; later calls allocate nothing, on the host or the
+ *   device.  Make the first call on each device before any stream capture.
+ * Nothing in the scratch needs clearing: every call writes each partial sum it
+ *   later reads.
+ * Overlapping calls race: all calls on one device share the scratch, so two of
+ *   them in flight at once (on different streams or from different threads)
+ *   corrupt each other's results.  Order them (one stream, or events).
+ */
+int axr_attention_static(const void *q, int qdtype, const uint8_t *idx, const float *norms, const void *V,
+                         int vdtype, int64_t n, int heads, int group, int d, int b, const int8_t *signs,
+                         float *scores, float *out, axr_stream stream);
+
+/*
  * Device-side status of the tensor-core kernels (no counterpart in the method;
  * a diagnostic).  Every wait inside those kernels is bounded; a wait that runs
  * out records a bit here instead of hanging: 1 = a tile load never arrived,

@@ -9,6 +9,7 @@ from .axr import (  # noqa: F401
     AxrError,
     axr_append_scores,
     axr_attention,
+    axr_attention_static,
     axr_attention_workspace_bytes,
     axr_device_status,
     axr_make_codebook,
@@ -22,6 +23,7 @@ __all__ = [
     "AxrError",
     "axr_append_scores",
     "axr_attention",
+    "axr_attention_static",
     "axr_attention_workspace_bytes",
     "axr_device_status",
     "axr_make_codebook",

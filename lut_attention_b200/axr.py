@@ -30,6 +30,7 @@ SIGNATURES = {
     "axr_append_scores": (_I32, [_P, _I32, _P, _I32, _P, _P, _I64, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
     "axr_attention_workspace_bytes": (_I32, [_I64, _I32, _I32, _I32, _P]),
     "axr_attention": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _I64, _P, _P]),
+    "axr_attention_static": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _P]),
     "axr_status_string": (ctypes.c_char_p, [_I32]),
     "axr_last_error": (ctypes.c_char_p, []),
     "axr_version": (_I32, []),
@@ -242,6 +243,37 @@ def axr_attention(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, V: to
                                  scores.data_ptr(), workspace.data_ptr(), ws_bytes, out.data_ptr(),
                                  _stream_handle(stream))
     _raise(rc, "axr_attention")
+    return out, scores
+
+
+def axr_attention_static(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, V: torch.Tensor, group: int,
+                         b: int, signs: torch.Tensor, scores: torch.Tensor, out: torch.Tensor,
+                         stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """axr_attention with the library's fixed scratch instead of a workspace.
+    scores (heads*group, n) and out (heads*group, d), fp32, come from the caller:
+    this call allocates nothing.  Calls on one device must not overlap."""
+    for t, name in ((q, "q"), (idx, "idx"), (norms, "norms"), (V, "V"), (signs, "signs"), (scores, "scores"),
+                    (out, "out")):
+        _require_cuda(t, name)
+    if q.dtype not in _DTYPE_CODE or V.dtype not in _DTYPE_CODE:
+        raise ValueError("q and V must be float32, float16 or bfloat16")
+    hg, d = q.shape
+    if group < 1 or hg % group:
+        raise ValueError("q must have heads*group rows")
+    heads = hg // group
+    if idx.dim() != 3 or idx.shape[0] != heads or idx.shape[2] != packed_row_bytes(d, b):
+        raise ValueError(f"idx must be (heads={heads}, n, {packed_row_bytes(d, b)})")
+    n = idx.shape[1]
+    if tuple(norms.shape) != (heads, n) or tuple(V.shape) != (heads, n, d):
+        raise ValueError(f"norms must be ({heads}, {n}) and V ({heads}, {n}, {d})")
+    if scores.dtype != torch.float32 or out.dtype != torch.float32 or scores.numel() < hg * n \
+            or out.numel() < hg * d:
+        raise ValueError("scores and out must be float32 and large enough")
+    rc = library().axr_attention_static(q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(),
+                                        V.data_ptr(), _DTYPE_CODE[V.dtype], n, heads, group, d, b,
+                                        signs.data_ptr(), scores.data_ptr(), out.data_ptr(),
+                                        _stream_handle(stream))
+    _raise(rc, "axr_attention_static")
     return out, scores
 
 

@@ -260,6 +260,49 @@ extern "C" int axr_attention(const void *q, int qdtype, const uint8_t *idx, cons
     return ok();
 }
 
+extern "C" int axr_attention_static(const void *q, int qdtype, const uint8_t *idx, const float *norms,
+                                    const void *V, int vdtype, int64_t n, int heads, int group, int d, int b,
+                                    const int8_t *signs, float *scores, float *out, axr_stream stream)
+{
+    int rc = check_shape(d, b);
+    if (rc != AXR_OK) return rc;
+    if (d < 32) return fail(AXR_EUNSUPPORTED, "d=%d: attention needs d >= 32", d);
+    if (elem_size(qdtype) == 0) return fail(AXR_EINVAL, "qdtype=%d is not an axr_dtype", qdtype);
+    if (elem_size(vdtype) == 0) return fail(AXR_EINVAL, "vdtype=%d is not an axr_dtype", vdtype);
+    if (n < 1) return fail(AXR_EINVAL, "n=%lld: attention needs at least one key", (long long)n);
+    if (heads < 1) return fail(AXR_EINVAL, "heads=%d must be >= 1", heads);
+    if (group < 1) return fail(AXR_EINVAL, "group=%d must be >= 1", group);
+    if (group > kMaxGroup) return fail(AXR_EUNSUPPORTED, "group=%d: at most %d", group, kMaxGroup);
+    if (n > (int64_t)INT32_MAX) return fail(AXR_EUNSUPPORTED, "n=%lld: at most 2^31-1 keys per head", (long long)n);
+    const int64_t need = attention_workspace_bytes(n, heads, group, d);
+    if (need > static_attention_scratch_bytes())
+        return fail(AXR_EUNSUPPORTED,
+                    "this shape needs %lld bytes of scratch; the fixed scratch holds %lld (use axr_attention "
+                    "with a workspace)",
+                    (long long)need, (long long)static_attention_scratch_bytes());
+    if ((rc = check_device_ptr(q, 16, "q")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(idx, 16, "idx")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(norms, 4, "norms")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(V, 16, "V")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(signs, 1, "signs")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(scores, 16, "scores")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(out, 4, "out")) != AXR_OK) return rc;
+
+    void *scratch = nullptr;
+    cudaError_t e = static_attention_scratch(&scratch);
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "fixed scratch address: %s", cudaGetErrorString(e));
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    ScoresArgs sa{q, qdtype, idx, norms, n, heads, group, d, b, signs, scores, Codebook{}};
+    sa.head_stride = n;
+    if (!get_codebook(d, b, &sa.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
+    e = scores_tc_supported(sa) ? launch_scores_tc(sa, st) : launch_scores(sa, st);
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "scores launch: %s", cudaGetErrorString(e));
+    AttentionArgs aa{scores, V, vdtype, n, heads, group, d, scratch, out};
+    e = launch_attention(aa, st);
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "attention launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 extern "C" const char *axr_status_string(int status)
 {
     switch (status) {

@@ -17,6 +17,8 @@
 //             out = sum_c e^(m_c - M) o_c / sum_c e^(m_c - M) l_c,  M = max_c m_c.
 // The value rows are the traffic (2d bytes per key in bf16); both kernels are
 // plain CUDA-core code.
+#include <mutex>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -24,6 +26,13 @@
 #include "axr_internal.cuh"
 
 namespace axr {
+
+// Fixed scratch for the partial sums of axr_attention_static, for callers that
+// cannot supply device memory of their own.  Part of the module image: it exists
+// once per device from the time the library's kernels are loaded there, and
+// every call of that entry point on the device uses the same bytes.
+constexpr int64_t kStaticScratchBytes = static_cast<int64_t>(16) << 20;
+static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
 namespace {
 
 constexpr int kChunkScores = 4096;    // scores staged per CTA (16 KB): chunk = 4096 / G keys
@@ -258,6 +267,28 @@ int64_t attention_workspace_bytes(int64_t n, int heads, int group, int d)
 {
     return static_cast<int64_t>(heads) * attention_splits(n, group) * padded_group(group) * (d + 2) *
            static_cast<int64_t>(sizeof(float));
+}
+
+int64_t static_attention_scratch_bytes() { return kStaticScratchBytes; }
+
+cudaError_t static_attention_scratch(void **ptr)
+{
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};      // per device, filled on its first call
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);      // with device `dev` current
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
 }
 
 cudaError_t launch_attention(const AttentionArgs &a, cudaStream_t stream)

@@ -110,6 +110,10 @@ struct AttentionArgs {
 int attention_splits(int64_t n, int group);
 int64_t attention_workspace_bytes(int64_t n, int heads, int group, int d);
 cudaError_t launch_attention(const AttentionArgs &a, cudaStream_t stream);
+// The fixed device scratch of axr_attention_static: its size, and its address on
+// the current device (looked up on the device's first call, cached after).
+int64_t static_attention_scratch_bytes();
+cudaError_t static_attention_scratch(void **ptr);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

@@ -33,13 +33,16 @@
 //                    of tile k - 2 are done, read its int32 sums (D), scale
 //                    them by the key norm and the query scale and store the
 //                    scores; then look up tile k's digits and store them to
-//                    A in the same buffer.  On entering a
-//                    new KV head they rotate its queries (sign flip,
-//                    Walsh-Hadamard butterflies, 1/d) and write their digits
-//                    into the other of the stream's two B buffers.
+//                    A in the same buffer.  On entering a new KV head they
+//                    rotate its queries (sign flip, Walsh-Hadamard
+//                    butterflies, 1/d) and write their digits into the other
+//                    of the stream's two B buffers.  In a decode step they
+//                    first quantize the head's new key when tile k is the
+//                    head's last (the one that holds it).
 //   1 MMA warp     : 8 tcgen05.mma (M = 128, N = 4G, K = 32) per tile and one
 //                    commit, which frees A and publishes D at once.
-// plus one TMA warp loading packed tiles HBM -> shared memory (6 stages).
+// plus one TMA warp loading each tile's packed rows and key norms HBM -> shared
+// memory (6 stages).
 // A tcgen05.mma issue blocks while the tensor pipe works, and a tile's 8
 // products take longer than its decode, so every stream has its own issuer:
 // together they keep the pipe fed while each waits for its own workers.

@@ -17,13 +17,24 @@ Recipes (``LogNormal(m, s)`` means ``exp(m + s * N(0,1))``):
                       KV head (seeded choice) are further scaled by 20.  With
                       ``head_sigma`` > 0 every (batch, KV head) is also scaled by
                       LogNormal(0, head_sigma) (per-head norm heterogeneity).
+* ``calibration``     calibration samples of one layer for choosing the sign
+                      pattern (the batch holds the samples): ``channel_scaled``
+                      keys whose KV-head scale LogNormal(0, head_sigma) belongs to
+                      the head and is shared by every sample, plus a fixed offset
+                      per KV head, ``key_bias`` times the head's channel scales
+                      times a seeded N(0,1)^d vector, the same for all tokens and
+                      samples.  Without a shared offset the distribution of the
+                      keys is symmetric in every coordinate, and then every sign
+                      pattern sees statistically the same keys.
 * ``unit_uniform``    rows of N(0,1)^d, normalised, times a norm ~ U(lo, hi).
 * ``student_t``       coordinates ~ Student-t(4) (a normal over the root of a
                       chi-square with 4 degrees of freedom / 4), rows renormalised
                       to a norm ~ U(lo, hi).
 
 Queries are N(0,1) in the workload's dtype.  The sign pattern D is a seeded
-+-1 int8 vector drawn on the CPU, one per workload (one per layer).
++-1 int8 vector drawn on the CPU, one per workload (one per layer); the
+candidates of a sign-pattern search are seeded +-1 rows, the first of them
+that default pattern.
 """
 from __future__ import annotations
 
@@ -50,6 +61,7 @@ class Workload:
     head_sigma: float = 0.0
     norm_lo: float = 0.0
     norm_hi: float = 0.0
+    key_bias: float = 0.0
 
     @property
     def heads(self) -> int:
@@ -83,6 +95,11 @@ WRITE_2E24 = Workload("write_2e24", 1, 1, 1, 128, 4, 1 << 24, "bf16", 4, "unit_u
 WIDE_D256 = Workload("wide_heads_d256", 16, 8, 2, 256, 2, 65536, "f16", 5, "student_t",
                      norm_lo=1.0, norm_hi=10.0)
 WIDE_D512 = WIDE_D256.with_(name="wide_heads_d512", d=512)
+# Sign-pattern search of one layer of the GQA shape: 8 calibration samples (the
+# batch) of 2048 tokens, 200 candidates.
+GQA_SIGN_CALIBRATION = Workload("gqa_sign_calibration", 8, 8, 4, 128, 4, 2048, "bf16", 6, "calibration",
+                                head_sigma=1.5, key_bias=1.0)
+SIGN_CANDIDATES = 200
 
 ALL = (PR1_REF, MHA_DECODE_32K, GQA_DECODE_128K, WRITE_2E24, WIDE_D256, WIDE_D512)
 BY_NAME = {w.name: w for w in ALL}
@@ -92,6 +109,16 @@ def make_signs(wl: Workload) -> torch.Tensor:
     """Seeded sign pattern D in {+1, -1}^d, int8, on the CPU."""
     g = torch.Generator(device="cpu").manual_seed(1_000_003 * wl.seed + wl.d)
     return (torch.randint(0, 2, (wl.d,), generator=g, dtype=torch.int8) * 2 - 1).to(torch.int8)
+
+
+def make_sign_candidates(wl: Workload, count: int) -> torch.Tensor:
+    """Seeded candidate sign patterns (count, d), int8 +-1, on the CPU; row 0 is
+    the workload's own pattern (:func:`make_signs`)."""
+    g = torch.Generator(device="cpu").manual_seed(2_000_029 * wl.seed + wl.d + count)
+    c = (torch.randint(0, 2, (count, wl.d), generator=g, dtype=torch.int8) * 2 - 1).to(torch.int8)
+    if count:
+        c[0] = make_signs(wl)
+    return c
 
 
 def make_queries(wl: Workload, device="cpu") -> torch.Tensor:
@@ -129,6 +156,22 @@ def make_keys(wl: Workload, device="cpu", chunk_rows: int = 1 << 20) -> torch.Te
                 t1 = min(T, t0 + chunk_rows)
                 z = torch.randn((t1 - t0, d), generator=g, device=device, dtype=torch.float32)
                 out[h, t0:t1] = (z * scale[h]).to(wl.torch_dtype)
+        return out
+
+    if wl.recipe == "calibration":
+        chan = _lognormal((wl.kv_heads, d), 1.0, g, device)
+        for h in range(wl.kv_heads):
+            pick = torch.randperm(d, generator=g, device=device)[:4]
+            chan[h, pick] *= 20.0
+        head = (_lognormal((wl.kv_heads,), wl.head_sigma, g, device) if wl.head_sigma > 0
+                else torch.ones(wl.kv_heads, device=device))
+        bias = wl.key_bias * torch.randn((wl.kv_heads, d), generator=g, device=device, dtype=torch.float32)
+        for s in range(wl.batch):
+            for h in range(wl.kv_heads):
+                for t0 in range(0, T, chunk_rows):
+                    t1 = min(T, t0 + chunk_rows)
+                    z = torch.randn((t1 - t0, d), generator=g, device=device, dtype=torch.float32)
+                    out[s * wl.kv_heads + h, t0:t1] = ((z + bias[h]) * chan[h] * head[h]).to(wl.torch_dtype)
         return out
 
     rows = heads * T

@@ -1,4 +1,4 @@
-"""CPU oracle for the AXELRAM write and read path: test infrastructure.
+"""CPU oracle for the AXELRAM write path, read path and sign-pattern choice: test infrastructure.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The CUDA library never uses it, and it
@@ -222,3 +222,54 @@ def attention(q, packed, norms, V, group: int, b: int, signs) -> np.ndarray:
     """Decode attention on the quantized keys: softmax of the LUT scores
     (:func:`scores`) times the value rows, (heads*group, d) fp64."""
     return attention_from_scores(scores(q, packed, norms, group, b, signs), V, group)
+
+
+def sign_errors(K, q, group: int, b: int, candidates) -> np.ndarray:
+    """Calibration score error of each candidate sign pattern, (C, heads) fp64.
+
+    AXELRAM abstract: the sign pattern D is chosen once, without gradients, from
+    a set of candidates (200) on a few calibration samples (8), which removes the
+    spikes that some patterns cause where key norms differ from head to head.  The
+    pages rank candidates by perplexity, which needs a model; this criterion is the
+    quantity the quantized cache perturbs, the attention logit.  For candidate
+    D_c every calibration key is quantized with D_c (:func:`quantize`) and scored
+    with D_c (:func:`scores`), and
+
+        E[c, h] = mean over samples s, query heads g < group and keys t of
+                  (score_c(q[s, h*group + g], k[s, h, t]) - q . k / sqrt(d))^2
+
+    is its mean squared error against the exact logit.
+
+    K: (samples, heads, n, d) keys; q: (samples, heads*group, d), the queries of
+    each sample; candidates: (C, d) of +-1.
+    """
+    K = np.asarray(K, dtype=np.float64)
+    if K.ndim != 4:
+        raise ValueError("K must be (samples, heads, n, d)")
+    S, heads, n, d = K.shape
+    q = np.asarray(q, dtype=np.float64)
+    if q.shape != (S, heads * group, d):
+        raise ValueError(f"q must be ({S}, {heads * group}, {d})")
+    cand = np.asarray(candidates)
+    if cand.ndim != 2 or cand.shape[1] != d:
+        raise ValueError(f"candidates must be (C, {d})")
+    if n == 0:
+        raise ValueError("no calibration keys")
+    sq = np.zeros((cand.shape[0], heads), dtype=np.float64)
+    for c in range(cand.shape[0]):
+        for s in range(S):
+            packed, norms, _ = quantize(K[s].reshape(heads * n, d), b, cand[c])
+            approx = scores(q[s], packed.reshape(heads, n, -1), norms.reshape(heads, n), group, b, cand[c])
+            for h in range(heads):
+                rows = slice(h * group, (h + 1) * group)
+                exact = q[s, rows] @ K[s, h].T / np.sqrt(d)
+                diff = approx[rows] - exact
+                sq[c, h] += np.sum(diff * diff)
+    return sq / (S * group * n)
+
+
+def select_signs(errors) -> int:
+    """The candidate whose worst head has the smallest error: argmin over c of
+    max over h of errors[c, h], the lowest index among equal values."""
+    worst = np.asarray(errors, dtype=np.float64).max(axis=1)
+    return int(np.argmin(worst))     # numpy returns the first of equal minima

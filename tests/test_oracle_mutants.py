@@ -49,6 +49,12 @@ PIN_CALLS = [
     ("test_attention_single_key_returns_its_value_row", {}),
     ("test_attention_brute_force_on_dequantized_keys", {}),
     ("test_attention_is_linear_in_values_and_shift_free_in_scores", {}),
+    ("test_sign_errors_brute_force_d8", {"b": 2}),
+    ("test_sign_errors_planted_pattern_closed_form", {"b": 4}),
+    ("test_sign_errors_symmetries_and_scaling", {}),
+    ("test_sign_errors_are_means_over_samples_queries_and_keys", {}),
+    ("test_sign_errors_match_lloyd_max_distortion", {"b": 3}),
+    ("test_select_signs_worst_head_and_lowest_index", {}),
 ]
 
 # name -> (text in oracle.c, replacement): one plausible mistake each
@@ -97,6 +103,18 @@ PY_MUTANTS = {
     "softmax_not_normalised": (
         "    p /= p.sum(axis=1, keepdims=True)\n",
         ""),
+    "exact_logit_without_temperature": (
+        "exact = q[s, rows] @ K[s, h].T / np.sqrt(d)",
+        "exact = q[s, rows] @ K[s, h].T"),
+    "sign_error_mean_over_keys_only": (
+        "return sq / (S * group * n)",
+        "return sq / n"),
+    "queries_read_with_first_candidate": (
+        "norms.reshape(heads, n), group, b, cand[c])",
+        "norms.reshape(heads, n), group, b, cand[0])"),
+    "selection_by_mean_over_heads": (
+        "worst = np.asarray(errors, dtype=np.float64).max(axis=1)",
+        "worst = np.asarray(errors, dtype=np.float64).mean(axis=1)"),
 }
 
 # the MSB-first mutant changes packing on both sides, as a consistent mistake would

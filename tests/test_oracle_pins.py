@@ -424,3 +424,151 @@ def test_attention_is_linear_in_values_and_shift_free_in_scores():
     a = oracle.attention_from_scores(s, V, 2)
     assert np.allclose(oracle.attention_from_scores(s + 123.0, V, 2), a, rtol=1e-13, atol=1e-13)
     assert np.allclose(oracle.attention_from_scores(s, 2.5 * V - 1.0, 2), 2.5 * a - 1.0, rtol=1e-13, atol=1e-13)
+
+
+# --------------------------------------------------- sign-pattern selection --
+# AXELRAM abstract: a gradient-free, one-time choice of the sign pattern among
+# candidates on a few calibration samples.  The criterion is the mean squared
+# error of the quantized attention logits against the exact ones, per KV head;
+# the choice minimises the worst head.
+
+def _calibration(S, heads, n, d, group, seed, C):
+    rng = np.random.default_rng(seed)
+    K = rng.standard_normal((S, heads, n, d)) * rng.lognormal(0, 1, (S, heads, 1, 1))
+    q = rng.standard_normal((S, heads * group, d))
+    cand = (rng.integers(0, 2, (C, d)) * 2 - 1).astype(np.int8)
+    return K, q, cand
+
+
+@pytest.mark.parametrize("b", [1, 2, 3])
+def test_sign_errors_brute_force_d8(b):
+    """Every calibration key dequantized through an explicit dense rotation and
+    a nearest-centroid search over all codewords, the logit error in loops."""
+    S, heads, n, d, group, C = 2, 2, 5, 8, 2, 3
+    K, q, cand = _calibration(S, heads, n, d, group, 30 + b, C)
+    cent, _ = oracle.codebook(d, b)
+    got = oracle.sign_errors(K, q, group, b, cand)
+    assert got.shape == (C, heads)
+    for c in range(C):
+        R = scipy.linalg.hadamard(d) * cand[c][None, :].astype(float) / math.sqrt(d)
+        for h in range(heads):
+            tot = 0.0
+            for s in range(S):
+                for t in range(n):
+                    k = K[s, h, t]
+                    norm = float(np.float32(math.sqrt(sum(x * x for x in k))))   # stored in fp32
+                    u = R @ k / math.sqrt(sum(x * x for x in k))
+                    code = [min(range(len(cent)), key=lambda l: abs(u[j] - float(cent[l]))) for j in range(d)]
+                    khat = R.T @ (norm * np.array([float(cent[l]) for l in code]))
+                    for g in range(group):
+                        qq = q[s, h * group + g]
+                        e = (np.dot(qq, khat) - np.dot(qq, k)) / math.sqrt(d)
+                        tot += e * e
+            expect = tot / (S * n * group)
+            assert abs(got[c, h] - expect) <= 1e-10 * expect
+
+
+@pytest.mark.parametrize("b", [2, 4])
+def test_sign_errors_planted_pattern_closed_form(b):
+    """Keys k = a (D* . h_r), h_r a Walsh-Hadamard row, and queries along them:
+    the pattern D* sends every key onto one rotated axis, u = e_r, which the
+    codebook maps to the top centroid c_max and every other coordinate (u_j = 0,
+    a tie with the central boundary) to the centroid c_0 just below zero.  A query
+    along a key of the same row gets the logit times c_max, error |q| |k|
+    (c_max - 1) / sqrt(d); along another row (exact logit 0) the error is
+    |q| |k| c_0 / sqrt(d) (|k| as stored, in fp32, where the method uses it).  D* and -D* are the two worst candidates and never
+    selected."""
+    d, S, heads, n, group = 128, 2, 3, 4, 2
+    rng = np.random.default_rng(40 + b)
+    H = scipy.linalg.hadamard(d).astype(float)
+    star = (rng.integers(0, 2, d) * 2 - 1).astype(np.int8)
+    K = np.empty((S, heads, n, d))
+    q = np.empty((S, heads * group, d))
+    for s in range(S):
+        for h in range(heads):
+            for t in range(n):
+                K[s, h, t] = 2.0 ** (h - t % 2) * star * H[rng.integers(0, d)]
+            for g in range(group):
+                q[s, h * group + g] = (g + 1) * 0.5 * K[s, h, 0]
+    cand = np.concatenate([(rng.integers(0, 2, (6, d)) * 2 - 1).astype(np.int8), star[None], -star[None]])
+    E = oracle.sign_errors(K, q, group, b, cand)
+    cent = oracle.codebook(d, b)[0].astype(np.float64)
+    c_max, c_0 = cent[-1], cent[(1 << b) // 2 - 1]
+    for h in range(heads):
+        expect = 0.0
+        for s in range(S):
+            k0 = K[s, h, 0] / np.linalg.norm(K[s, h, 0])
+            for t in range(n):
+                for g in range(group):
+                    qn, kn = np.linalg.norm(q[s, h * group + g]), np.linalg.norm(K[s, h, t])
+                    kn32 = float(np.float32(kn))                    # the stored norm
+                    same = np.array_equal(K[s, h, t] / kn, k0)     # queries lie along key 0
+                    e = qn * ((kn32 * c_max - kn) if same else kn32 * c_0) / math.sqrt(d)
+                    expect += e * e
+        expect /= S * n * group
+        for c in (6, 7):
+            assert abs(E[c, h] - expect) <= 1e-9 * expect
+    worst = E.max(axis=1)
+    assert worst[6] > 10 * worst[:6].max() and worst[7] > 10 * worst[:6].max()
+    assert oracle.select_signs(E) < 6
+
+
+def test_sign_errors_symmetries_and_scaling():
+    """-D gives the same errors as D (the codebook is symmetric); doubling the
+    keys or the queries multiplies every error by 4 exactly."""
+    S, heads, n, d, group, C = 2, 2, 30, 64, 3, 3
+    K, q, cand = _calibration(S, heads, n, d, group, 50, C)
+    E = oracle.sign_errors(K, q, group, 3, cand)
+    assert np.array_equal(oracle.sign_errors(K, q, group, 3, -cand), E)
+    assert np.array_equal(oracle.sign_errors(2.0 * K, q, group, 3, cand), 4.0 * E)
+    assert np.array_equal(oracle.sign_errors(K, 2.0 * q, group, 3, cand), 4.0 * E)
+
+
+def test_sign_errors_are_means_over_samples_queries_and_keys():
+    """Two samples of equal size average their errors; a group of identical
+    query heads has the error of one; the order of the keys does not matter."""
+    S, heads, n, d, group, C = 2, 3, 40, 32, 1, 4
+    K, q, cand = _calibration(S, heads, n, d, group, 60, C)
+    b = 2
+    E = oracle.sign_errors(K, q, group, b, cand)
+    E0 = oracle.sign_errors(K[:1], q[:1], group, b, cand)
+    E1 = oracle.sign_errors(K[1:], q[1:], group, b, cand)
+    np.testing.assert_allclose(E, 0.5 * (E0 + E1), rtol=1e-12)
+    q3 = np.repeat(q, 3, axis=1)                       # query head h*3 + g repeats q[:, h]
+    np.testing.assert_allclose(oracle.sign_errors(K, q3, 3, b, cand), E, rtol=1e-12)
+    perm = np.random.default_rng(61).permutation(n)
+    np.testing.assert_allclose(oracle.sign_errors(K[:, :, perm], q, group, b, cand), E, rtol=1e-12)
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_sign_errors_match_lloyd_max_distortion(b):
+    """Isotropic keys and queries with |q|^2 = d: each rotated coordinate is
+    quantized with the Lloyd-Max error D_b / d of Max's table, so the logit error
+    is about |q|^2 E|k|^2 D_b / d^2 = D_b (within 6%: sampling, and the unit-norm
+    constraint couples the coordinates)."""
+    mse = {}
+    with open(os.path.join(GOLDEN, "lloyd_max_classical.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                parts = line.split()
+                mse[int(parts[0])] = float(parts[1])
+    rng = np.random.default_rng(70 + b)
+    d, n, group = 128, 3000, 8
+    K = rng.standard_normal((1, 1, n, d))
+    q = rng.standard_normal((1, group, d))
+    q *= math.sqrt(d) / np.linalg.norm(q, axis=2, keepdims=True)
+    cand = _rng_signs(d, 71)[None]
+    E = oracle.sign_errors(K, q, group, b, cand)[0, 0]
+    assert abs(E / mse[b] - 1.0) < 0.06, E / mse[b]
+
+
+def test_select_signs_worst_head_and_lowest_index():
+    E = np.array([[1.0, 5.0], [3.0, 3.0], [2.0, 4.0], [3.0, 2.5], [0.5, 3.0]])
+    assert oracle.select_signs(E) == 1          # worst heads 5, 3, 4, 3, 3: the first 3
+    assert oracle.select_signs(E[2:]) == 1
+    S, heads, n, d, group = 1, 2, 20, 16, 2
+    K, q, cand = _calibration(S, heads, n, d, group, 80, 3)
+    dup = np.stack([cand[0], cand[1], cand[1], -cand[1], cand[2]])
+    Ed = oracle.sign_errors(K, q, group, 2, dup)
+    assert np.array_equal(Ed[1], Ed[2]) and np.array_equal(Ed[1], Ed[3])
+    assert oracle.select_signs(Ed) != 2 and oracle.select_signs(Ed) != 3

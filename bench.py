@@ -298,6 +298,63 @@ def run_attention(path: Path, steps: int) -> dict:
             "value_dtype": "bf16", "launches": 3}
 
 
+# fp32 lanes of one B200 SM and its maximum SM clock: the ALU roofline of the
+# CUDA-core sign-choice kernel is 148 SMs x 128 lanes x 1.965 GHz (one op per
+# lane per cycle, an FMA counted as one op)
+ALU_LANES_PER_SM = 128
+SM_MAX_GHZ = 1.965
+
+
+def sign_select_ops_per_key(wl: workloads.Workload) -> int:
+    """Arithmetic that scoring one calibration key against one candidate needs:
+    the Walsh-Hadamard butterflies (d log2 d), the squared norm and the
+    normalisation (2d), a b-step binary search (d b compares), the residual (d),
+    the projection on G rotated queries (G d FMAs), and scaling and squaring
+    each of the G logit errors (2G)."""
+    d = wl.d
+    return d * (d.bit_length() - 1) + 2 * d + d * wl.b + d + wl.group * d + 2 * wl.group
+
+
+def run_sign_select(device, steps: int) -> dict:
+    """The one-time sign-pattern choice of one layer of the GQA shape: 200
+    candidates on 8 calibration samples of 2048 tokens (axr_select_signs: the
+    error kernel and the argmin)."""
+    wl = workloads.GQA_SIGN_CALIBRATION
+    K = workloads.make_keys(wl, device).reshape(wl.batch, wl.kv_heads, wl.T, wl.d)
+    q = workloads.make_queries(wl, device).reshape(wl.batch, wl.kv_heads * wl.group, wl.d)
+    C = workloads.SIGN_CANDIDATES
+    cand = workloads.make_sign_candidates(wl, C).to(device)
+    errors = torch.empty((C, wl.kv_heads), dtype=torch.float32, device=device)
+    best = torch.empty(1, dtype=torch.int32, device=device)
+
+    def step():
+        axr.axr_select_signs(K, q, wl.group, wl.b, cand, errors=errors, best=best)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    key_cands = wl.rows * C
+    ops = key_cands * sign_select_ops_per_key(wl)
+    peak = torch.cuda.get_device_properties(device).multi_processor_count * ALU_LANES_PER_SM * SM_MAX_GHZ * 1e9
+    out = {"ms": ms, "candidates": C, "samples": wl.batch, "kv_heads": wl.kv_heads, "tokens": wl.T,
+           "chosen": int(best.item()), "key_candidates_per_s": key_cands / (ms * 1e-3),
+           "roofline": {"bound": "alu", "kernel": "sign_errors", "source": "sign_select.cu",
+                        "ops_per_key_candidate": sign_select_ops_per_key(wl),
+                        "achieved": ops / (ms * 1e-3) / 1e12, "peak": peak / 1e12, "unit": "Tops/s",
+                        "peak_kind": "nominal: SMs x 128 fp32 lanes x 1.965 GHz",
+                        "frac": ops / (ms * 1e-3) / peak},
+           "launches": 2}
+    del K, q, cand, errors, best
+    return out
+
+
 def run_cpu_baseline(wl: workloads.Workload, target_s: float):
     """The oracle, as it stands (single thread), on a bounded sample of the
     workload: consecutive chunks of keys of one KV head (drawn by the workload's
@@ -461,6 +518,7 @@ def main():
     e2e = run_e2e(wl, path, device, args.e2e_steps, world)
     decode_step = run_decode_step(path, 200)
     attention = run_attention(path, 100)
+    sign_select = run_sign_select(device, 5)
     clocks.stop()
 
     if rank != 0:
@@ -510,6 +568,7 @@ def main():
         "e2e": e2e,
         "decode_step": decode_step,
         "attention": attention,
+        "sign_select": sign_select,
         "cpu_baseline": cpu_baseline,
     }
     print(json.dumps(line), flush=True)

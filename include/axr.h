@@ -189,6 +189,41 @@ int axr_attention_static(const void *q, int qdtype, const uint8_t *idx, const fl
                          float *scores, float *out, axr_stream stream);
 
 /*
+ * Sign-pattern choice (AXELRAM, arXiv 2604.02638, abstract: the sign pattern is
+ * chosen once, without gradients, among candidates (200) on a few calibration
+ * samples (8); some patterns cause large errors on heads whose key norms stand
+ * out).  The pages rank candidates by perplexity, which needs a model; this call
+ * ranks them by the error of the attention logits that the quantized cache
+ * gives.  For candidate c and KV head h,
+ *   errors[c*heads + h] = mean over samples s, query heads g < group and keys t
+ *                         of (score_c - q.k / sqrt(d))^2,
+ * with score_c the score that axr_quantize_keys + axr_scores would give with
+ * signs = candidate c, q = q[s, h*group + g] and k = K[s, h, t] (fp32 arithmetic,
+ * accumulated in fp64 in a fixed order: the result is deterministic).  *best
+ * (if best is not NULL) receives the index of the candidate whose worst head
+ * has the smallest error, the lowest index among equal values (-1 only if every
+ * candidate has a NaN error, which only non-finite inputs give).
+ *
+ *   K           device, (samples, heads, n, d) row-major keys of kdtype, 16-byte
+ *               aligned: the calibration keys of one layer, sample by sample;
+ *   q           device, (samples, heads*group, d) queries of qdtype (element
+ *               aligned); query head h*group + g of sample s reads KV head h;
+ *   candidates  device int8 (n_candidates, d): candidate sign patterns, a
+ *               negative entry is -1, any other +1;
+ *   errors      device float (n_candidates, heads), written;
+ *   best        device int32, one element, written; or NULL.
+ *
+ * The caller owns every buffer; the call allocates nothing and enqueues two
+ * kernels on `stream` (one if best is NULL).  AXR_EINVAL for NULL or misaligned
+ * pointers, n < 1, samples, heads, group or n_candidates < 1, or more than
+ * 2^31 - 1 (candidate, head) pairs; AXR_EUNSUPPORTED for d or b outside the
+ * write path's range or group above 8.
+ */
+int axr_select_signs(const void *K, int kdtype, const void *q, int qdtype, int64_t n, int samples, int heads,
+                     int group, int d, int b, const int8_t *candidates, int n_candidates, float *errors,
+                     int32_t *best, axr_stream stream);
+
+/*
  * Device-side status of the tensor-core kernels (no counterpart in the method;
  * a diagnostic).  Every wait inside those kernels is bounded; a wait that runs
  * out records a bit here instead of hanging: 1 = a tile load never arrived,

@@ -15,6 +15,7 @@ from .axr import (  # noqa: F401
     axr_make_codebook,
     axr_quantize_keys,
     axr_scores,
+    axr_select_signs,
     library,
     packed_row_bytes,
 )
@@ -29,6 +30,7 @@ __all__ = [
     "axr_make_codebook",
     "axr_quantize_keys",
     "axr_scores",
+    "axr_select_signs",
     "library",
     "packed_row_bytes",
 ]

@@ -31,6 +31,7 @@ SIGNATURES = {
     "axr_attention_workspace_bytes": (_I32, [_I64, _I32, _I32, _I32, _P]),
     "axr_attention": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _I64, _P, _P]),
     "axr_attention_static": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _P]),
+    "axr_select_signs": (_I32, [_P, _I32, _P, _I32, _I64, _I32, _I32, _I32, _I32, _I32, _P, _I32, _P, _P, _P]),
     "axr_status_string": (ctypes.c_char_p, [_I32]),
     "axr_last_error": (ctypes.c_char_p, []),
     "axr_version": (_I32, []),
@@ -275,6 +276,44 @@ def axr_attention_static(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor
                                         _stream_handle(stream))
     _raise(rc, "axr_attention_static")
     return out, scores
+
+
+def axr_select_signs(K: torch.Tensor, q: torch.Tensor, group: int, b: int, candidates: torch.Tensor,
+                     errors: torch.Tensor | None = None, best: torch.Tensor | None = None,
+                     stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Sign-pattern choice on calibration keys K (samples, heads, n, d) and
+    queries q (samples, heads*group, d) among candidates (C, d) int8: returns
+    (errors (C, heads) fp32, the logit error of each candidate per KV head;
+    best, a one-element int32 tensor holding the chosen candidate's index)."""
+    for t, name in ((K, "K"), (q, "q"), (candidates, "candidates")):
+        _require_cuda(t, name)
+    if K.dtype not in _DTYPE_CODE or q.dtype not in _DTYPE_CODE:
+        raise ValueError("K and q must be float32, float16 or bfloat16")
+    if candidates.dtype != torch.int8 or candidates.dim() != 2:
+        raise ValueError("candidates must be a (C, d) int8 tensor")
+    if K.dim() != 4:
+        raise ValueError("K must be (samples, heads, n, d)")
+    samples, heads, n, d = K.shape
+    if tuple(q.shape) != (samples, heads * group, d):
+        raise ValueError(f"q must be ({samples}, {heads * group}, {d})")
+    C = candidates.shape[0]
+    if candidates.shape[1] != d:
+        raise ValueError(f"candidates must have {d} columns")
+    if not (K.is_contiguous() and q.is_contiguous() and candidates.is_contiguous()):
+        raise ValueError("K, q and candidates must be contiguous")
+    if errors is None:
+        errors = torch.empty((C, heads), dtype=torch.float32, device=K.device)
+    if best is None:
+        best = torch.empty(1, dtype=torch.int32, device=K.device)
+    for t, name in ((errors, "errors"), (best, "best")):
+        _require_cuda(t, name)
+    if errors.dtype != torch.float32 or errors.numel() < C * heads or best.dtype != torch.int32:
+        raise ValueError("errors must be float32 with C*heads elements, best int32")
+    rc = library().axr_select_signs(K.data_ptr(), _DTYPE_CODE[K.dtype], q.data_ptr(), _DTYPE_CODE[q.dtype], n,
+                                    samples, heads, group, d, b, candidates.data_ptr(), C, errors.data_ptr(),
+                                    best.data_ptr(), _stream_handle(stream))
+    _raise(rc, "axr_select_signs")
+    return errors, best
 
 
 def axr_device_status(clear: bool = True) -> int:

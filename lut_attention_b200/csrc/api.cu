@@ -303,6 +303,36 @@ extern "C" int axr_attention_static(const void *q, int qdtype, const uint8_t *id
     return ok();
 }
 
+extern "C" int axr_select_signs(const void *K, int kdtype, const void *q, int qdtype, int64_t n, int samples,
+                                int heads, int group, int d, int b, const int8_t *candidates, int n_candidates,
+                                float *errors, int32_t *best, axr_stream stream)
+{
+    int rc = check_shape(d, b);
+    if (rc != AXR_OK) return rc;
+    if (elem_size(kdtype) == 0) return fail(AXR_EINVAL, "kdtype=%d is not an axr_dtype", kdtype);
+    if (elem_size(qdtype) == 0) return fail(AXR_EINVAL, "qdtype=%d is not an axr_dtype", qdtype);
+    if (n < 1) return fail(AXR_EINVAL, "n=%lld: the choice needs at least one calibration key", (long long)n);
+    if (samples < 1) return fail(AXR_EINVAL, "samples=%d must be >= 1", samples);
+    if (heads < 1) return fail(AXR_EINVAL, "heads=%d must be >= 1", heads);
+    if (group < 1) return fail(AXR_EINVAL, "group=%d must be >= 1", group);
+    if (n_candidates < 1) return fail(AXR_EINVAL, "n_candidates=%d must be >= 1", n_candidates);
+    if (group > kMaxGroup) return fail(AXR_EUNSUPPORTED, "group=%d: at most %d", group, kMaxGroup);
+    if ((int64_t)n_candidates * heads > (int64_t)INT32_MAX)
+        return fail(AXR_EINVAL, "%d candidates x %d heads: at most 2^31-1 pairs", n_candidates, heads);
+    if ((rc = check_device_ptr(K, 16, "K")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(q, (uintptr_t)elem_size(qdtype), "q")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(candidates, 1, "candidates")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(errors, 4, "errors")) != AXR_OK) return rc;
+    if (best && (rc = check_device_ptr(best, 4, "best")) != AXR_OK) return rc;
+
+    SignSelectArgs a{K, kdtype, q, qdtype, n, samples, heads, group, d, b, candidates, n_candidates, errors, best,
+                     Codebook{}};
+    if (!get_codebook(d, b, &a.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
+    const cudaError_t e = launch_sign_select(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "sign selection launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 extern "C" const char *axr_status_string(int status)
 {
     switch (status) {

@@ -115,6 +115,27 @@ cudaError_t launch_attention(const AttentionArgs &a, cudaStream_t stream);
 int64_t static_attention_scratch_bytes();
 cudaError_t static_attention_scratch(void **ptr);
 
+// Sign-pattern choice (sign_select.cu): the calibration logit error of every
+// candidate pattern per KV head, and the candidate with the smallest worst head.
+struct SignSelectArgs {
+    const void *K;             // (samples, heads, n, d), kdtype
+    int kdtype;
+    const void *q;             // (samples, heads*group, d), qdtype
+    int qdtype;
+    int64_t n;
+    int samples;
+    int heads;
+    int group;
+    int d;
+    int b;
+    const int8_t *candidates;  // (candidates_count, d)
+    int candidates_count;
+    float *errors;             // (candidates_count, heads)
+    int *best;                 // one int, or nullptr
+    Codebook cb;
+};
+cudaError_t launch_sign_select(const SignSelectArgs &a, cudaStream_t stream);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

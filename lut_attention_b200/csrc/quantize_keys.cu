@@ -21,6 +21,7 @@
 #include <cuda_fp16.h>
 
 #include "axr_internal.cuh"
+#include "row_load.cuh"
 
 namespace axr {
 namespace {
@@ -38,55 +39,6 @@ struct QParams {
     int64_t out_stride;        // key r goes to row r * out_stride + out_offset
     int64_t out_offset;
     float bnd[kMaxLevels - 1];
-};
-
-// 8 consecutive input elements -> fp32 (streaming loads: each key is read once)
-template <typename T>
-struct Load8;
-
-template <>
-struct Load8<float> {
-    __device__ static void run(const void *base, int64_t elem, float *v)
-    {
-        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(base) + elem);
-        const float4 a = __ldcs(p);
-        const float4 b = __ldcs(p + 1);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    }
-};
-
-template <>
-struct Load8<__nv_bfloat16> {
-    __device__ static void run(const void *base, int64_t elem, float *v)
-    {
-        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(base) + elem);
-        const uint4 w = __ldcs(p);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[2 * i] = __uint_as_float(ws[i] << 16);
-            v[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
-        }
-    }
-};
-
-template <>
-struct Load8<__half> {
-    __device__ static void run(const void *base, int64_t elem, float *v)
-    {
-        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const __half *>(base) + elem);
-        const uint4 w = __ldcs(p);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            __half2 h2;
-            memcpy(&h2, &ws[i], 4);
-            const float2 f = __half22float2(h2);
-            v[2 * i] = f.x;
-            v[2 * i + 1] = f.y;
-        }
-    }
 };
 
 template <int D, int B, typename T>

@@ -125,6 +125,26 @@ def test_attention_workspace_and_argument_errors(axr_lib):
     assert f(p, 2, p, p, p, 2, 10, 1, 1, 128, 4, p, p, p, 1 << 20, p, None) == axr.AXR_EINVAL      # host memory
 
 
+def test_select_signs_argument_errors(axr_lib):
+    f = axr_lib.axr_select_signs
+    host = np.zeros(4096, np.uint8)
+    p = host.ctypes.data
+    # (K, kdt, q, qdt, n, samples, heads, group, d, b, candidates, C, errors, best, stream)
+    assert f(p, 2, p, 2, 0, 8, 8, 4, 128, 4, p, 200, p, p, None) == axr.AXR_EINVAL            # no keys
+    assert f(p, 2, p, 2, 64, 0, 8, 4, 128, 4, p, 200, p, p, None) == axr.AXR_EINVAL           # samples
+    assert f(p, 2, p, 2, 64, 8, 0, 4, 128, 4, p, 200, p, p, None) == axr.AXR_EINVAL           # heads
+    assert f(p, 2, p, 2, 64, 8, 8, 0, 128, 4, p, 200, p, p, None) == axr.AXR_EINVAL           # group
+    assert f(p, 2, p, 2, 64, 8, 8, 4, 128, 4, p, 0, p, p, None) == axr.AXR_EINVAL             # no candidates
+    assert f(p, 2, p, 2, 64, 8, 8, 9, 128, 4, p, 200, p, p, None) == axr.AXR_EUNSUPPORTED     # group > 8
+    assert f(p, 2, p, 2, 64, 8, 8, 4, 100, 4, p, 200, p, p, None) == axr.AXR_EUNSUPPORTED     # d
+    assert f(p, 2, p, 2, 64, 8, 8, 4, 128, 5, p, 200, p, p, None) == axr.AXR_EUNSUPPORTED     # b
+    assert f(p, 2, p, 2, 64, 8, 1 << 20, 4, 128, 4, p, 1 << 12, p, p, None) == axr.AXR_EINVAL  # 2^32 pairs
+    assert f(p, 6, p, 2, 64, 8, 8, 4, 128, 4, p, 200, p, p, None) == axr.AXR_EINVAL           # key dtype
+    assert f(p + 8, 2, p, 2, 64, 8, 8, 4, 128, 4, p, 200, p, p, None) == axr.AXR_EINVAL       # misaligned K
+    assert f(p, 2, p, 2, 64, 8, 8, 4, 128, 4, p, 200, p, p, None) == axr.AXR_EINVAL           # host memory
+    assert f(None, 2, p, 2, 64, 8, 8, 4, 128, 4, p, 200, p, p, None) == axr.AXR_EINVAL        # NULL K
+
+
 def test_binding_refuses_cpu_tensors():
     """No CPU path: the binding raises instead of computing on the host."""
     K = torch.zeros(4, 128)

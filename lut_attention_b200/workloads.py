@@ -34,7 +34,8 @@ Recipes (``LogNormal(m, s)`` means ``exp(m + s * N(0,1))``):
 Queries are N(0,1) in the workload's dtype.  The sign pattern D is a seeded
 +-1 int8 vector drawn on the CPU, one per workload (one per layer); the
 candidates of a sign-pattern search are seeded +-1 rows, the first of them
-that default pattern.
+that default pattern.  A block rotation takes seeded unit quaternions, two per
+4-element block (one for the fast variant).
 """
 from __future__ import annotations
 
@@ -119,6 +120,18 @@ def make_sign_candidates(wl: Workload, count: int) -> torch.Tensor:
     if count:
         c[0] = make_signs(wl)
     return c
+
+
+def make_block_quats(wl: Workload, fast: bool = False) -> torch.Tensor:
+    """Seeded unit quaternions for a block rotation, (d/4, 8) fp32 on the CPU:
+    per 4-element block qL then qR, each (w, x, y, z) uniform on the unit sphere
+    (a normalised N(0, I_4) draw).  fast: qR = (1, 0, 0, 0) on every block."""
+    g = torch.Generator(device="cpu").manual_seed(3_000_017 * wl.seed + wl.d)
+    z = torch.randn((wl.d // 4, 2, 4), generator=g, dtype=torch.float64)
+    z = z / z.norm(dim=2, keepdim=True)
+    if fast:
+        z[:, 1] = torch.tensor([1.0, 0.0, 0.0, 0.0], dtype=torch.float64)
+    return z.reshape(wl.d // 4, 8).to(torch.float32)
 
 
 def make_queries(wl: Workload, device="cpu") -> torch.Tensor:

@@ -1,4 +1,4 @@
-"""CPU oracle for the AXELRAM write path, read path and sign-pattern choice: test infrastructure.
+"""CPU oracle for the AXELRAM write path, read path, sign-pattern choice and block rotation: test infrastructure.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The CUDA library never uses it, and it
@@ -58,6 +58,10 @@ def _load():
             "oracle_quantize": [P, i64, i32, i32, P, P, P, P],
             "oracle_scores": [P, P, P, i64, i32, i32, i32, i32, P, P],
             "oracle_dequant_scores": [P, P, P, i64, i32, i32, i32, i32, P, P],
+            "oracle_block_rotation": [i32, P, P],
+            "oracle_quantize_block": [P, i64, i32, i32, P, P, P, P],
+            "oracle_scores_block": [P, P, P, i64, i32, i32, i32, i32, P, P],
+            "oracle_dequant_scores_block": [P, P, P, i64, i32, i32, i32, i32, P, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -222,6 +226,51 @@ def attention(q, packed, norms, V, group: int, b: int, signs) -> np.ndarray:
     """Decode attention on the quantized keys: softmax of the LUT scores
     (:func:`scores`) times the value rows, (heads*group, d) fp64."""
     return attention_from_scores(scores(q, packed, norms, group, b, signs), V, group)
+
+
+def _quats(quats, d: int) -> np.ndarray:
+    qs = np.ascontiguousarray(np.asarray(quats, dtype=np.float64))
+    if qs.shape != (d // 4, 8):
+        raise ValueError(f"quats must be ({d // 4}, 8): qL then qR of every 4-block")
+    return qs
+
+
+def block_rotation(d: int, quats) -> np.ndarray:
+    """IsoQuant block rotation T (d, d): block m of coordinates 4m..4m+3 read as
+    a quaternion v and mapped to qL v conj(qR), quats[m] = (qL, qR)."""
+    R = np.empty((d, d), dtype=np.float64)
+    _check(_load().oracle_block_rotation(d, _ptr(_quats(quats, d)), _ptr(R)), "block_rotation")
+    return R
+
+
+def quantize_block(K: np.ndarray, b: int, quats, margins: bool = False):
+    """:func:`quantize` with the block rotation in place of H diag(signs)/sqrt(d)."""
+    K = np.ascontiguousarray(K, dtype=np.float64)
+    n, d = K.shape
+    packed = np.empty((n, d * b // 8), dtype=np.uint8)
+    norms = np.empty(n, dtype=np.float32)
+    marg = np.empty((n, d), dtype=np.float64) if margins else None
+    _check(_load().oracle_quantize_block(_ptr(K), n, d, b, _ptr(_quats(quats, d)), _ptr(packed), _ptr(norms),
+                                         _ptr(marg)), "quantize_block")
+    return packed, norms, marg
+
+
+def scores_block(q, packed, norms, group: int, b: int, quats) -> np.ndarray:
+    """:func:`scores` with the queries rotated by the block rotation."""
+    q, packed, norms, heads, n, d = _read_args(q, packed, norms, group, b)
+    out = np.empty((heads * group, n), dtype=np.float64)
+    _check(_load().oracle_scores_block(_ptr(q), _ptr(packed), _ptr(norms), n, heads, group, d, b,
+                                       _ptr(_quats(quats, d)), _ptr(out)), "scores_block")
+    return out
+
+
+def dequant_scores_block(q, packed, norms, group: int, b: int, quats) -> np.ndarray:
+    """:func:`dequant_scores` with the block rotation."""
+    q, packed, norms, heads, n, d = _read_args(q, packed, norms, group, b)
+    out = np.empty((heads * group, n), dtype=np.float64)
+    _check(_load().oracle_dequant_scores_block(_ptr(q), _ptr(packed), _ptr(norms), n, heads, group, d, b,
+                                               _ptr(_quats(quats, d)), _ptr(out)), "dequant_scores_block")
+    return out
 
 
 def sign_errors(K, q, group: int, b: int, candidates) -> np.ndarray:

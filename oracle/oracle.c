@@ -299,6 +299,32 @@ static int nearest_centroid(double u, const float *cent, int L, double *margin)
     return best;
 }
 
+/* quantize-on-write with the rotation R given (the steps of oracle_quantize) */
+static int quantize_with(const double *K, int64_t n, int d, int b, const double *R, uint8_t *packed,
+                         float *norms, double *margins)
+{
+    const int L = 1 << b;
+    const int P = d * b / 8;
+    float cent[256];
+    if (oracle_codebook(d, b, cent, NULL) != ORACLE_OK) return ORACLE_EINVAL;
+    double *u = (double *)malloc(sizeof(double) * (size_t)d);
+    uint8_t *codes = (uint8_t *)malloc((size_t)d);
+    if (!u || !codes) {
+        free(u);
+        free(codes);
+        return ORACLE_EINVAL;
+    }
+    for (int64_t r = 0; r < n; ++r) {
+        rotate_unit_row(R, K + r * d, d, norms + r, u);
+        for (int j = 0; j < d; ++j)
+            codes[j] = (uint8_t)nearest_centroid(u[j], cent, L, margins ? margins + r * d + j : NULL);
+        pack_row(codes, d, b, packed + r * P);
+    }
+    free(u);
+    free(codes);
+    return ORACLE_OK;
+}
+
 /*
  * Quantize-on-write: keys K (n x d, fp64) -> packed indices (n x d*b/8 bytes)
  * and fp32 norms.  margins (n x d, may be NULL) receives, per coordinate, the
@@ -311,29 +337,14 @@ int oracle_quantize(const double *K, int64_t n, int d, int b, const int8_t *sign
 {
     if (!is_pow2(d) || d < 8 || b < 1 || b > 8 || n < 0 || !K || !signs || !packed || !norms)
         return ORACLE_EINVAL;
-    const int L = 1 << b;
-    const int P = d * b / 8;
-    float cent[256];
-    if (oracle_codebook(d, b, cent, NULL) != ORACLE_OK) return ORACLE_EINVAL;
     double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
-    double *u = (double *)malloc(sizeof(double) * (size_t)d);
-    uint8_t *codes = (uint8_t *)malloc((size_t)d);
-    if (!R || !u || !codes || oracle_rotation(d, signs, R) != ORACLE_OK) {
+    if (!R || oracle_rotation(d, signs, R) != ORACLE_OK) {
         free(R);
-        free(u);
-        free(codes);
         return ORACLE_EINVAL;
     }
-    for (int64_t r = 0; r < n; ++r) {
-        rotate_unit_row(R, K + r * d, d, norms + r, u);
-        for (int j = 0; j < d; ++j)
-            codes[j] = (uint8_t)nearest_centroid(u[j], cent, L, margins ? margins + r * d + j : NULL);
-        pack_row(codes, d, b, packed + r * P);
-    }
+    const int rc = quantize_with(K, n, d, b, R, packed, norms, margins);
     free(R);
-    free(u);
-    free(codes);
-    return ORACLE_OK;
+    return rc;
 }
 
 /* ---------------------------------------------------------------------------
@@ -341,29 +352,16 @@ int oracle_quantize(const double *K, int64_t n, int d, int b, const int8_t *sign
  * never transformed back.
  * --------------------------------------------------------------------------- */
 
-/*
- * Scores of every query against every quantized key of its KV head.
- *   q:      (heads*group) x d, fp64; query head h*group + g reads KV head h
- *   packed: heads x n x (d*b/8) bytes;  norms: heads x n (fp32)
- *   scores: (heads*group) x n, fp64
- * For each query: q' = R q once (no inverse transform on the keys), then
- *   score[t] = norms[t] * sum_j q'_j * c[idx_t[j]] / sqrt(d).
- * The 1/sqrt(d) is the attention temperature, separate from the one inside R.
- */
-int oracle_scores(const double *q, const uint8_t *packed, const float *norms, int64_t n,
-                  int heads, int group, int d, int b, const int8_t *signs, double *scores)
+/* scores with the rotation R given (the steps of oracle_scores) */
+static int scores_with(const double *q, const uint8_t *packed, const float *norms, int64_t n, int heads,
+                       int group, int d, int b, const double *R, double *scores)
 {
-    if (!is_pow2(d) || d < 8 || b < 1 || b > 8 || n < 0 || heads < 1 || group < 1 || !q ||
-        !packed || !norms || !signs || !scores)
-        return ORACLE_EINVAL;
     const int P = d * b / 8;
     float cent[256];
     if (oracle_codebook(d, b, cent, NULL) != ORACLE_OK) return ORACLE_EINVAL;
-    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
     double *qr = (double *)malloc(sizeof(double) * (size_t)d);
     uint8_t *codes = (uint8_t *)malloc((size_t)d);
-    if (!R || !qr || !codes || oracle_rotation(d, signs, R) != ORACLE_OK) {
-        free(R);
+    if (!qr || !codes) {
         free(qr);
         free(codes);
         return ORACLE_EINVAL;
@@ -385,32 +383,46 @@ int oracle_scores(const double *q, const uint8_t *packed, const float *norms, in
                 out[t] = (double)norms[(int64_t)h * n + t] * s * inv_sqrt_d;
             }
         }
-    free(R);
     free(qr);
     free(codes);
     return ORACLE_OK;
 }
 
 /*
- * The same scores the long way, for the cross-check that table lookup without an
- * inverse transform equals attention on dequantized keys:
- *   k_hat_t = norms[t] * R^T c[idx_t],   score[t] = q . k_hat_t / sqrt(d).
+ * Scores of every query against every quantized key of its KV head.
+ *   q:      (heads*group) x d, fp64; query head h*group + g reads KV head h
+ *   packed: heads x n x (d*b/8) bytes;  norms: heads x n (fp32)
+ *   scores: (heads*group) x n, fp64
+ * For each query: q' = R q once (no inverse transform on the keys), then
+ *   score[t] = norms[t] * sum_j q'_j * c[idx_t[j]] / sqrt(d).
+ * The 1/sqrt(d) is the attention temperature, separate from the one inside R.
  */
-int oracle_dequant_scores(const double *q, const uint8_t *packed, const float *norms,
-                          int64_t n, int heads, int group, int d, int b,
-                          const int8_t *signs, double *scores)
+int oracle_scores(const double *q, const uint8_t *packed, const float *norms, int64_t n,
+                  int heads, int group, int d, int b, const int8_t *signs, double *scores)
 {
     if (!is_pow2(d) || d < 8 || b < 1 || b > 8 || n < 0 || heads < 1 || group < 1 || !q ||
         !packed || !norms || !signs || !scores)
         return ORACLE_EINVAL;
+    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
+    if (!R || oracle_rotation(d, signs, R) != ORACLE_OK) {
+        free(R);
+        return ORACLE_EINVAL;
+    }
+    const int rc = scores_with(q, packed, norms, n, heads, group, d, b, R, scores);
+    free(R);
+    return rc;
+}
+
+/* dequantized scores with the rotation R given (the steps of oracle_dequant_scores) */
+static int dequant_scores_with(const double *q, const uint8_t *packed, const float *norms, int64_t n,
+                               int heads, int group, int d, int b, const double *R, double *scores)
+{
     const int P = d * b / 8;
     float cent[256];
     if (oracle_codebook(d, b, cent, NULL) != ORACLE_OK) return ORACLE_EINVAL;
-    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
     double *khat = (double *)malloc(sizeof(double) * (size_t)d);
     uint8_t *codes = (uint8_t *)malloc((size_t)d);
-    if (!R || !khat || !codes || oracle_rotation(d, signs, R) != ORACLE_OK) {
-        free(R);
+    if (!khat || !codes) {
         free(khat);
         free(codes);
         return ORACLE_EINVAL;
@@ -432,8 +444,120 @@ int oracle_dequant_scores(const double *q, const uint8_t *packed, const float *n
                 scores[((int64_t)h * group + g) * n + t] = s * inv_sqrt_d;
             }
         }
-    free(R);
     free(khat);
     free(codes);
     return ORACLE_OK;
+}
+
+/*
+ * The same scores the long way, for the cross-check that table lookup without an
+ * inverse transform equals attention on dequantized keys:
+ *   k_hat_t = norms[t] * R^T c[idx_t],   score[t] = q . k_hat_t / sqrt(d).
+ */
+int oracle_dequant_scores(const double *q, const uint8_t *packed, const float *norms,
+                          int64_t n, int heads, int group, int d, int b,
+                          const int8_t *signs, double *scores)
+{
+    if (!is_pow2(d) || d < 8 || b < 1 || b > 8 || n < 0 || heads < 1 || group < 1 || !q ||
+        !packed || !norms || !signs || !scores)
+        return ORACLE_EINVAL;
+    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
+    if (!R || oracle_rotation(d, signs, R) != ORACLE_OK) {
+        free(R);
+        return ORACLE_EINVAL;
+    }
+    const int rc = dequant_scores_with(q, packed, norms, n, heads, group, d, b, R, scores);
+    free(R);
+    return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Block rotation (IsoQuant, arXiv 2603.28430, abstract), an alternative write
+ * transform: the d coordinates split into d/4 blocks of 4, each read as a
+ * quaternion v = v0 + v1 i + v2 j + v3 k, and T(v) = qL v conj(qR) with one
+ * pair of unit quaternions per block (IsoQuant-Full; qR = 1 is IsoQuant-Fast).
+ * The write and read steps are those above with R = T.
+ * --------------------------------------------------------------------------- */
+
+/* Hamilton product out = a b, with i^2 = j^2 = k^2 = ijk = -1 */
+static void quat_mul(const double *a, const double *b, double *out)
+{
+    out[0] = a[0] * b[0] - a[1] * b[1] - a[2] * b[2] - a[3] * b[3];
+    out[1] = a[0] * b[1] + a[1] * b[0] + a[2] * b[3] - a[3] * b[2];
+    out[2] = a[0] * b[2] - a[1] * b[3] + a[2] * b[0] + a[3] * b[1];
+    out[3] = a[0] * b[3] + a[1] * b[2] - a[2] * b[1] + a[3] * b[0];
+}
+
+/*
+ * T as a dense d x d matrix.  quats: (d/4) x 8 doubles, block m's qL then qR
+ * (w, x, y, z each).  Column 4m + c is T applied to the basis quaternion e_c of
+ * block m; every entry outside the diagonal blocks is 0.
+ */
+int oracle_block_rotation(int d, const double *quats, double *R)
+{
+    if (d < 4 || d % 4 || !quats || !R) return ORACLE_EINVAL;
+    for (size_t i = 0; i < (size_t)d * d; ++i) R[i] = 0.0;
+    for (int m = 0; m < d / 4; ++m) {
+        const double *qL = quats + 8 * m, *qR = quats + 8 * m + 4;
+        const double qRc[4] = {qR[0], -qR[1], -qR[2], -qR[3]};
+        for (int c = 0; c < 4; ++c) {
+            double e[4] = {0.0, 0.0, 0.0, 0.0}, w[4], y[4];
+            e[c] = 1.0;
+            quat_mul(qL, e, w);
+            quat_mul(w, qRc, y);
+            for (int r = 0; r < 4; ++r) R[(size_t)(4 * m + r) * d + 4 * m + c] = y[r];
+        }
+    }
+    return ORACLE_OK;
+}
+
+static double *block_matrix(int d, const double *quats)
+{
+    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
+    if (R && oracle_block_rotation(d, quats, R) != ORACLE_OK) {
+        free(R);
+        return NULL;
+    }
+    return R;
+}
+
+/* oracle_quantize with the block rotation in place of H diag(signs) / sqrt(d) */
+int oracle_quantize_block(const double *K, int64_t n, int d, int b, const double *quats,
+                          uint8_t *packed, float *norms, double *margins)
+{
+    if (!is_pow2(d) || d < 8 || b < 1 || b > 8 || n < 0 || !K || !quats || !packed || !norms)
+        return ORACLE_EINVAL;
+    double *R = block_matrix(d, quats);
+    if (!R) return ORACLE_EINVAL;
+    const int rc = quantize_with(K, n, d, b, R, packed, norms, margins);
+    free(R);
+    return rc;
+}
+
+/* oracle_scores with the queries rotated by the block rotation */
+int oracle_scores_block(const double *q, const uint8_t *packed, const float *norms, int64_t n,
+                        int heads, int group, int d, int b, const double *quats, double *scores)
+{
+    if (!is_pow2(d) || d < 8 || b < 1 || b > 8 || n < 0 || heads < 1 || group < 1 || !q ||
+        !packed || !norms || !quats || !scores)
+        return ORACLE_EINVAL;
+    double *R = block_matrix(d, quats);
+    if (!R) return ORACLE_EINVAL;
+    const int rc = scores_with(q, packed, norms, n, heads, group, d, b, R, scores);
+    free(R);
+    return rc;
+}
+
+/* oracle_dequant_scores with the block rotation */
+int oracle_dequant_scores_block(const double *q, const uint8_t *packed, const float *norms, int64_t n,
+                                int heads, int group, int d, int b, const double *quats, double *scores)
+{
+    if (!is_pow2(d) || d < 8 || b < 1 || b > 8 || n < 0 || heads < 1 || group < 1 || !q ||
+        !packed || !norms || !quats || !scores)
+        return ORACLE_EINVAL;
+    double *R = block_matrix(d, quats);
+    if (!R) return ORACLE_EINVAL;
+    const int rc = dequant_scores_with(q, packed, norms, n, heads, group, d, b, R, scores);
+    free(R);
+    return rc;
 }

@@ -55,6 +55,12 @@ PIN_CALLS = [
     ("test_sign_errors_are_means_over_samples_queries_and_keys", {}),
     ("test_sign_errors_match_lloyd_max_distortion", {"b": 3}),
     ("test_select_signs_worst_head_and_lowest_index", {}),
+    ("test_block_rotation_follows_hamilton_rules", {}),
+    ("test_block_rotation_is_orthonormal_and_block_diagonal", {}),
+    ("test_block_rotation_isoclinic_and_conjugation_closed_forms", {}),
+    ("test_block_quantize_and_scores_brute_force_d8", {"b": 2}),
+    ("test_block_lut_scores_equal_dequantized_dot", {"d": 128, "b": 4}),
+    ("test_block_quantization_mse_matches_lloyd_max_on_isotropic_keys", {"b": 4}),
 ]
 
 # name -> (text in oracle.c, replacement): one plausible mistake each
@@ -90,6 +96,15 @@ MUTANTS = {
     "squared_norm_stored": (
         "const float norm = (float)sqrt(ss);",
         "const float norm = (float)ss;"),
+    "block_right_factor_not_conjugated": (
+        "const double qRc[4] = {qR[0], -qR[1], -qR[2], -qR[3]};",
+        "const double qRc[4] = {qR[0], qR[1], qR[2], qR[3]};"),
+    "hamilton_cross_term_sign": (
+        "out[1] = a[0] * b[1] + a[1] * b[0] + a[2] * b[3] - a[3] * b[2];",
+        "out[1] = a[0] * b[1] + a[1] * b[0] - a[2] * b[3] + a[3] * b[2];"),
+    "block_matrix_transposed": (
+        "for (int r = 0; r < 4; ++r) R[(size_t)(4 * m + r) * d + 4 * m + c] = y[r];",
+        "for (int r = 0; r < 4; ++r) R[(size_t)(4 * m + c) * d + 4 * m + r] = y[r];"),
     "boundary_at_lower_centroid": (
         "boundaries[i] = (float)(0.5 * ((double)centroids[i] + (double)centroids[i + 1]));",
         "boundaries[i] = centroids[i];"),

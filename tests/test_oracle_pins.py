@@ -572,3 +572,140 @@ def test_select_signs_worst_head_and_lowest_index():
     Ed = oracle.sign_errors(K, q, group, 2, dup)
     assert np.array_equal(Ed[1], Ed[2]) and np.array_equal(Ed[1], Ed[3])
     assert oracle.select_signs(Ed) != 2 and oracle.select_signs(Ed) != 3
+
+
+# ------------------------------------------------------------ block rotation --
+# IsoQuant abstract: each 4-element block is a quaternion v, rotated to
+# qL v conj(qR) (IsoQuant-Full; qR = 1 is IsoQuant-Fast).
+
+def _unit_quats(rng, m):
+    z = rng.standard_normal((m, 2, 4))
+    return (z / np.linalg.norm(z, axis=2, keepdims=True)).reshape(m, 8)
+
+
+def _block_of(d, qL, qR):
+    return oracle.block_rotation(d, np.concatenate([qL, qR])[None].repeat(d // 4, axis=0))[:4, :4]
+
+
+def test_block_rotation_follows_hamilton_rules():
+    """i, j, k multiply as i^2 = j^2 = k^2 = ijk = -1: left multiplication by i
+    sends (1, i, j, k) to (i, -1, k, -j), and so on; right multiplication by
+    conj(i) = -i sends them to (-i, 1, k, -j)."""
+    one, i, j, k = np.eye(4)
+    # columns = images of 1, i, j, k
+    assert np.array_equal(_block_of(4, i, one), np.array([i, -one, k, -j]).T)
+    assert np.array_equal(_block_of(4, j, one), np.array([j, -k, -one, i]).T)
+    assert np.array_equal(_block_of(4, k, one), np.array([k, j, -i, -one]).T)
+    assert np.array_equal(_block_of(4, one, i), np.array([-i, one, k, -j]).T)
+    assert np.array_equal(_block_of(4, one, one), np.eye(4))
+
+
+def test_block_rotation_is_orthonormal_and_block_diagonal():
+    rng = np.random.default_rng(90)
+    for d in (8, 32, 128, 512):
+        quats = _unit_quats(rng, d // 4)
+        R = oracle.block_rotation(d, quats)
+        np.testing.assert_allclose(R @ R.T, np.eye(d), rtol=0, atol=1e-14)
+        mask = np.kron(np.eye(d // 4), np.ones((4, 4)))
+        assert np.all(R[mask == 0] == 0)
+
+
+def test_block_rotation_isoclinic_and_conjugation_closed_forms():
+    """Fast (qR = 1) turns every vector by the same angle: <v, a v> = a0 |v|^2.
+    Full with qL = qR = a = cos(t/2) + sin(t/2) n fixes the real axis and turns
+    the imaginary part about n by t (Rodrigues' formula)."""
+    rng = np.random.default_rng(91)
+    for _ in range(5):
+        a = rng.standard_normal(4)
+        a /= np.linalg.norm(a)
+        T = _block_of(4, a, np.eye(4)[0])
+        for _ in range(4):
+            v = rng.standard_normal(4)
+            assert abs(v @ T @ v - a[0] * (v @ v)) < 1e-13
+        t = rng.uniform(0, np.pi)
+        nvec = rng.standard_normal(3)
+        nvec /= np.linalg.norm(nvec)
+        a = np.concatenate([[math.cos(t / 2)], math.sin(t / 2) * nvec])
+        T = _block_of(4, a, a)
+        x = rng.standard_normal(3)
+        rod = (x * math.cos(t) + np.cross(nvec, x) * math.sin(t) + nvec * (nvec @ x) * (1 - math.cos(t)))
+        np.testing.assert_allclose(T @ np.concatenate([[2.5], x]), np.concatenate([[2.5], rod]), atol=1e-13)
+
+
+@pytest.mark.parametrize("b", [1, 2, 3])
+def test_block_quantize_and_scores_brute_force_d8(b):
+    """d = 8 (two blocks): T built from the 4 x 4 left and right multiplication
+    matrices, nearest codeword over all centroids, and the scores in loops."""
+    d, n, heads, group = 8, 6, 2, 2
+    rng = np.random.default_rng(100 + b)
+    quats = _unit_quats(rng, 2)
+
+    def left(a):
+        return np.array([[a[0], -a[1], -a[2], -a[3]], [a[1], a[0], -a[3], a[2]],
+                         [a[2], a[3], a[0], -a[1]], [a[3], -a[2], a[1], a[0]]])
+
+    def right(c):     # v -> v c
+        return np.array([[c[0], -c[1], -c[2], -c[3]], [c[1], c[0], c[3], -c[2]],
+                         [c[2], -c[3], c[0], c[1]], [c[3], c[2], -c[1], c[0]]])
+
+    T = np.zeros((d, d))
+    for m in range(2):
+        qL, qR = quats[m, :4], quats[m, 4:]
+        T[4 * m:4 * m + 4, 4 * m:4 * m + 4] = right(qR * np.array([1, -1, -1, -1])) @ left(qL)
+    K = rng.standard_normal((heads * n, d)) * 2.0
+    packed, norms, _ = oracle.quantize_block(K, b, quats)
+    cent, _ = oracle.codebook(d, b)
+    codes = oracle.unpack(packed, d, b)
+    for r in range(heads * n):
+        nk = math.sqrt(sum(x * x for x in K[r]))
+        assert norms[r] == np.float32(nk)
+        u = T @ K[r] / float(np.float32(nk))
+        for j in range(d):
+            best = min(range(len(cent)), key=lambda l: abs(u[j] - float(cent[l])))
+            assert codes[r, j] == best
+    q = rng.standard_normal((heads * group, d))
+    got = oracle.scores_block(q, packed.reshape(heads, n, -1), norms.reshape(heads, n), group, b, quats)
+    for hq in range(heads * group):
+        qr = T @ q[hq]
+        for t in range(n):
+            r = (hq // group) * n + t
+            expect = norms[r] * sum(qr[j] * float(cent[codes[r, j]]) for j in range(d)) / math.sqrt(d)
+            assert abs(got[hq, t] - expect) < 1e-12 * (1 + abs(expect))
+
+
+@pytest.mark.parametrize("d,b", [(128, 4), (256, 2), (512, 3)])
+def test_block_lut_scores_equal_dequantized_dot(d, b):
+    """T is orthonormal, so reading through the once-rotated query equals the dot
+    product with the dequantized, inverse-rotated key."""
+    heads, n, group = 2, 7, 2
+    rng = np.random.default_rng(d + b)
+    quats = _unit_quats(rng, d // 4)
+    K = rng.standard_normal((heads * n, d)) * rng.lognormal(0, 1, (heads * n, 1))
+    packed, norms, _ = oracle.quantize_block(K, b, quats)
+    q = rng.standard_normal((heads * group, d))
+    a = oracle.scores_block(q, packed.reshape(heads, n, -1), norms.reshape(heads, n), group, b, quats)
+    c = oracle.dequant_scores_block(q, packed.reshape(heads, n, -1), norms.reshape(heads, n), group, b, quats)
+    scale = np.linalg.norm(q, axis=1)[:, None] * np.repeat(norms.reshape(heads, n), group, axis=0)
+    assert np.max(np.abs(a - c) / scale) < 1e-12
+
+
+@pytest.mark.parametrize("b", [2, 4])
+def test_block_quantization_mse_matches_lloyd_max_on_isotropic_keys(b):
+    """An orthonormal T keeps isotropic keys isotropic, so the coordinates of the
+    rotated unit keys are ~N(0, 1/d) and quantize with Max's mean squared error
+    D_b per unit variance (within 5%)."""
+    mse = {}
+    with open(os.path.join(GOLDEN, "lloyd_max_classical.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                parts = line.split()
+                mse[int(parts[0])] = float(parts[1])
+    d, n = 128, 2000
+    rng = np.random.default_rng(110 + b)
+    quats = _unit_quats(rng, d // 4)
+    K = rng.standard_normal((n, d))
+    packed, norms, _ = oracle.quantize_block(K, b, quats)
+    cent, _ = oracle.codebook(d, b)
+    U = (oracle.block_rotation(d, quats) @ K.T).T / norms[:, None].astype(np.float64)
+    err = np.mean((cent[oracle.unpack(packed, d, b)].astype(np.float64) - U) ** 2) * d
+    assert abs(err / mse[b] - 1.0) < 0.05, err / mse[b]

@@ -355,6 +355,58 @@ def run_sign_select(device, steps: int) -> dict:
     return out
 
 
+BLOCK_GRID_DIMS = (128, 256, 512)
+BLOCK_GRID_BITS = (2, 3, 4)
+BLOCK_GRID_DTYPES = ("f16", "f32")
+
+
+def run_block_grid(device, steps: int) -> dict:
+    """Quantize-on-write with the IsoQuant block rotation against the sign flip and
+    Walsh-Hadamard transform, on the 18 settings d x b x key dtype of the IsoQuant
+    comparison: 2^28 bytes of keys per setting (larger than L2), rows N(0,1)^d
+    normalised and scaled by U(0.1, 50).  Times each write call with CUDA events
+    (average of `steps` after 3 warm-up calls) and its algorithmic HBM rate."""
+    rows = []
+    peak, _ = measured_peak()
+    for dt in BLOCK_GRID_DTYPES:
+        for d in BLOCK_GRID_DIMS:
+            esize = 2 if dt == "f16" else 4
+            n = (1 << 28) // (d * esize)
+            wl = workloads.WRITE_2E24.with_(d=d, T=n, dtype=dt, seed=40 + d)
+            K = workloads.make_keys(wl, device).reshape(n, d)
+            signs = workloads.make_signs(wl).to(device)
+            quats = workloads.make_block_quats(wl).to(device)
+            for b in BLOCK_GRID_BITS:
+                P = d * b // 8
+                idx = torch.empty((n, P), dtype=torch.uint8, device=device)
+                norms = torch.empty(n, dtype=torch.float32, device=device)
+
+                def time_ms(fn):
+                    for _ in range(3):
+                        fn()
+                    torch.cuda.synchronize()
+                    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    for _ in range(steps):
+                        fn()
+                    e.record()
+                    torch.cuda.synchronize()
+                    return a.elapsed_time(e) / steps
+
+                t_h = time_ms(lambda: axr.axr_quantize_keys(K, b, signs, idx=idx, norms=norms))
+                t_b = time_ms(lambda: axr.axr_quantize_keys_block(K, b, quats, idx=idx, norms=norms))
+                byts = n * (d * esize + P + 4)
+                rows.append({"d": d, "b": b, "dtype": dt, "keys": n, "hadamard_ms": t_h, "block_ms": t_b,
+                             "hadamard_gbs": byts / (t_h * 1e-3) / 1e9, "block_gbs": byts / (t_b * 1e-3) / 1e9,
+                             "block_frac_of_measured": byts / (t_b * 1e-3) / 1e9 / peak,
+                             "block_speedup": t_h / t_b})
+                del idx, norms
+            del K
+    sp = [r["block_speedup"] for r in rows]
+    return {"settings": rows, "mean_block_speedup": sum(sp) / len(sp),
+            "bytes_per_key": "d * key bytes + d*b/8 + 4", "peak_gbs": peak}
+
+
 def run_cpu_baseline(wl: workloads.Workload, target_s: float):
     """The oracle, as it stands (single thread), on a bounded sample of the
     workload: consecutive chunks of keys of one KV head (drawn by the workload's
@@ -519,6 +571,7 @@ def main():
     decode_step = run_decode_step(path, 200)
     attention = run_attention(path, 100)
     sign_select = run_sign_select(device, 5)
+    block_rotation = run_block_grid(device, 10)
     clocks.stop()
 
     if rank != 0:
@@ -569,6 +622,7 @@ def main():
         "decode_step": decode_step,
         "attention": attention,
         "sign_select": sign_select,
+        "block_rotation": block_rotation,
         "cpu_baseline": cpu_baseline,
     }
     print(json.dumps(line), flush=True)

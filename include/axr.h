@@ -189,6 +189,40 @@ int axr_attention_static(const void *q, int qdtype, const uint8_t *idx, const fl
                          float *scores, float *out, axr_stream stream);
 
 /*
+ * Quantize-on-write with a block rotation in place of the sign flip and the
+ * Walsh-Hadamard transform (IsoQuant, arXiv 2603.28430, abstract: the d
+ * coordinates form d/4 blocks of 4, each read as a quaternion v = v0 + v1 i +
+ * v2 j + v3 k and turned into qL v conj(qR); IsoQuant-Full, or IsoQuant-Fast
+ * when every qR is 1).  Then as axr_quantize_keys: the fp32 norm of the key is
+ * stored, the rotated unit key u = T k / |k| is quantized to the same Lloyd-Max
+ * codebook of N(0, 1/d) and bit-packed in the same layout.
+ *
+ *   K      device, (n, d) row-major keys of kdtype, 16-byte aligned;
+ *   quats  device float (d/4, 8), 16-byte aligned: block m's qL then qR, each
+ *          (w, x, y, z), unit quaternions (used as given; the transform is
+ *          orthonormal only if they are unit);
+ *   idx    device uint8 (n, d*b/8), 16-byte aligned, written;
+ *   norms  device float (n), written.
+ *
+ * The caller owns every buffer; one kernel on `stream`, no allocation.  Both
+ * variants cost the same here (each block's two products are composed into one
+ * 4 x 4 matrix).  Errors as axr_quantize_keys; n = 0 is a no-op.  Keys written
+ * this way are read with axr_scores_block and the same quats.
+ */
+int axr_quantize_keys_block(const void *K, int kdtype, int64_t n, int d, int b, const float *quats,
+                            uint8_t *idx, float *norms, axr_stream stream);
+
+/*
+ * Score-on-read for keys written by axr_quantize_keys_block: each query is
+ * rotated once by the same block rotation, q' = T q, and
+ * score[t] = |k_t| * sum_j q'_j c[idx_t[j]] / sqrt(d), with no inverse transform
+ * of the keys.  Arguments, layouts and errors as axr_scores, with quats (as in
+ * axr_quantize_keys_block) in place of signs.
+ */
+int axr_scores_block(const void *q, int qdtype, const uint8_t *idx, const float *norms, int64_t n, int heads,
+                     int group, int d, int b, const float *quats, float *scores, axr_stream stream);
+
+/*
  * Sign-pattern choice (AXELRAM, arXiv 2604.02638, abstract: the sign pattern is
  * chosen once, without gradients, among candidates (200) on a few calibration
  * samples (8); some patterns cause large errors on heads whose key norms stand

@@ -14,7 +14,9 @@ from .axr import (  # noqa: F401
     axr_device_status,
     axr_make_codebook,
     axr_quantize_keys,
+    axr_quantize_keys_block,
     axr_scores,
+    axr_scores_block,
     axr_select_signs,
     library,
     packed_row_bytes,
@@ -29,7 +31,9 @@ __all__ = [
     "axr_device_status",
     "axr_make_codebook",
     "axr_quantize_keys",
+    "axr_quantize_keys_block",
     "axr_scores",
+    "axr_scores_block",
     "axr_select_signs",
     "library",
     "packed_row_bytes",

@@ -31,6 +31,8 @@ SIGNATURES = {
     "axr_attention_workspace_bytes": (_I32, [_I64, _I32, _I32, _I32, _P]),
     "axr_attention": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _I64, _P, _P]),
     "axr_attention_static": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _P]),
+    "axr_quantize_keys_block": (_I32, [_P, _I32, _I64, _I32, _I32, _P, _P, _P, _P]),
+    "axr_scores_block": (_I32, [_P, _I32, _P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
     "axr_select_signs": (_I32, [_P, _I32, _P, _I32, _I64, _I32, _I32, _I32, _I32, _I32, _P, _I32, _P, _P, _P]),
     "axr_status_string": (ctypes.c_char_p, [_I32]),
     "axr_last_error": (ctypes.c_char_p, []),
@@ -157,6 +159,69 @@ def axr_scores(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, group: i
                               heads, group, d, b, signs.data_ptr(), scores.data_ptr(),
                               _stream_handle(stream))
     _raise(rc, "axr_scores")
+    return scores
+
+
+def _check_quats(quats: torch.Tensor, d: int) -> None:
+    _require_cuda(quats, "quats")
+    if quats.dtype != torch.float32 or tuple(quats.shape) != (d // 4, 8) or not quats.is_contiguous():
+        raise ValueError(f"quats must be a contiguous ({d // 4}, 8) float32 tensor: qL then qR per 4-block")
+
+
+def axr_quantize_keys_block(K: torch.Tensor, b: int, quats: torch.Tensor, idx: torch.Tensor | None = None,
+                            norms: torch.Tensor | None = None, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Quantize-on-write of keys K (..., d) with the IsoQuant block rotation given
+    by quats (d/4, 8) -> (idx (..., d*b/8) uint8, norms (...) fp32)."""
+    _require_cuda(K, "K")
+    if K.dtype not in _DTYPE_CODE:
+        raise ValueError(f"K dtype {K.dtype} not supported")
+    d = K.shape[-1]
+    _check_quats(quats, d)
+    lead = K.shape[:-1]
+    n = K.numel() // d if d else 0
+    P = packed_row_bytes(d, b)
+    if idx is None:
+        idx = torch.empty(lead + (P,), dtype=torch.uint8, device=K.device)
+    if norms is None:
+        norms = torch.empty(lead, dtype=torch.float32, device=K.device)
+    _require_cuda(idx, "idx")
+    _require_cuda(norms, "norms")
+    if idx.numel() < n * P or norms.numel() < n:
+        raise ValueError("idx/norms too small")
+    rc = library().axr_quantize_keys_block(K.data_ptr(), _DTYPE_CODE[K.dtype], n, d, b, quats.data_ptr(),
+                                           idx.data_ptr(), norms.data_ptr(), _stream_handle(stream))
+    _raise(rc, "axr_quantize_keys_block")
+    return idx, norms
+
+
+def axr_scores_block(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, group: int, b: int,
+                     quats: torch.Tensor, scores: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """LUT scores (heads*group, n) fp32 of queries q (heads*group, d) against keys
+    written by :func:`axr_quantize_keys_block` with the same quats."""
+    for t, name in ((q, "q"), (idx, "idx"), (norms, "norms")):
+        _require_cuda(t, name)
+    if q.dtype not in _DTYPE_CODE:
+        raise ValueError(f"q dtype {q.dtype} not supported")
+    if idx.dtype != torch.uint8 or norms.dtype != torch.float32:
+        raise ValueError("idx must be uint8, norms float32")
+    hg, d = q.shape
+    _check_quats(quats, d)
+    if group < 1 or hg % group:
+        raise ValueError("q must have heads*group rows")
+    heads = hg // group
+    if idx.dim() != 3 or idx.shape[0] != heads or idx.shape[2] != packed_row_bytes(d, b):
+        raise ValueError(f"idx must be (heads={heads}, n, {packed_row_bytes(d, b)})")
+    n = idx.shape[1]
+    if tuple(norms.shape) != (heads, n):
+        raise ValueError(f"norms must be ({heads}, {n})")
+    if scores is None:
+        scores = torch.empty((hg, n), dtype=torch.float32, device=q.device)
+    _require_cuda(scores, "scores")
+    if scores.numel() < hg * n or scores.dtype != torch.float32:
+        raise ValueError("scores must be float32 with (heads*group)*n elements")
+    rc = library().axr_scores_block(q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), n,
+                                    heads, group, d, b, quats.data_ptr(), scores.data_ptr(), _stream_handle(stream))
+    _raise(rc, "axr_scores_block")
     return scores
 
 

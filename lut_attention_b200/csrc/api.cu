@@ -303,6 +303,54 @@ extern "C" int axr_attention_static(const void *q, int qdtype, const uint8_t *id
     return ok();
 }
 
+extern "C" int axr_quantize_keys_block(const void *K, int kdtype, int64_t n, int d, int b, const float *quats,
+                                       uint8_t *idx, float *norms, axr_stream stream)
+{
+    int rc = check_shape(d, b);
+    if (rc != AXR_OK) return rc;
+    if (elem_size(kdtype) == 0) return fail(AXR_EINVAL, "kdtype=%d is not an axr_dtype", kdtype);
+    if (n < 0) return fail(AXR_EINVAL, "n=%lld is negative", (long long)n);
+    if (n == 0) return ok();
+    if ((rc = check_device_ptr(K, 16, "K")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(quats, 16, "quats")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(idx, 16, "idx")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(norms, 4, "norms")) != AXR_OK) return rc;
+    QuantizeArgs a{K, kdtype, n, d, b, nullptr, idx, norms, Codebook{}};
+    a.quats = quats;
+    if (!get_codebook(d, b, &a.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
+    const cudaError_t e = launch_quantize_keys_block(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "block-rotation quantize launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+extern "C" int axr_scores_block(const void *q, int qdtype, const uint8_t *idx, const float *norms, int64_t n,
+                                int heads, int group, int d, int b, const float *quats, float *scores,
+                                axr_stream stream)
+{
+    int rc = check_shape(d, b);
+    if (rc != AXR_OK) return rc;
+    if (elem_size(qdtype) == 0) return fail(AXR_EINVAL, "qdtype=%d is not an axr_dtype", qdtype);
+    if (n < 0) return fail(AXR_EINVAL, "n=%lld is negative", (long long)n);
+    if (heads < 1) return fail(AXR_EINVAL, "heads=%d must be >= 1", heads);
+    if (group < 1) return fail(AXR_EINVAL, "group=%d must be >= 1", group);
+    if (group > kMaxGroup) return fail(AXR_EUNSUPPORTED, "group=%d: at most %d", group, kMaxGroup);
+    if (n > (int64_t)INT32_MAX) return fail(AXR_EUNSUPPORTED, "n=%lld: at most 2^31-1 keys per head", (long long)n);
+    if (n == 0) return ok();
+    if ((rc = check_device_ptr(q, 16, "q")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(idx, 16, "idx")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(norms, 4, "norms")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(quats, 16, "quats")) != AXR_OK) return rc;
+    if ((rc = check_device_ptr(scores, 4, "scores")) != AXR_OK) return rc;
+    ScoresArgs a{q, qdtype, idx, norms, n, heads, group, d, b, nullptr, scores, Codebook{}};
+    a.head_stride = n;
+    a.quats = quats;
+    if (!get_codebook(d, b, &a.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = scores_tc_supported(a) ? launch_scores_tc(a, st) : launch_scores(a, st);
+    if (e != cudaSuccess) return fail(AXR_ECUDA, "block-rotation scores launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 extern "C" int axr_select_signs(const void *K, int kdtype, const void *q, int qdtype, int64_t n, int samples,
                                 int heads, int group, int d, int b, const int8_t *candidates, int n_candidates,
                                 float *errors, int32_t *best, axr_stream stream)

@@ -53,6 +53,9 @@ struct QuantizeArgs {
     // key per head is appended)
     int64_t out_stride = 1;
     int64_t out_offset = 0;
+    // IsoQuant block rotation in place of diag(signs) and H: (d/4) x 8 floats,
+    // qL then qR of every 4-element block (quantize_keys_block.cu)
+    const float *quats = nullptr;
 };
 
 struct ScoresArgs {
@@ -77,11 +80,15 @@ struct ScoresArgs {
     int64_t append_pos = -1;
     uint8_t *idx_out = nullptr;
     float *norms_out = nullptr;
+    // queries rotated by the IsoQuant block rotation instead of H diag(signs)
+    const float *quats = nullptr;
 };
 
 // Kernel launchers (quantize_keys.cu, scores.cu).  They return cudaSuccess or
 // the launch error; arguments are already validated.
 cudaError_t launch_quantize_keys(const QuantizeArgs &a, cudaStream_t stream);
+// Write path with the block rotation (quantize_keys_block.cu): every d, dense output.
+cudaError_t launch_quantize_keys_block(const QuantizeArgs &a, cudaStream_t stream);
 
 // Tensor-core write path (quantize_keys_tc.cu): d = 128, bf16/fp16 keys.
 bool quantize_tc_supported(const QuantizeArgs &a);

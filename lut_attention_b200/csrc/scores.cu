@@ -4,7 +4,9 @@
 // One CTA serves one KV head h (batch folded in) and a tile of its keys.
 //   prologue: q''_g = H diag(signs) q_g / D for the G query heads of h
 //             (the orthonormal 1/sqrt(D) of the rotation times the attention
-//             temperature 1/sqrt(D); D is a power of two, so 1/D is exact);
+//             temperature 1/sqrt(D); D is a power of two, so 1/D is exact),
+//             or q''_g = T q_g / sqrt(D) with the IsoQuant block rotation T
+//             (arXiv 2603.28430, abstract) when the keys were written with it;
 //   per key t: s_g[t] = norms[t] * sum_j q''_g[j] * c[idx_t[j]]
 // The index stream of a key is read once and serves all G queries (GQA).
 //
@@ -18,6 +20,7 @@
 #include <cuda_fp16.h>
 
 #include "axr_internal.cuh"
+#include "quat.cuh"
 
 namespace axr {
 namespace {
@@ -36,6 +39,7 @@ struct SParams {
     int64_t head_stride;       // rows between KV heads in idx and norms
     int group;
     const int8_t *signs;
+    const float *quats;        // block rotation of the queries instead of H diag(signs), or null
     float *scores;
     float cent[kMaxLevels];
 };
@@ -133,22 +137,37 @@ __global__ void __launch_bounds__(kThreads) scores_kernel(SParams p)
         if (g < p.group) {
             const int64_t qrow = static_cast<int64_t>(h) * p.group + g;
             for (int j = lane; j < D; j += 32)
-                sq[j] = (p.signs[j] < 0 ? -1.0f : 1.0f) * load_q(p.q, p.qdtype, qrow * D + j);
+                sq[j] = (p.quats || p.signs[j] >= 0 ? 1.0f : -1.0f) * load_q(p.q, p.qdtype, qrow * D + j);
         } else {
             for (int j = lane; j < D; j += 32) sq[j] = 0.0f;
         }
         __syncwarp();
-        for (int hh = 1; hh < D; hh <<= 1) {
-            for (int pi = lane; pi < D / 2; pi += 32) {
-                const int i = (pi / hh) * 2 * hh + (pi % hh);
-                const float a = sq[i], b = sq[i + hh];
-                sq[i] = a + b;
-                sq[i + hh] = a - b;
+        if (p.quats) {
+            // q'' = T q / sqrt(D): the block rotation is orthonormal, 1/sqrt(D) is the temperature
+            const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+            for (int m = lane; m < D / 4; m += 32) {
+                Quat qL, qRc;
+                block_quats(p.quats, m, qL, qRc);
+                const Quat y = block_rotate(qL, qRc, {sq[4 * m], sq[4 * m + 1], sq[4 * m + 2], sq[4 * m + 3]});
+                sq[4 * m] = y.w * inv_sqrt_d;
+                sq[4 * m + 1] = y.x * inv_sqrt_d;
+                sq[4 * m + 2] = y.y * inv_sqrt_d;
+                sq[4 * m + 3] = y.z * inv_sqrt_d;
             }
             __syncwarp();
+        } else {
+            for (int hh = 1; hh < D; hh <<= 1) {
+                for (int pi = lane; pi < D / 2; pi += 32) {
+                    const int i = (pi / hh) * 2 * hh + (pi % hh);
+                    const float a = sq[i], b = sq[i + hh];
+                    sq[i] = a + b;
+                    sq[i + hh] = a - b;
+                }
+                __syncwarp();
+            }
+            for (int j = lane; j < D; j += 32) sq[j] *= 1.0f / static_cast<float>(D);
+            __syncwarp();
         }
-        for (int j = lane; j < D; j += 32) sq[j] *= 1.0f / static_cast<float>(D);
-        __syncwarp();
     }
     __syncthreads();
 
@@ -206,6 +225,7 @@ cudaError_t launch_dbg(const ScoresArgs &a, cudaStream_t stream)
     p.head_stride = a.head_stride;
     p.group = a.group;
     p.signs = a.signs;
+    p.quats = a.quats;
     p.scores = a.scores;
     for (int i = 0; i < kMaxLevels; ++i) p.cent[i] = a.cb.centroids[i];
     const dim3 grid(static_cast<unsigned>((a.n + kTile - 1) / kTile), static_cast<unsigned>(a.heads));

@@ -52,6 +52,7 @@
 #include <cuda_runtime.h>
 
 #include "axr_internal.cuh"
+#include "quat.cuh"
 #include "sm100.cuh"
 
 namespace axr {
@@ -60,6 +61,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
+constexpr float kInvSqrtD = 0.08838834764831845f;   // 1 / sqrt(128), the attention temperature
 constexpr int kTileRows = 128;
 constexpr int kStages = 6;            // a multiple of every stream count: a stream owns whole stages
 constexpr int kGroupThreads = 128;    // worker threads of one stream (one per key of a tile)
@@ -111,6 +113,7 @@ struct TcParams {
     int qdtype;
     int nshift;                // norms[0] is element nshift of nmap
     const int8_t *signs;
+    const float *quats;              // block rotation of the queries instead of H diag(signs), or null
     float *scores;
     int n;                     // keys per head
     int head_stride;           // rows between KV heads in the packed rows and norms (>= n)
@@ -181,28 +184,43 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
     using LK = Lookup<B>;
     const int tid = threadIdx.x & (kGroupThreads - 1);
     float(*q)[kD] = reinterpret_cast<float(*)[kD]>(S.q + g * NQ * kD);
-    const float sg = p.signs[tid] < 0 ? -1.0f : 1.0f;
+    const float sg = (p.quats || p.signs[tid] >= 0) ? 1.0f : -1.0f;
 #pragma unroll
     for (int qi = 0; qi < NQ; ++qi)
         q[qi][tid] = (qi < p.group)
                          ? sg * load_q(p.q, p.qdtype, (static_cast<int64_t>(h) * p.group + qi) * kD + tid)
                          : 0.0f;
     if (!stream_sync(S, g, phase)) return false;
-    for (int hh = 1; hh < kD; hh <<= 1) {
-        for (int t = tid; t < NQ * (kD / 2); t += kGroupThreads) {
-            const int qi = t / (kD / 2), pi = t % (kD / 2);
-            const int i = (pi / hh) * 2 * hh + (pi % hh);
-            const float x = q[qi][i], y = q[qi][i + hh];
-            q[qi][i] = x + y;
-            q[qi][i + hh] = x - y;
-        }
-        if (!stream_sync(S, g, phase)) return false;
-    }
-    // q'' = H diag(s) q / d  (rotation 1/sqrt(d) times temperature 1/sqrt(d))
     float qq[NQ];
+    if (p.quats) {
+        // q'' = T q / sqrt(d): the IsoQuant block rotation T (orthonormal) times the
+        // temperature; this thread's coordinate from its 4-element block
+        Quat qL, qRc;
+        block_quats(p.quats, tid >> 2, qL, qRc);
+        const int b0 = tid & ~3;
+#pragma unroll
+        for (int qi = 0; qi < NQ; ++qi) {
+            const Quat y = block_rotate(qL, qRc, {q[qi][b0], q[qi][b0 + 1], q[qi][b0 + 2], q[qi][b0 + 3]});
+            const float c = (tid & 3) == 0 ? y.w : (tid & 3) == 1 ? y.x : (tid & 3) == 2 ? y.y : y.z;
+            qq[qi] = c * kInvSqrtD;
+        }
+    } else {
+        for (int hh = 1; hh < kD; hh <<= 1) {
+            for (int t = tid; t < NQ * (kD / 2); t += kGroupThreads) {
+                const int qi = t / (kD / 2), pi = t % (kD / 2);
+                const int i = (pi / hh) * 2 * hh + (pi % hh);
+                const float x = q[qi][i], y = q[qi][i + hh];
+                q[qi][i] = x + y;
+                q[qi][i + hh] = x - y;
+            }
+            if (!stream_sync(S, g, phase)) return false;
+        }
+        // q'' = H diag(s) q / d  (rotation 1/sqrt(d) times temperature 1/sqrt(d))
+#pragma unroll
+        for (int qi = 0; qi < NQ; ++qi) qq[qi] = q[qi][tid] * (1.0f / kD);
+    }
 #pragma unroll
     for (int qi = 0; qi < NQ; ++qi) {
-        qq[qi] = q[qi][tid] * (1.0f / kD);
         float m = fabsf(qq[qi]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -747,6 +765,7 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     p.q = a.q;
     p.qdtype = a.qdtype;
     p.signs = a.signs;
+    p.quats = a.quats;
     p.scores = a.scores;
     p.n = static_cast<int>(a.n);
     p.head_stride = static_cast<int>(a.head_stride);

@@ -48,13 +48,16 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
 
 
 def check_quantize(K_rows: torch.Tensor, idx_rows: torch.Tensor, norms_rows: torch.Tensor,
-                   b: int, signs: torch.Tensor) -> QuantizeReport:
+                   b: int, signs: torch.Tensor | None, quats: torch.Tensor | None = None) -> QuantizeReport:
     """K_rows (m, d) inputs on any device, idx_rows / norms_rows the GPU outputs for
-    those rows; compares with the oracle run on the same inputs."""
+    those rows; compares with the oracle run on the same inputs (the block rotation
+    of `quats` instead of the sign flip and Walsh-Hadamard transform if given)."""
     d = K_rows.shape[-1]
     Kh = to_f64(K_rows.reshape(-1, d))
-    s = signs.cpu().numpy()
-    o_idx, o_norms, marg = oracle.quantize(Kh, b, s, margins=True)
+    if quats is not None:
+        o_idx, o_norms, marg = oracle.quantize_block(Kh, b, to_f64(quats), margins=True)
+    else:
+        o_idx, o_norms, marg = oracle.quantize(Kh, b, signs.cpu().numpy(), margins=True)
     g_idx = idx_rows.reshape(len(Kh), -1).cpu().numpy()
     g_norms = norms_rows.reshape(-1).cpu().numpy().astype(np.float64)
     oc = oracle.unpack(o_idx, d, b)
@@ -76,12 +79,16 @@ def check_quantize(K_rows: torch.Tensor, idx_rows: torch.Tensor, norms_rows: tor
 
 
 def check_scores(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, scores: torch.Tensor,
-                 group: int, b: int, signs: torch.Tensor) -> float:
+                 group: int, b: int, signs: torch.Tensor | None, quats: torch.Tensor | None = None) -> float:
     """Worst |s_gpu - s_oracle| / (||q|| ||k|| / sqrt(d)) over the given keys.
-    idx (heads, m, P) / norms (heads, m) / scores (heads*group, m) on any device."""
+    idx (heads, m, P) / norms (heads, m) / scores (heads*group, m) on any device;
+    queries rotated by the block rotation of `quats` if given."""
     d = q.shape[-1]
     qh = to_f64(q)
-    exp = oracle.scores(qh, idx.cpu().numpy(), norms.cpu().numpy(), group, b, signs.cpu().numpy())
+    if quats is not None:
+        exp = oracle.scores_block(qh, idx.cpu().numpy(), norms.cpu().numpy(), group, b, to_f64(quats))
+    else:
+        exp = oracle.scores(qh, idx.cpu().numpy(), norms.cpu().numpy(), group, b, signs.cpu().numpy())
     got = scores.cpu().numpy().astype(np.float64)
     qn = np.linalg.norm(qh, axis=1)[:, None]
     kn = np.repeat(norms.cpu().numpy().astype(np.float64), group, axis=0)

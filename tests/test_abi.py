@@ -145,6 +145,27 @@ def test_select_signs_argument_errors(axr_lib):
     assert f(None, 2, p, 2, 64, 8, 8, 4, 128, 4, p, 200, p, p, None) == axr.AXR_EINVAL        # NULL K
 
 
+def test_block_rotation_argument_errors(axr_lib):
+    fq = axr_lib.axr_quantize_keys_block
+    fs = axr_lib.axr_scores_block
+    host = np.zeros(4096, np.uint8)
+    p = host.ctypes.data
+    # (K, kdt, n, d, b, quats, idx, norms, stream)
+    assert fq(p, 2, 0, 128, 4, p, p, p, None) == axr.AXR_OK                  # n = 0: no-op
+    assert fq(p, 2, -1, 128, 4, p, p, p, None) == axr.AXR_EINVAL             # n < 0
+    assert fq(p, 2, 10, 96, 4, p, p, p, None) == axr.AXR_EUNSUPPORTED        # d
+    assert fq(p, 2, 10, 128, 0, p, p, p, None) == axr.AXR_EUNSUPPORTED       # b
+    assert fq(p, 4, 10, 128, 4, p, p, p, None) == axr.AXR_EINVAL             # key dtype
+    assert fq(p, 2, 10, 128, 4, None, p, p, None) == axr.AXR_EINVAL          # NULL quats
+    assert fq(p, 2, 10, 128, 4, p, p, p, None) == axr.AXR_EINVAL             # host memory
+    # (q, qdt, idx, norms, n, heads, group, d, b, quats, scores, stream)
+    assert fs(p, 2, p, p, 0, 1, 1, 128, 4, p, p, None) == axr.AXR_OK          # n = 0: no-op
+    assert fs(p, 2, p, p, 10, 0, 1, 128, 4, p, p, None) == axr.AXR_EINVAL     # heads
+    assert fs(p, 2, p, p, 10, 1, 9, 128, 4, p, p, None) == axr.AXR_EUNSUPPORTED   # group > 8
+    assert fs(p, 2, p, p, 10, 1, 1, 128, 4, None, p, None) == axr.AXR_EINVAL  # NULL quats
+    assert fs(p, 2, p, p, 10, 1, 1, 128, 4, p, p, None) == axr.AXR_EINVAL     # host memory
+
+
 def test_binding_refuses_cpu_tensors():
     """No CPU path: the binding raises instead of computing on the host."""
     K = torch.zeros(4, 128)

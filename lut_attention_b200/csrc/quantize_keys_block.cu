@@ -20,6 +20,7 @@
 // bucket of u (the bucket table of the codebook) names the one boundary that can
 // decide it, and u itself is compared with that boundary.  Each thread's codes
 // fill EPT*B/8 whole bytes of the packed row, stored straight from registers.
+#include <cstring>
 #include <type_traits>
 
 #include <cuda_bf16.h>
@@ -27,7 +28,6 @@
 
 #include "axr_internal.cuh"
 #include "quat.cuh"
-#include "row_load.cuh"
 
 namespace axr {
 namespace {
@@ -37,7 +37,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr uint32_t kMagicBits = 0x4B400000u;    // bits of 1.5 * 2^23
 constexpr float kMagic = 12582912.0f;
-constexpr int kBytesInFlight = 2048;            // key bytes a warp loads before computing
+constexpr int kBytesInFlight = 2048;            // key bytes per warp and group of rows (two groups in flight)
 
 // Warp steps per loop iteration: about kBytesInFlight of keys per warp, at most
 // 64 staged values per thread.
@@ -62,6 +62,83 @@ struct BParams {
     float tau[kMaxBuckets];
     int base[kMaxBuckets];
 };
+
+// Code of one rotated unit coordinate u, given the bits of f = round(g) + 1.5 * 2^23
+// for its bucket value g: entry {boundary, code below it} of bucket round(g) sits
+// at bits * 8 + (table - 1.5 * 2^23 * 8), one multiply-add (the bias wraps mod
+// 2^32 by design).  kClamp bounds the bucket to the table instead, for rows whose
+// squared norm is zero, tiny or not finite, where |u| <= 1 can fail.
+// One thread's EPT coordinates of a row as loaded (16-byte words), converted to
+// fp32 only when the row is processed, so the next rows' loads stay in flight.
+template <typename T, int EPT>
+struct RawRow {
+    static constexpr int N = EPT * static_cast<int>(sizeof(T)) / 16;
+    uint4 w[N];
+};
+
+template <typename T, int EPT>
+__device__ __forceinline__ void load_row(const void *K, int64_t elem, bool ok, RawRow<T, EPT> &r)
+{
+    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(K) + elem);
+#pragma unroll
+    for (int i = 0; i < RawRow<T, EPT>::N; ++i) r.w[i] = ok ? __ldcs(src + i) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+template <typename T, int EPT>
+__device__ __forceinline__ void to_f32(const RawRow<T, EPT> &r, float (&v)[EPT])
+{
+#pragma unroll
+    for (int i = 0; i < RawRow<T, EPT>::N; ++i) {
+        const uint32_t ws[4] = {r.w[i].x, r.w[i].y, r.w[i].z, r.w[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if constexpr (std::is_same<T, float>::value) {
+                v[4 * i + k] = __uint_as_float(ws[k]);
+            } else if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+                v[8 * i + 2 * k] = __uint_as_float(ws[k] << 16);
+                v[8 * i + 2 * k + 1] = __uint_as_float(ws[k] & 0xffff0000u);
+            } else {
+                __half2 h2;
+                memcpy(&h2, &ws[k], 4);
+                const float2 f = __half22float2(h2);
+                v[8 * i + 2 * k] = f.x;
+                v[8 * i + 2 * k + 1] = f.y;
+            }
+        }
+    }
+}
+
+template <bool kClamp>
+__device__ __forceinline__ uint32_t code_of(float u, float f, uint32_t tab, uint32_t bias, uint32_t last)
+{
+    uint32_t addr;
+    if constexpr (kClamp) {
+        addr = tab + min(__float_as_uint(f) - kMagicBits, last) * 8u;
+    } else {
+        addr = __float_as_uint(f) * 8u + bias;
+    }
+    float t;
+    uint32_t base;
+    asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(t), "=r"(base) : "r"(addr));
+    return base + (u > t ? 1u : 0u);
+}
+
+template <int B, int EPT, bool kClamp, typename Word>
+__device__ __forceinline__ Word pack_codes(const float (&y)[EPT], float inv, float a, float2 offm2, uint32_t tab,
+                                           uint32_t bias, uint32_t last)
+{
+    const float2 inv2 = make_float2(inv, inv), a2 = make_float2(a, a);
+    Word word = 0;
+#pragma unroll
+    for (int e = 0; e < EPT; e += 2) {
+        const float2 ye = make_float2(y[e], y[e + 1]);
+        const float2 u = __fmul2_rn(ye, inv2);
+        const float2 f = __ffma2_rn(ye, a2, offm2);
+        word |= static_cast<Word>(code_of<kClamp>(u.x, f.x, tab, bias, last)) << (B * e);
+        word |= static_cast<Word>(code_of<kClamp>(u.y, f.y, tab, bias, last)) << (B * (e + 1));
+    }
+    return word;
+}
 
 template <int D, int B, typename T>
 __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const __grid_constant__ BParams p)
@@ -101,35 +178,43 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const 
     }
     const float2 offm2 = make_float2(p.g_off + kMagic, p.g_off + kMagic);
     const uint32_t last = static_cast<uint32_t>(p.nt - 1);
-    // U warp steps per iteration: their loads are issued together, so each warp
-    // keeps U steps' bytes in flight (one step alone leaves HBM latency-bound)
+    const uint32_t tab = static_cast<uint32_t>(__cvta_generic_to_shared(s_tab));
+    const uint32_t bias = tab - kMagicBits * 8u;     // wraps mod 2^32 by design
+    // U warp steps per group: a group's loads are issued together, one group ahead
+    // of the one being processed (one step at a time leaves HBM latency-bound)
     const int64_t nsteps = (p.n + RW - 1) / RW;
     const int64_t ngroups = (nsteps + U - 1) / U;
 
-    for (int64_t grp = static_cast<int64_t>(blockIdx.x) * kWarps + warp; grp < ngroups;
-         grp += static_cast<int64_t>(gridDim.x) * kWarps) {
-        float v[U][EPT];
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarps;
+    RawRow<T, EPT> cur[U], nxt[U];
+    int64_t grp = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    if (grp < ngroups) {
 #pragma unroll
         for (int uu = 0; uu < U; ++uu) {
             const int64_t row = (grp * U + uu) * RW + slot;
+            load_row<T, EPT>(p.K, row * D + t * EPT, row < p.n, cur[uu]);
+        }
+    }
+    for (; grp < ngroups; grp += stride) {
+        // the next group's loads go out before this group is processed
+        const int64_t gn = grp + stride;
+        if (gn < ngroups) {
 #pragma unroll
-            for (int k = 0; k < EPT / 8; ++k) {
-                if (row < p.n) {
-                    Load8<T>::run(p.K, row * D + t * EPT + 8 * k, v[uu] + 8 * k);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[uu][8 * k + e] = 0.0f;
-                }
+            for (int uu = 0; uu < U; ++uu) {
+                const int64_t row = (gn * U + uu) * RW + slot;
+                load_row<T, EPT>(p.K, row * D + t * EPT, row < p.n, nxt[uu]);
             }
         }
 #pragma unroll
         for (int uu = 0; uu < U; ++uu) {
             const int64_t row = (grp * U + uu) * RW + slot;
             const bool valid = row < p.n;
+            float v[EPT];
+            to_f32<T, EPT>(cur[uu], v);
             float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int e = 0; e < EPT; e += 2) {
-                const float2 x = make_float2(v[uu][e], v[uu][e + 1]);
+                const float2 x = make_float2(v[e], v[e + 1]);
                 ss2 = __ffma2_rn(x, x, ss2);
             }
             float ss = ss2.x + ss2.y;
@@ -142,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const 
                 float2 a01 = make_float2(0.0f, 0.0f), a23 = make_float2(0.0f, 0.0f);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const float2 vc = make_float2(v[uu][4 * i + c], v[uu][4 * i + c]);
+                    const float2 vc = make_float2(v[4 * i + c], v[4 * i + c]);
                     a01 = __ffma2_rn(m01[i][c], vc, a01);
                     a23 = __ffma2_rn(m23[i][c], vc, a23);
                 }
@@ -156,20 +241,9 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const 
             // a zero key has u = 0, which the codes map to 2^(B-1) - 1
             const float inv = (norm > 0.0f) ? 1.0f / norm : 0.0f;
             const float a = p.g_scale * inv;
-            const float2 inv2 = make_float2(inv, inv), a2 = make_float2(a, a);
-            Word word = 0;
-#pragma unroll
-            for (int e = 0; e < EPT; e += 2) {
-                const float2 ye = make_float2(y[e], y[e + 1]);
-                const float2 u = __fmul2_rn(ye, inv2);
-                const float2 f = __ffma2_rn(ye, a2, offm2);
-                const float2 e0 = s_tab[min(__float_as_uint(f.x) - kMagicBits, last)];
-                const float2 e1 = s_tab[min(__float_as_uint(f.y) - kMagicBits, last)];
-                const uint32_t c0 = static_cast<uint32_t>(__float_as_int(e0.y)) + (u.x > e0.x ? 1u : 0u);
-                const uint32_t c1 = static_cast<uint32_t>(__float_as_int(e1.y)) + (u.y > e1.x ? 1u : 0u);
-                word |= static_cast<Word>(c0) << (B * e);
-                word |= static_cast<Word>(c1) << (B * (e + 1));
-            }
+            const Word word = (ss >= 1e-36f && ss <= 3.402823466e38f)
+                                  ? pack_codes<B, EPT, false, Word>(y, inv, a, offm2, tab, bias, last)
+                                  : pack_codes<B, EPT, true, Word>(y, inv, a, offm2, tab, bias, last);
             if (valid) {
                 uint8_t *dst = p.idx + row * P + t * TB;
                 if constexpr (TB == 8) {
@@ -186,6 +260,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const 
                 if (t == 0) p.norms[row] = norm;
             }
         }
+#pragma unroll
+        for (int uu = 0; uu < U; ++uu) cur[uu] = nxt[uu];
     }
 }
 

@@ -503,6 +503,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="skip the legs after the step (decode step, attention, sign choice, block-rotation grid)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -568,10 +570,12 @@ def main():
 
     # end to end through the public API with host buffers
     e2e = run_e2e(wl, path, device, args.e2e_steps, world)
-    decode_step = run_decode_step(path, 200)
-    attention = run_attention(path, 100)
-    sign_select = run_sign_select(device, 5)
-    block_rotation = run_block_grid(device, 10)
+    decode_step = attention = sign_select = block_rotation = None
+    if not args.no_legs:
+        decode_step = run_decode_step(path, 200)
+        attention = run_attention(path, 100)
+        sign_select = run_sign_select(device, 5)
+        block_rotation = run_block_grid(device, 10)
     clocks.stop()
 
     if rank != 0:

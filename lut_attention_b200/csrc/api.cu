@@ -189,23 +189,24 @@ extern "C" int axr_append_scores(const void *k_new, int kdtype, const void *q, i
     // every query head against keys 0 .. pos of its KV head
     ScoresArgs sa{q, qdtype, idx, norms, pos + 1, heads, group, d, b, signs, scores, cb};
     sa.head_stride = capacity;
+    ScoresArgs fused = sa;
+    fused.k_new = k_new;
+    fused.kdtype = kdtype;
+    fused.append_pos = pos;
+    fused.idx_out = idx;
+    fused.norms_out = norms;
     cudaError_t e;
-    if (scores_tc_supported(sa)) {
+    if (scores_tc_supported(fused)) {
         // one launch: the tensor-core read kernel quantizes the new key of each
         // head into row h * capacity + pos itself, in the CTA that scores it
-        sa.k_new = k_new;
-        sa.kdtype = kdtype;
-        sa.append_pos = pos;
-        sa.idx_out = idx;
-        sa.norms_out = norms;
-        e = launch_scores_tc(sa, st);
+        e = launch_scores_tc(fused, st);
     } else {
         // two launches: the new key of KV head h goes to cache row h * capacity + pos
         QuantizeArgs qa{k_new, kdtype, heads, d, b, signs, idx, norms, cb};
         qa.out_stride = capacity;
         qa.out_offset = pos;
         e = launch_quantize_keys(qa, st);
-        if (e == cudaSuccess) e = launch_scores(sa, st);
+        if (e == cudaSuccess) e = scores_tc_supported(sa) ? launch_scores_tc(sa, st) : launch_scores(sa, st);
     }
     if (e != cudaSuccess) return fail(AXR_ECUDA, "decode step launch: %s", cudaGetErrorString(e));
     return ok();

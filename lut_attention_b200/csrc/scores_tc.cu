@@ -79,20 +79,30 @@ constexpr int kLutBytes = 256 * 256;          // up to 256 fields x 256 bytes
 constexpr int kInvSlots = 8;          // per-stream ring of query scales, one slot per head
 constexpr int kBBytesMax = 32 * kK;   // one B buffer at most: 8 queries x 4 digit rows x K bytes
 
-// launch shape for NQ query columns per KV head (G <= NQ)
-template <int NQ>
+// launch shape for NQ query columns per KV head (G <= NQ) and head dimension
+// 128 * NH.  A tile of 128 keys is processed as NH subtiles of 128 coordinates
+// (one stage, one A buffer and one K = 256 block of B each) accumulating into one
+// D.  At NH = 1 each stream double-buffers B (the next head's digits are written
+// while the last head's products run); wider heads keep one B buffer per stream
+// (shared memory), and the streams wait for their products before a new head.
+template <int NQ, int NH>
 struct Cfg {
     static constexpr int N = 4 * NQ;                  // B rows = D columns
-    static constexpr int S = (NQ <= 4) ? 3 : 2;       // tile streams
+    static constexpr int S = (NH == 1) ? ((NQ <= 4) ? 3 : 2)
+                           : (NH == 2) ? ((NQ <= 4) ? 3 : 2)
+                                       : ((NQ <= 4) ? 2 : 1);   // tile streams
+    static constexpr int kBBufs = (NH == 1) ? 2 : 1;  // B buffers per stream
     static constexpr int kWorkerWarps = 4 * S;
     static constexpr int kWarpTma = kWorkerWarps;
     static constexpr int kWarpMma0 = kWorkerWarps + 1;
     static constexpr int kThreads = (kWorkerWarps + 1 + S) * 32;
     static constexpr int kDOff = S * 2 * kACols;      // A buffers first, then D buffers
-    static constexpr int kBBytes = N * kK;
+    static constexpr int kSliceB = N * kK;            // B bytes of one subtile's K block
+    static constexpr int kBBytes = kSliceB * NH;      // one B buffer
     static_assert(kStages % S == 0, "streams must own whole stages");
     static_assert(kDOff + S * 2 * N <= kTmemCols, "tensor memory budget");
-    static_assert(kBBytes <= kBBytesMax, "B buffer");
+    static_assert(kSliceB <= kBBytesMax, "B buffer");
+    static_assert(NH == 1 || kBBytes >= NQ * kD * NH * 4, "a wide head's B buffer holds its rotation scratch");
 };
 
 __device__ unsigned int g_status;
@@ -177,37 +187,52 @@ __device__ __forceinline__ int b_offset(int n, int k)
 }
 
 // Rotate the G queries of KV head h and write their digits into B buffer `b`
-// of stream g (the stream's 128 threads; thread j owns coordinate j).
-template <int B, int NQ>
+// of stream g (the stream's 128 threads; thread j owns coordinates j + 128 l of
+// the NH slices l).  Slice l's digits form their own K = 256 block of B, at
+// l * N * kK bytes.  The rotation works in S.q at d = 128; for wider heads the
+// B buffer itself is the scratch (it is free, and every byte of it is written
+// with digits only after the last read of the rotated values).
+template <int B, int NQ, int NH>
 __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *inv, int h, int &phase)
 {
     using LK = Lookup<B>;
+    constexpr int D = kD * NH;
+    constexpr int kSliceB = 4 * NQ * kK;        // bytes of one slice's digits (N rows x K)
     const int tid = threadIdx.x & (kGroupThreads - 1);
-    float(*q)[kD] = reinterpret_cast<float(*)[kD]>(S.q + g * NQ * kD);
-    const float sg = (p.quats || p.signs[tid] >= 0) ? 1.0f : -1.0f;
+    float(*q)[D] = reinterpret_cast<float(*)[D]>(NH == 1 ? S.q + g * NQ * kD : reinterpret_cast<float *>(b));
 #pragma unroll
-    for (int qi = 0; qi < NQ; ++qi)
-        q[qi][tid] = (qi < p.group)
-                         ? sg * load_q(p.q, p.qdtype, (static_cast<int64_t>(h) * p.group + qi) * kD + tid)
-                         : 0.0f;
+    for (int sl = 0; sl < NH; ++sl) {
+        const int j = tid + kD * sl;
+        const float sg = (p.quats || p.signs[j] >= 0) ? 1.0f : -1.0f;
+#pragma unroll
+        for (int qi = 0; qi < NQ; ++qi)
+            q[qi][j] = (qi < p.group)
+                           ? sg * load_q(p.q, p.qdtype, (static_cast<int64_t>(h) * p.group + qi) * D + j)
+                           : 0.0f;
+    }
     if (!stream_sync(S, g, phase)) return false;
-    float qq[NQ];
+    float qq[NQ][NH];
     if (p.quats) {
         // q'' = T q / sqrt(d): the IsoQuant block rotation T (orthonormal) times the
-        // temperature; this thread's coordinate from its 4-element block
-        Quat qL, qRc;
-        block_quats(p.quats, tid >> 2, qL, qRc);
-        const int b0 = tid & ~3;
+        // temperature; each coordinate from its 4-element block
+        const float inv_sqrt_d = (NH == 1) ? kInvSqrtD : 1.0f / sqrtf(static_cast<float>(D));
 #pragma unroll
-        for (int qi = 0; qi < NQ; ++qi) {
-            const Quat y = block_rotate(qL, qRc, {q[qi][b0], q[qi][b0 + 1], q[qi][b0 + 2], q[qi][b0 + 3]});
-            const float c = (tid & 3) == 0 ? y.w : (tid & 3) == 1 ? y.x : (tid & 3) == 2 ? y.y : y.z;
-            qq[qi] = c * kInvSqrtD;
+        for (int sl = 0; sl < NH; ++sl) {
+            const int j = tid + kD * sl;
+            Quat qL, qRc;
+            block_quats(p.quats, j >> 2, qL, qRc);
+            const int b0 = j & ~3;
+#pragma unroll
+            for (int qi = 0; qi < NQ; ++qi) {
+                const Quat y = block_rotate(qL, qRc, {q[qi][b0], q[qi][b0 + 1], q[qi][b0 + 2], q[qi][b0 + 3]});
+                const float c = (j & 3) == 0 ? y.w : (j & 3) == 1 ? y.x : (j & 3) == 2 ? y.y : y.z;
+                qq[qi][sl] = c * inv_sqrt_d;
+            }
         }
     } else {
-        for (int hh = 1; hh < kD; hh <<= 1) {
-            for (int t = tid; t < NQ * (kD / 2); t += kGroupThreads) {
-                const int qi = t / (kD / 2), pi = t % (kD / 2);
+        for (int hh = 1; hh < D; hh <<= 1) {
+            for (int t = tid; t < NQ * (D / 2); t += kGroupThreads) {
+                const int qi = t / (D / 2), pi = t % (D / 2);
                 const int i = (pi / hh) * 2 * hh + (pi % hh);
                 const float x = q[qi][i], y = q[qi][i + hh];
                 q[qi][i] = x + y;
@@ -217,11 +242,15 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
         }
         // q'' = H diag(s) q / d  (rotation 1/sqrt(d) times temperature 1/sqrt(d))
 #pragma unroll
-        for (int qi = 0; qi < NQ; ++qi) qq[qi] = q[qi][tid] * (1.0f / kD);
+        for (int qi = 0; qi < NQ; ++qi)
+#pragma unroll
+            for (int sl = 0; sl < NH; ++sl) qq[qi][sl] = q[qi][tid + kD * sl] * (1.0f / D);
     }
 #pragma unroll
     for (int qi = 0; qi < NQ; ++qi) {
-        float m = fabsf(qq[qi]);
+        float m = 0.0f;
+#pragma unroll
+        for (int sl = 0; sl < NH; ++sl) m = fmaxf(m, fabsf(qq[qi][sl]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if ((tid & 31) == 0) S.qmax[g][tid >> 5][qi] = m;
@@ -237,23 +266,27 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
         for (int w = 0; w < 4; ++w) m = fmaxf(m, S.qmax[g][w][qi]);
         const float sq = (m > 0.0f) ? 64.0f / m : 1.0f;
         if (tid == 0) inv[qi] = p.inv_sc / sq;
-        const float Q = qq[qi] * sq;                      // |Q| <= 64
-        const float d0 = rintf(Q);
-        const float r1 = (Q - d0) * 128.0f;
-        const float d1 = rintf(r1);
-        const float d2 = rintf((r1 - d1) * 128.0f);
-        const uint8_t D0 = static_cast<uint8_t>(static_cast<int8_t>(d0));
-        const uint8_t D1 = static_cast<uint8_t>(static_cast<int8_t>(d1));
-        const uint8_t D2 = static_cast<uint8_t>(static_cast<int8_t>(d2));
-        // column weights (128, 1, 1/128, 1/128^2): hi rows (D0, D1, D2, 0), lo rows (0, D0, D1, D2)
-        b[b_offset(4 * qi + 0, k_hi)] = D0;
-        b[b_offset(4 * qi + 1, k_hi)] = D1;
-        b[b_offset(4 * qi + 2, k_hi)] = D2;
-        b[b_offset(4 * qi + 3, k_hi)] = 0;
-        b[b_offset(4 * qi + 0, k_lo)] = 0;
-        b[b_offset(4 * qi + 1, k_lo)] = D0;
-        b[b_offset(4 * qi + 2, k_lo)] = D1;
-        b[b_offset(4 * qi + 3, k_lo)] = D2;
+#pragma unroll
+        for (int sl = 0; sl < NH; ++sl) {
+            uint8_t *bs = b + sl * kSliceB;
+            const float Q = qq[qi][sl] * sq;                  // |Q| <= 64
+            const float d0 = rintf(Q);
+            const float r1 = (Q - d0) * 128.0f;
+            const float d1 = rintf(r1);
+            const float d2 = rintf((r1 - d1) * 128.0f);
+            const uint8_t D0 = static_cast<uint8_t>(static_cast<int8_t>(d0));
+            const uint8_t D1 = static_cast<uint8_t>(static_cast<int8_t>(d1));
+            const uint8_t D2 = static_cast<uint8_t>(static_cast<int8_t>(d2));
+            // column weights (128, 1, 1/128, 1/128^2): hi rows (D0, D1, D2, 0), lo rows (0, D0, D1, D2)
+            bs[b_offset(4 * qi + 0, k_hi)] = D0;
+            bs[b_offset(4 * qi + 1, k_hi)] = D1;
+            bs[b_offset(4 * qi + 2, k_hi)] = D2;
+            bs[b_offset(4 * qi + 3, k_hi)] = 0;
+            bs[b_offset(4 * qi + 0, k_lo)] = 0;
+            bs[b_offset(4 * qi + 1, k_lo)] = D0;
+            bs[b_offset(4 * qi + 2, k_lo)] = D1;
+            bs[b_offset(4 * qi + 3, k_lo)] = D2;
+        }
     }
     fence_proxy_async_smem();
     return stream_sync(S, g, phase);
@@ -371,16 +404,22 @@ constexpr int kBRegion = 32768;       // two B buffers per stream, for every str
 constexpr int kRestBytes = kStages * kStageBytes + kBRegion + kSmemBook;
 constexpr size_t kSmemRequest = 1024 + 65536 + kLutBytes + kRestBytes;
 static_assert(kSmemRequest <= 232448, "shared memory per block");
-static_assert(Cfg<8>::S * 2 * Cfg<8>::kBBytes <= kBRegion && Cfg<4>::S * 2 * Cfg<4>::kBBytes <= kBRegion,
+template <int NQ, int NH>
+constexpr bool b_fits()
+{
+    return Cfg<NQ, NH>::S * Cfg<NQ, NH>::kBBufs * Cfg<NQ, NH>::kBBytes <= kBRegion;
+}
+static_assert(b_fits<4, 1>() && b_fits<8, 1>() && b_fits<4, 2>() && b_fits<8, 2>() && b_fits<4, 4>() &&
+                  b_fits<8, 4>(),
               "B buffers of every stream fit");
 
 // Worker threads of tile stream g (local tiles k = 0, 1, ... are the CTA's
 // tiles t0 + g + S*k): one thread per key of a tile.
-template <int B, int NQ>
+template <int B, int NQ, int NH>
 struct Worker {
     using LK = Lookup<B>;
-    using C = Cfg<NQ>;
-    static constexpr int P = kD * B / 8;
+    using C = Cfg<NQ, NH>;
+    static constexpr int P = kD * B / 8;      // bytes of one 128-coordinate slice of a packed row
     static constexpr int NW = P / 4;
 
     static constexpr int NL = C::N / 16;      // 16-column loads of one D buffer
@@ -442,100 +481,130 @@ struct Worker {
         float inv[NQ];
 
         for (int tile = t0 + g; tile < t1; tile += C::S, ++k) {
-            if (!mbar_wait_warp(smem_u32(&S.full[s]), sph)) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutLoad);
-                ok = false;
-                break;
-            }
-            uint32_t w[NW + 1];
-            {
-                const uint8_t *st = sStage + s * kStageBytes;
-#pragma unroll
-                for (int c = 0; c < P / 16; ++c) {
-                    const uint4 x = *reinterpret_cast<const uint4 *>(st + chunk_offset<P>(r, c));
-                    w[4 * c] = x.x; w[4 * c + 1] = x.y; w[4 * c + 2] = x.z; w[4 * c + 3] = x.w;
+            float nk = 0.0f;
+#pragma unroll 1
+            for (int sl = 0; sl < NH; ++sl) {
+                const int m = k * NH + sl;      // this stream's subtile count
+                if constexpr (NH > 1) {
+                    // the CTA's load of (tile, slice) went to stage i mod kStages
+                    const int i = (tile - t0) * NH + sl;
+                    s = i % kStages;
+                    sph = static_cast<uint32_t>(i / kStages) & 1u;
                 }
-                w[NW] = 0;
-            }
-            // this tile's key norm (its scores are due two tiles from now)
-            float nk = reinterpret_cast<const float *>(sStage + s * kStageBytes + kStageCodeBytes)
-                [((h * p.head_stride + ti * kTileRows + p.nshift) & 3) + r];
-            mbar_arrive(smem_u32(&S.empty[s]));
-
-            // products of tile k - 2 done: its D is readable, its A buffer and the
-            // B buffer of two heads back are free
-            const int ab = k & 1;
-            if (!mbar_wait_warp(smem_u32(&S.mma_done[g][ab]), ((k >> 1) & 1) ^ 1)) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                ok = false;
-                break;
-            }
-            tc_fence_after_sync();
-            // scores of tile k - 2, read out of D before tile k's products may overwrite it
-            if (k >= 2) {
-                uint32_t acc[NL][16];
-                load_sums(tmem_lane + C::kDOff + (2 * g + ab) * C::N, acc);
-                store_sums(p, S, g, acc, nk2, hs2, h2, t2k + r, inv_hc, inv);
-            }
-
-            if (h != prev_h) {
-                bsel = (bsel < 0) ? 0 : (bsel ^ 1);
-                prev_h = h;
-                ++hc;
-                if (!build_b<B, NQ>(p, S, g, sB + (2 * g + bsel) * C::kBBytes, S.inv[g][hc & (kInvSlots - 1)], h,
-                                    sync_phase)) {
-                    if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                if (!mbar_wait_warp(smem_u32(&S.full[s]), sph)) {
+                    if (lane == 0) atomicOr(&g_status, kErrTimeoutLoad);
                     ok = false;
                     break;
                 }
-            }
-            // decode step: this head's last tile holds the appended key, whose row
-            // the stage has only as it was before this launch
-            if (p.append_pos >= 0 && ti == (p.append_pos >> 7)) {
-                float nka;
-                if (!append_key<B, NQ>(p, S, g, h, &nka, sync_phase)) {
-                    if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                uint32_t w[NW + 1];
+                {
+                    const uint8_t *st = sStage + s * kStageBytes;
+#pragma unroll
+                    for (int c = 0; c < P / 16; ++c) {
+                        const uint4 x = *reinterpret_cast<const uint4 *>(st + chunk_offset<P>(r, c));
+                        w[4 * c] = x.x; w[4 * c + 1] = x.y; w[4 * c + 2] = x.z; w[4 * c + 3] = x.w;
+                    }
+                    w[NW] = 0;
+                }
+                // this tile's key norm, with its first slice (its scores are due two tiles from now)
+                if (sl == 0)
+                    nk = reinterpret_cast<const float *>(sStage + s * kStageBytes + kStageCodeBytes)
+                        [((h * p.head_stride + ti * kTileRows + p.nshift) & 3) + r];
+                mbar_arrive(smem_u32(&S.empty[s]));
+
+                // products of subtile m - 2 done: its A buffer is free, and with it
+                // every product of tile k - 2 (its D is readable) and of the B
+                // buffer of two heads back
+                const int ab = m & 1;
+                if (!mbar_wait_warp(smem_u32(&S.mma_done[g][ab]), ((m >> 1) & 1) ^ 1)) {
+                    if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
                     ok = false;
                     break;
                 }
-                if (r == (p.append_pos & (kTileRows - 1))) {
+                tc_fence_after_sync();
+                if (sl == 0) {
+                    // scores of tile k - 2, read out of D before tile k's products may overwrite it
+                    if (k >= 2) {
+                        uint32_t acc[NL][16];
+                        load_sums(tmem_lane + C::kDOff + (2 * g + (k & 1)) * C::N, acc);
+                        store_sums(p, S, g, acc, nk2, hs2, h2, t2k + r, inv_hc, inv);
+                    }
+                    if (h != prev_h) {
+                        if constexpr (C::kBBufs == 1) {
+                            // one B buffer: the last head's products must be done with it
+                            if (m >= 1 && !mbar_wait_warp(smem_u32(&S.mma_done[g][(m - 1) & 1]), ((m - 1) >> 1) & 1)) {
+                                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after_sync();
+                            bsel = 0;
+                        } else {
+                            bsel = (bsel < 0) ? 0 : (bsel ^ 1);
+                        }
+                        prev_h = h;
+                        ++hc;
+                        if (!build_b<B, NQ, NH>(p, S, g, sB + (C::kBBufs * g + bsel) * C::kBBytes,
+                                                S.inv[g][hc & (kInvSlots - 1)], h, sync_phase)) {
+                            if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                            ok = false;
+                            break;
+                        }
+                    }
+                    // decode step: this head's last tile holds the appended key, whose row
+                    // the stage has only as it was before this launch
+                    if constexpr (NH == 1) {
+                        if (p.append_pos >= 0 && ti == (p.append_pos >> 7)) {
+                            float nka;
+                            if (!append_key<B, NQ>(p, S, g, h, &nka, sync_phase)) {
+                                if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                                ok = false;
+                                break;
+                            }
+                            if (r == (p.append_pos & (kTileRows - 1))) {
 #pragma unroll
-                    for (int i = 0; i < NW; ++i) w[i] = S.arow[g][i];
-                    nk = nka;
+                                for (int i = 0; i < NW; ++i) w[i] = S.arow[g][i];
+                                nk = nka;
+                            }
+                        }
+                    }
                 }
-            }
 
-            // lookup l fills A columns l (4-byte entries) or 2l, 2l+1 (8-byte entries)
-            const uint32_t a_addr = tmem_lane + (2 * g + ab) * kACols;
+                // lookup l fills A columns l (4-byte entries) or 2l, 2l+1 (8-byte entries)
+                const uint32_t a_addr = tmem_lane + (2 * g + ab) * kACols;
 #pragma unroll
-            for (int qt = 0; qt < 4; ++qt) {
-                uint32_t a[16];
-                if constexpr (LK::EB == 4) {
+                for (int qt = 0; qt < 4; ++qt) {
+                    uint32_t a[16];
+                    if constexpr (LK::EB == 4) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint32_t ad = lut_addr<B>(w, 16 * qt + i, base_lane);
-                        asm("ld.shared.u32 %0, [%1];" : "=r"(a[i]) : "r"(ad));
+                        for (int i = 0; i < 16; ++i) {
+                            const uint32_t ad = lut_addr<B>(w, 16 * qt + i, base_lane);
+                            asm("ld.shared.u32 %0, [%1];" : "=r"(a[i]) : "r"(ad));
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t ad = lut_addr<B>(w, 8 * qt + i, base_lane);
+                            asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a[2 * i]), "=r"(a[2 * i + 1]) : "r"(ad));
+                        }
                     }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t ad = lut_addr<B>(w, 8 * qt + i, base_lane);
-                        asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a[2 * i]), "=r"(a[2 * i + 1]) : "r"(ad));
+                    tmem_st16(a_addr + 16 * qt, a);
+                }
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(smem_u32(&S.a_full[g][ab]));
+                if constexpr (NH == 1) {
+                    s += C::S;
+                    if (s >= kStages) {
+                        s -= kStages;
+                        sph ^= 1;
                     }
                 }
-                tmem_st16(a_addr + 16 * qt, a);
             }
-            tmem_wait_st();
-            tc_fence_before_sync();
-            mbar_arrive(smem_u32(&S.a_full[g][ab]));
+            if (!ok) break;
 
             h2 = h1; t2k = t1k; hs2 = hs1; nk2 = nk1;
             h1 = h; t1k = ti * kTileRows; hs1 = hc; nk1 = nk;
-            s += C::S;
-            if (s >= kStages) {
-                s -= kStages;
-                sph ^= 1;
-            }
             ti += C::S;
             while (ti >= p.tiles_per_head) {
                 ti -= p.tiles_per_head;
@@ -543,11 +612,12 @@ struct Worker {
             }
         }
 
-        // the last two tiles' scores
+        // the last two tiles' scores (each complete with the products of its last subtile)
         if (ok) {
             for (int j = (k >= 2 ? k - 2 : 0); j < k; ++j) {
                 const bool last = (j == k - 1);
-                if (!mbar_wait_warp(smem_u32(&S.mma_done[g][j & 1]), (j >> 1) & 1)) {
+                const int mj = j * NH + NH - 1;
+                if (!mbar_wait_warp(smem_u32(&S.mma_done[g][mj & 1]), (mj >> 1) & 1)) {
                     if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
                     break;
                 }
@@ -561,12 +631,12 @@ struct Worker {
     }
 };
 
-template <int B, int NQ>
-__global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const __grid_constant__ TcParams p)
+template <int B, int NQ, int NH>
+__global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(const __grid_constant__ TcParams p)
 {
     using LK = Lookup<B>;
-    using C = Cfg<NQ>;
-    constexpr int P = kD * B / 8;
+    using C = Cfg<NQ, NH>;
+    constexpr int P = kD * B / 8;             // bytes of one 128-coordinate slice of a packed row
     static_assert(kTileRows * P <= kStageCodeBytes && kStageCodeBytes + kNormBox * 4 <= kStageBytes,
                   "stage too small for a tile of packed rows and its norms");
     static_assert(LK::NF * 256 <= kLutBytes, "lookup table too large");
@@ -621,20 +691,26 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const _
             int it = 0, s = 0;
             uint32_t ph = 0;
             int h = t0 / p.tiles_per_head, ti = t0 - h * p.tiles_per_head;
-            for (int tile = t0; tile < t1; ++tile, ++it) {
-                if (!mbar_wait(smem_u32(&S.empty[s]), ph ^ 1)) {
-                    atomicOr(&g_status, kErrTimeoutDrain);
-                    break;
-                }
-                const uint32_t full = smem_u32(&S.full[s]);
+            bool stop = false;
+            for (int tile = t0; tile < t1 && !stop; ++tile) {
                 const int row = h * p.head_stride + ti * kTileRows;
-                mbar_arrive_expect_tx(full, kTileRows * P + kNormBox * 4);
-                tma_load_2d(smem_u32(sStage + s * kStageBytes), &p.tmap, 0, row, full);
-                tma_load_1d(smem_u32(sStage + s * kStageBytes + kStageCodeBytes), &p.nmap, (row + p.nshift) & ~3,
-                            full);
-                if (++s == kStages) {
-                    s = 0;
-                    ph ^= 1;
+                // one stage per 128-coordinate slice of the tile; the norms come with the first
+                for (int sl = 0; sl < NH; ++sl, ++it) {
+                    if (!mbar_wait(smem_u32(&S.empty[s]), ph ^ 1)) {
+                        atomicOr(&g_status, kErrTimeoutDrain);
+                        stop = true;
+                        break;
+                    }
+                    const uint32_t full = smem_u32(&S.full[s]);
+                    mbar_arrive_expect_tx(full, kTileRows * P + (sl == 0 ? kNormBox * 4 : 0));
+                    tma_load_2d(smem_u32(sStage + s * kStageBytes), &p.tmap, sl * P, row, full);
+                    if (sl == 0)
+                        tma_load_1d(smem_u32(sStage + s * kStageBytes + kStageCodeBytes), &p.nmap,
+                                    (row + p.nshift) & ~3, full);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
                 }
                 if (++ti == p.tiles_per_head) {
                     ti = 0;
@@ -652,7 +728,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const _
         if (lane == 0) {
             const int g = warp - C::kWarpMma0;
             const uint32_t id = idesc(kAccS32, kFmtS8, kFmtS8, 128, C::N);
-            const uint32_t b0 = smem_u32(sB) + 2 * g * C::kBBytes;
+            const uint32_t b0 = smem_u32(sB) + C::kBBufs * g * C::kBBytes;
             const uint32_t a0 = tmem + 2 * g * kACols;
             const uint32_t d0 = tmem + C::kDOff + 2 * g * C::N;
             // the stream's B buffer flips whenever its tiles enter a new head,
@@ -660,25 +736,34 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const _
             int bsel = 1, prev_h = -1;
             int h = (t0 + g) / p.tiles_per_head, ti = (t0 + g) - h * p.tiles_per_head;
             int k = 0;
-            for (int tile = t0 + g; tile < t1; tile += C::S, ++k) {
+            bool stop = false;
+            for (int tile = t0 + g; tile < t1 && !stop; tile += C::S, ++k) {
                 if (h != prev_h) {
-                    bsel ^= 1;
+                    bsel = (C::kBBufs == 1) ? 0 : (bsel ^ 1);
                     prev_h = h;
                 }
-                const int ab = k & 1;
-                // A of this tile written (which also means the workers have read
-                // the D of tile k - 2 out of this buffer)
-                if (!mbar_wait(smem_u32(&S.a_full[g][ab]), (k >> 1) & 1)) {
-                    atomicOr(&g_status, kErrTimeoutLoad);
-                    break;
-                }
-                tc_fence_after_sync();
-                // K step kk reads B 256 bytes further on: +16 in the address field
-                const uint64_t bd = desc_k_interleave(b0 + bsel * C::kBBytes, 128, (kK / 16) * 128);
-                const uint32_t d = d0 + ab * C::N, a = a0 + ab * kACols;
+                const uint32_t d = d0 + (k & 1) * C::N;
+                for (int sl = 0; sl < NH; ++sl) {
+                    const int m = k * NH + sl;
+                    const int ab = m & 1;
+                    // A of this subtile written (which also means the workers have read
+                    // the D of tile k - 2 out of this tile's D buffer)
+                    if (!mbar_wait(smem_u32(&S.a_full[g][ab]), (m >> 1) & 1)) {
+                        atomicOr(&g_status, kErrTimeoutLoad);
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    // K step kk reads B 256 bytes further on: +16 in the address field;
+                    // slice sl's digits are the sl-th K block of the buffer
+                    const uint64_t bd =
+                        desc_k_interleave(b0 + bsel * C::kBBytes + sl * C::kSliceB, 128, (kK / 16) * 128);
+                    const uint32_t a = a0 + ab * kACols;
 #pragma unroll
-                for (int kk = 0; kk < kK / 32; ++kk) mma_i8_ts(d, a + 8 * kk, bd + 16 * kk, id, kk > 0);
-                mma_commit(smem_u32(&S.mma_done[g][ab]));
+                    for (int kk = 0; kk < kK / 32; ++kk)
+                        mma_i8_ts(d, a + 8 * kk, bd + 16 * kk, id, sl > 0 || kk > 0);
+                    mma_commit(smem_u32(&S.mma_done[g][ab]));
+                }
                 ti += C::S;
                 while (ti >= p.tiles_per_head) {
                     ti -= p.tiles_per_head;
@@ -690,7 +775,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc_kernel(const _
         }
     } else {
         // ----------------------------------------------------------- workers
-        Worker<B, NQ>::run(p, S, warp / 4, sStage, sB, lut_pos, tmem, t0, t1);
+        Worker<B, NQ, NH>::run(p, S, warp / 4, sStage, sB, lut_pos, tmem, t0, t1);
     }
 
     tc_fence_before_sync();
@@ -721,11 +806,12 @@ EncodeTiledFn encode_tiled()
     return fn;
 }
 
-template <int B, int NQ>
+template <int B, int NQ, int NH>
 cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
 {
-    constexpr int P = kD * B / 8;
-    auto kernel = scores_tc_kernel<B, NQ>;
+    constexpr int P = kD * B / 8;             // one slice of a row: the TMA box width
+    constexpr int PT = P * NH;                // the whole packed row
+    auto kernel = scores_tc_kernel<B, NQ, NH>;
     const size_t smem = kSmemRequest;
     static bool configured = false;
     if (!configured) {
@@ -737,9 +823,9 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return cudaErrorNotSupported;
     TcParams p{};
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(P),
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(PT),
                                 static_cast<cuuint64_t>(a.heads) * static_cast<cuuint64_t>(a.head_stride)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(P)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(PT)};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(P), kTileRows};
     const cuuint32_t estr[2] = {1, 1};
     const CUtensorMapSwizzle swz = (P == 64) ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -794,32 +880,45 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
         p.lo[i] = static_cast<int8_t>(vi - 128 * hi);
     }
     const int used = (p.total_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
-    kernel<<<used, Cfg<NQ>::kThreads, smem, stream>>>(p);
+    kernel<<<used, Cfg<NQ, NH>::kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
-template <int B>
+template <int B, int NH>
 cudaError_t launch_b(const ScoresArgs &a, cudaStream_t stream)
 {
-    return a.group <= 4 ? launch_bn<B, 4>(a, stream) : launch_bn<B, 8>(a, stream);
+    return a.group <= 4 ? launch_bn<B, 4, NH>(a, stream) : launch_bn<B, 8, NH>(a, stream);
+}
+
+template <int NH>
+cudaError_t launch_h(const ScoresArgs &a, cudaStream_t stream)
+{
+    switch (a.b) {
+    case 1: return launch_b<1, NH>(a, stream);
+    case 2: return launch_b<2, NH>(a, stream);
+    case 3: return launch_b<3, NH>(a, stream);
+    default: return launch_b<4, NH>(a, stream);
+    }
 }
 
 }  // namespace
 
 bool scores_tc_supported(const ScoresArgs &a)
 {
-    return a.d == kD && a.b >= 1 && a.b <= 4 && a.group <= 8 && a.n > 0 &&
+    // d = 256 and 512 run as 2 and 4 slices of 128 coordinates; the fused decode
+    // step (one appended key quantized in the kernel) exists for d = 128 only
+    const bool width = a.d == kD || ((a.d == 2 * kD || a.d == 4 * kD) && a.k_new == nullptr);
+    return width && a.b >= 1 && a.b <= 4 && a.group <= 8 && a.n > 0 &&
            static_cast<int64_t>(a.heads) * a.head_stride < (static_cast<int64_t>(1) << 31) - kTileRows &&
            encode_tiled() != nullptr;
 }
 
 cudaError_t launch_scores_tc(const ScoresArgs &a, cudaStream_t stream)
 {
-    switch (a.b) {
-    case 1: return launch_b<1>(a, stream);
-    case 2: return launch_b<2>(a, stream);
-    case 3: return launch_b<3>(a, stream);
-    default: return launch_b<4>(a, stream);
+    switch (a.d) {
+    case 2 * kD: return launch_h<2>(a, stream);
+    case 4 * kD: return launch_h<4>(a, stream);
+    default: return launch_h<1>(a, stream);
     }
 }
 

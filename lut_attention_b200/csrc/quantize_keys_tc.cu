@@ -51,7 +51,10 @@ constexpr int kHalfBytes = kTileRows * 128;     // one 64-element K block of a t
 constexpr int kGroupWarps = 8;                  // one epilogue group: two warps per lane quadrant
 constexpr int kEpiWarps = 2 * kGroupWarps;      // two groups, one per accumulator
 constexpr int kThreads = (kEpiWarps + 2) * 32;
-constexpr int kTmemCols = 256;                  // two 128-column accumulators
+// d = 128 * NH: a tile's keys arrive as NH stages of 128 coordinates, and each
+// 128-key tile has NH accumulators of 128 columns (two tiles in flight)
+template <int NH>
+__host__ __device__ constexpr int tmem_cols() { return 256 * NH; }
 constexpr int kWarpTma = kEpiWarps, kWarpMma = kEpiWarps + 1;
 constexpr uint32_t kMagicBits = 0x4B400000u;    // bits of 1.5 * 2^23
 constexpr float kMagic = 12582912.0f;
@@ -126,17 +129,33 @@ __device__ __forceinline__ void quantize_chunk(const uint32_t (&v)[32], float2 a
     }
 }
 
-template <int B, bool kBF16>
+// one run of NWH packed words (64 coordinates), 16- or 8-byte streaming stores
+template <int NWH>
+__device__ __forceinline__ void store_run(uint8_t *dst, const uint32_t *w)
+{
+    if constexpr (NWH % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NWH / 4; ++i)
+            __stcs(reinterpret_cast<uint4 *>(dst) + i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+    } else {
+#pragma unroll
+        for (int i = 0; i < NWH / 2; ++i) __stcs(reinterpret_cast<uint2 *>(dst) + i, make_uint2(w[2 * i], w[2 * i + 1]));
+    }
+}
+
+template <int B, bool kBF16, int NH>
 __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __grid_constant__ TcParams p)
 {
-    constexpr int P = kD * B / 8;            // packed bytes per key
-    constexpr int NW = P / 4;                // packed 32-bit words per key
+    constexpr int D = kD * NH;
+    constexpr int kTmemCols = tmem_cols<NH>();
+    constexpr int P = D * B / 8;             // packed bytes per key
+    constexpr int NW = kD * B / 8 / 4;       // packed 32-bit words per 128 coordinates
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
     uint8_t *sA = base;                                      // kStages x 32 KB
-    uint8_t *sB = sA + kStages * kABytes;                    // 32 KB
-    float2 *sTab = reinterpret_cast<float2 *>(sB + kBBytes); // kMaxBuckets entries
+    uint8_t *sB = sA + kStages * kABytes;                    // NH x 32 KB
+    float2 *sTab = reinterpret_cast<float2 *>(sB + NH * kBBytes); // kMaxBuckets entries
     Smem &S = *reinterpret_cast<Smem *>(sTab + kMaxBuckets);
 
     const int warp = threadIdx.x >> 5;
@@ -158,10 +177,14 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
     }
     if (warp == kWarpTma && lane == 0) prefetch_tensormap(&p.tmap);
 
-    // B = H diag(s) as [n = output coordinate][k = input coordinate], K-major,
-    // two 64-column blocks of 128-byte swizzled rows (the layout TMA gives A).
-    for (int chunk = threadIdx.x; chunk < kD * (kD / 8); chunk += kThreads) {
-        const int n = chunk / (kD / 8);
+    // B_l = H diag(s_l), s_l the signs of coordinates 128 l .. 128 l + 127, as
+    // [n = output coordinate][k = input coordinate], K-major, two 64-column blocks
+    // of 128-byte swizzled rows (the layout TMA gives A).  For d = 256 the
+    // Sylvester recursion H_256 = [[H, H], [H, -H]] gives y = (z_0 + z_1, z_0 - z_1)
+    // with z_l = B_l k_l, which the epilogue forms.
+    for (int chunk = threadIdx.x; chunk < NH * kD * (kD / 8); chunk += kThreads) {
+        const int l = chunk / (kD * (kD / 8));
+        const int n = (chunk / (kD / 8)) % kD;
         const int c = chunk % (kD / 8);          // 8-element chunk along k
         uint32_t w[4];
 #pragma unroll
@@ -170,14 +193,14 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int k = 8 * c + 2 * e2 + h;
-                const bool neg = ((__popc(n & k) & 1) != 0) != (p.signs[k] < 0);
+                const bool neg = ((__popc(n & k) & 1) != 0) != (p.signs[kD * l + k] < 0);
                 const uint16_t one = kBF16 ? (neg ? 0xBF80 : 0x3F80) : (neg ? 0xBC00 : 0x3C00);
                 pair |= static_cast<uint32_t>(one) << (16 * h);
             }
             w[e2] = pair;
         }
         const int kb = c / 8, cc = c % 8;
-        uint4 *dst = reinterpret_cast<uint4 *>(sB + kb * kHalfBytes + n * 128 + ((cc ^ (n & 7)) * 16));
+        uint4 *dst = reinterpret_cast<uint4 *>(sB + l * kBBytes + kb * kHalfBytes + n * 128 + ((cc ^ (n & 7)) * 16));
         *dst = make_uint4(w[0], w[1], w[2], w[3]);
     }
     for (int j = threadIdx.x; j < kMaxBuckets; j += kThreads)
@@ -197,17 +220,21 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         // ---------------------------------------------------------- producer
         if (lane == 0) {
             int it = 0;
-            for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
-                if (!mbar_wait(smem_u32(&S.empty[s]), ph ^ 1)) {
-                    atomicOr(&g_status, kErrTimeoutMma);
-                    break;
+            bool stop = false;
+            for (int t = blockIdx.x; t < p.ntiles && !stop; t += gridDim.x) {
+                for (int l = 0; l < NH; ++l, ++it) {         // one stage per 128 coordinates
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!mbar_wait(smem_u32(&S.empty[s]), ph ^ 1)) {
+                        atomicOr(&g_status, kErrTimeoutMma);
+                        stop = true;
+                        break;
+                    }
+                    const uint32_t full = smem_u32(&S.full[s]);
+                    mbar_arrive_expect_tx(full, kABytes);
+                    tma_load_2d(smem_u32(sA + s * kABytes), &p.tmap, kD * l, t * kTileRows, full);
+                    tma_load_2d(smem_u32(sA + s * kABytes + kHalfBytes), &p.tmap, kD * l + 64, t * kTileRows, full);
                 }
-                const uint32_t full = smem_u32(&S.full[s]);
-                mbar_arrive_expect_tx(full, kABytes);
-                tma_load_2d(smem_u32(sA + s * kABytes), &p.tmap, 0, t * kTileRows, full);
-                tma_load_2d(smem_u32(sA + s * kABytes + kHalfBytes), &p.tmap, 64, t * kTileRows, full);
             }
             // let every load this thread issued land before the CTA exits
             for (int k = 0; k < kStages && k < it; ++k) {
@@ -220,28 +247,35 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         if (lane == 0) {
             const uint32_t id = idesc(kAccF32, kBF16 ? kFmtBF16 : kFmtF16, kBF16 ? kFmtBF16 : kFmtF16, 128, kD);
             const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
-            int it = 0;
-            for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
+            int it = 0, st = 0;                               // tiles, stages
+            bool stop = false;
+            for (int t = blockIdx.x; t < p.ntiles && !stop; t += gridDim.x, ++it) {
                 const int acc = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
-                if (!mbar_wait(smem_u32(&S.full[s]), ph)) {
-                    atomicOr(&g_status, kErrTimeoutLoad);
-                    break;
-                }
                 if (!mbar_wait(smem_u32(&S.acc_empty[acc]), aph ^ 1)) {
                     atomicOr(&g_status, kErrTimeoutDrain);
                     break;
                 }
-                tc_fence_after_sync();
-                const uint32_t d = tmem + acc * kD;
+                for (int l = 0; l < NH; ++l, ++st) {
+                    const int s = st % kStages;
+                    const uint32_t ph = (st / kStages) & 1;
+                    if (!mbar_wait(smem_u32(&S.full[s]), ph)) {
+                        atomicOr(&g_status, kErrTimeoutLoad);
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    // accumulator acc holds z_0 .. z_{NH-1}, 128 columns each
+                    const uint32_t d = tmem + (acc * NH + l) * kD;
 #pragma unroll
-                for (int k = 0; k < kD / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
-                    mma_f16_ss(d, desc_k_sw128(a0 + s * kABytes + off), desc_k_sw128(b0 + off), id, k > 0);
+                    for (int k = 0; k < kD / 16; ++k) {
+                        const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
+                        mma_f16_ss(d, desc_k_sw128(a0 + s * kABytes + off), desc_k_sw128(b0 + l * kBBytes + off), id,
+                                   k > 0);
+                    }
+                    mma_commit(smem_u32(&S.empty[s]));
                 }
-                mma_commit(smem_u32(&S.empty[s]));
+                if (stop) break;
                 mma_commit(smem_u32(&S.acc_full[acc]));
             }
             // all MMAs of this thread complete before the tensor memory is freed
@@ -270,21 +304,37 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                 break;
             }
             tc_fence_after_sync();
-            const uint32_t col_addr = tmem + lane_base + acc * kD + half * kHalfCols;
+            // this warp's 64 columns of z_0 (and of z_1 at d = 256)
+            const uint32_t col_addr = tmem + lane_base + acc * NH * kD + half * kHalfCols;
             // pass 1: this half's sum of y^2 (four interleaved partial sums); the
             // pair adds both halves in a fixed order
-            // (partial sums 0,1 and 2,3 in paired FMAs: coordinates e = 0, 1 mod 4 and 2, 3 mod 4)
+            // (partial sums 0,1 and 2,3 in paired FMAs: coordinates e = 0, 1 mod 4 and 2, 3 mod 4;
+            // at d = 256, 0,1 for y = z_0 + z_1 and 2,3 for y = z_0 - z_1)
             float2 p01 = make_float2(0.0f, 0.0f), p23 = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int c = 0; c < kHalfCols / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(col_addr + 32 * c, v);
+                if constexpr (NH == 1) {
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    const float2 x01 = make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                    const float2 x23 = make_float2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                    p01 = __ffma2_rn(x01, x01, p01);
-                    p23 = __ffma2_rn(x23, x23, p23);
+                    for (int e = 0; e < 32; e += 4) {
+                        const float2 x01 = make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                        const float2 x23 = make_float2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                        p01 = __ffma2_rn(x01, x01, p01);
+                        p23 = __ffma2_rn(x23, x23, p23);
+                    }
+                } else {
+                    uint32_t v1[32];
+                    tmem_ld32(col_addr + kD + 32 * c, v1);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float2 z0 = make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                        const float2 z1 = make_float2(__uint_as_float(v1[e]), __uint_as_float(v1[e + 1]));
+                        const float2 ya = __fadd2_rn(z0, z1);
+                        const float2 yb = __ffma2_rn(z1, make_float2(-1.0f, -1.0f), z0);
+                        p01 = __ffma2_rn(ya, ya, p01);
+                        p23 = __ffma2_rn(yb, yb, p23);
+                    }
                 }
             }
             S.ss[acc][half][key] = (p01.x + p01.y) + (p23.x + p23.y);
@@ -296,9 +346,9 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const float ss = S.ss[acc][0][key] + S.ss[acc][1][key];
             const float norm = sqrtf(ss) * p.inv_sqrt_d;
 
-            uint32_t w[NWH + 1];
+            uint32_t w[NWH + 1], w1[NWH + 1];      // codes of y (z_0 + z_1 at d = 256) and of z_0 - z_1
 #pragma unroll
-            for (int i = 0; i <= NWH; ++i) w[i] = 0;
+            for (int i = 0; i <= NWH; ++i) w[i] = w1[i] = 0;
             // pass 2: quantize and pack this half, 32 coordinates at a time.  The
             // tensor-memory loads stay outside the per-key branches (warp-collective).
             // |y| <= sqrt(ss) keeps round(g) inside the table; a zero or denormal
@@ -310,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const float2 a2 = make_float2(a, a);
             const float2 goff2 = make_float2(p.g_off, p.g_off);
             const float2 offm2 = make_float2(p.g_off + kMagic, p.g_off + kMagic);
-            {
+            if constexpr (NH == 1) {
                 uint32_t v[32];
                 tmem_ld32(col_addr, v);
                 if (finite && !clamp) quantize_chunk<B, 0, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
@@ -318,13 +368,52 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                 tmem_ld32(col_addr + 32, v);
                 if (finite && !clamp) quantize_chunk<B, 32, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
                 else if (finite) quantize_chunk<B, 32, 0, true>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
+            } else {
+#pragma unroll
+                for (int c = 0; c < kHalfCols / 32; ++c) {
+                    uint32_t v[32], v1[32];
+                    tmem_ld32(col_addr + 32 * c, v);
+                    tmem_ld32(col_addr + kD + 32 * c, v1);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float2 z0 = make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                        const float2 z1 = make_float2(__uint_as_float(v1[e]), __uint_as_float(v1[e + 1]));
+                        const float2 ya = __fadd2_rn(z0, z1);
+                        const float2 yb = __ffma2_rn(z1, make_float2(-1.0f, -1.0f), z0);
+                        v[e] = __float_as_uint(ya.x);
+                        v[e + 1] = __float_as_uint(ya.y);
+                        v1[e] = __float_as_uint(yb.x);
+                        v1[e + 1] = __float_as_uint(yb.y);
+                    }
+                    if (c == 0) {
+                        if (finite && !clamp) {
+                            quantize_chunk<B, 0, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 0, 0, false>(v1, a2, goff2, offm2, tab_u32, tab_bias, w1);
+                        } else if (finite) {
+                            quantize_chunk<B, 0, 0, true>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 0, 0, true>(v1, a2, goff2, offm2, tab_u32, tab_bias, w1);
+                        }
+                    } else {
+                        if (finite && !clamp) {
+                            quantize_chunk<B, 32, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 32, 0, false>(v1, a2, goff2, offm2, tab_u32, tab_bias, w1);
+                        } else if (finite) {
+                            quantize_chunk<B, 32, 0, true>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 32, 0, true>(v1, a2, goff2, offm2, tab_u32, tab_bias, w1);
+                        }
+                    }
+                }
             }
             if (!finite) {
 #pragma unroll
                 for (int j = 0; j < kHalfCols; ++j) {
                     const int o = j * B;
                     w[o >> 5] |= kCentral << (o & 31);
-                    if ((o & 31) + B > 32) w[(o >> 5) + 1] |= kCentral >> (32 - (o & 31));
+                    w1[o >> 5] |= kCentral << (o & 31);
+                    if ((o & 31) + B > 32) {
+                        w[(o >> 5) + 1] |= kCentral >> (32 - (o & 31));
+                        w1[(o >> 5) + 1] |= kCentral >> (32 - (o & 31));
+                    }
                 }
             }
             tc_fence_before_sync();
@@ -332,17 +421,11 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
 
             const int64_t row = static_cast<int64_t>(t) * kTileRows + key;
             if (row < p.n) {
-                uint8_t *dst = p.idx + row * P + half * (P / 2);
-                if constexpr (NWH % 4 == 0) {
-#pragma unroll
-                    for (int i = 0; i < NWH / 4; ++i)
-                        __stcs(reinterpret_cast<uint4 *>(dst) + i,
-                               make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
-                } else {
-#pragma unroll
-                    for (int i = 0; i < NWH / 2; ++i)
-                        __stcs(reinterpret_cast<uint2 *>(dst) + i, make_uint2(w[2 * i], w[2 * i + 1]));
-                }
+                // this warp's 64 coordinates of each 128: runs of NWH words at
+                // coordinates 64 half and (d = 256) 128 + 64 half
+                uint8_t *dst = p.idx + row * P + half * (NWH * 4);
+                store_run<NWH>(dst, w);
+                if constexpr (NH == 2) store_run<NWH>(dst + 2 * NWH * 4, w1);
                 if (half == 0) __stcs(p.norms + row, norm);
             }
         }
@@ -376,11 +459,14 @@ EncodeTiledFn encode_tiled()
     return fn;
 }
 
-template <int B, bool kBF16>
+template <int B, bool kBF16, int NH>
 cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_t stream)
 {
-    auto kernel = quantize_keys_tc_kernel<B, kBF16>;
-    const size_t smem = 1024 + kStages * kABytes + kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem);
+    constexpr int D = kD * NH;
+    auto kernel = quantize_keys_tc_kernel<B, kBF16, NH>;
+    const size_t smem = 1024 + kStages * kABytes + NH * kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem);
+    static_assert(1024 + kStages * kABytes + NH * kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem) <= 232448,
+                  "shared memory per block");
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -391,8 +477,8 @@ cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_
     TcParams p{};
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return cudaErrorNotSupported;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(a.n)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(a.n)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
     const cuuint32_t box[2] = {64, kTileRows};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&p.tmap, kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
@@ -407,7 +493,7 @@ cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_
     p.ntiles = static_cast<int>((a.n + kTileRows - 1) / kTileRows);
     p.g_scale = tab.g_scale;
     p.g_off = tab.g_off;
-    p.inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(kD));
+    p.inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
     p.nt = tab.nt;
     for (int j = 0; j < kMaxBuckets; ++j) {
         p.tau[j] = tab.tau[j];
@@ -418,22 +504,29 @@ cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_
     return cudaGetLastError();
 }
 
-template <bool kBF16>
+template <bool kBF16, int NH>
 cudaError_t launch_typed(const QuantizeArgs &a, const BucketTable &tab, cudaStream_t stream)
 {
     switch (a.b) {
-    case 1: return launch_tc<1, kBF16>(a, tab, stream);
-    case 2: return launch_tc<2, kBF16>(a, tab, stream);
-    case 3: return launch_tc<3, kBF16>(a, tab, stream);
-    default: return launch_tc<4, kBF16>(a, tab, stream);
+    case 1: return launch_tc<1, kBF16, NH>(a, tab, stream);
+    case 2: return launch_tc<2, kBF16, NH>(a, tab, stream);
+    case 3: return launch_tc<3, kBF16, NH>(a, tab, stream);
+    default: return launch_tc<4, kBF16, NH>(a, tab, stream);
     }
+}
+
+template <int NH>
+cudaError_t launch_width(const QuantizeArgs &a, const BucketTable &tab, cudaStream_t stream)
+{
+    return a.kdtype == AXR_BF16 ? launch_typed<true, NH>(a, tab, stream) : launch_typed<false, NH>(a, tab, stream);
 }
 
 }  // namespace
 
 bool quantize_tc_supported(const QuantizeArgs &a)
 {
-    return a.d == kD && (a.kdtype == AXR_BF16 || a.kdtype == AXR_F16) && a.n > 0 && a.out_stride == 1 &&
+    return (a.d == kD || a.d == 2 * kD) && (a.kdtype == AXR_BF16 || a.kdtype == AXR_F16) && a.n > 0 &&
+           a.out_stride == 1 &&
            a.out_offset == 0 &&
            a.n <= static_cast<int64_t>(0x7fffffff) - kTileRows && encode_tiled() != nullptr;
 }
@@ -442,7 +535,7 @@ cudaError_t launch_quantize_keys_tc(const QuantizeArgs &a, cudaStream_t stream)
 {
     BucketTable tab;
     if (!get_bucket_table(a.d, a.b, &tab)) return cudaErrorInvalidValue;
-    return a.kdtype == AXR_BF16 ? launch_typed<true>(a, tab, stream) : launch_typed<false>(a, tab, stream);
+    return a.d == 2 * kD ? launch_width<2>(a, tab, stream) : launch_width<1>(a, tab, stream);
 }
 
 unsigned int quantize_tc_status(bool clear)

@@ -54,7 +54,14 @@ constexpr int kThreads = (kEpiWarps + 2) * 32;
 // d = 128 * NH: a tile's keys arrive as NH stages of 128 coordinates, and each
 // 128-key tile has NH accumulators of 128 columns (two tiles in flight)
 template <int NH>
-__host__ __device__ constexpr int tmem_cols() { return 256 * NH; }
+__host__ __device__ constexpr int tmem_cols() { return NH == 4 ? 512 : 256 * NH; }
+// d = 512 fills tensor memory with one tile's four accumulators (single buffered,
+// drained by all epilogue warps together) and shared memory with its four B
+// matrices, which leaves room for two stages
+template <int NH>
+__host__ __device__ constexpr int stages() { return NH == 4 ? 2 : kStages; }
+template <int NH>
+__host__ __device__ constexpr int acc_bufs() { return NH == 4 ? 1 : 2; }
 constexpr int kWarpTma = kEpiWarps, kWarpMma = kEpiWarps + 1;
 constexpr uint32_t kMagicBits = 0x4B400000u;    // bits of 1.5 * 2^23
 constexpr float kMagic = 12582912.0f;
@@ -129,6 +136,51 @@ __device__ __forceinline__ void quantize_chunk(const uint32_t (&v)[32], float2 a
     }
 }
 
+// y_q = sum_l (-1)^popcount(q & l) z_l (Sylvester H_4) for columns e, e + 1 of
+// the four accumulators' pieces z[l][0 .. 7]
+__device__ __forceinline__ void h4(const uint32_t (&z)[4][8], int e, float2 (&y)[4])
+{
+    const float2 m1 = make_float2(-1.0f, -1.0f);
+    const float2 z0 = make_float2(__uint_as_float(z[0][e]), __uint_as_float(z[0][e + 1]));
+    const float2 z1 = make_float2(__uint_as_float(z[1][e]), __uint_as_float(z[1][e + 1]));
+    const float2 z2 = make_float2(__uint_as_float(z[2][e]), __uint_as_float(z[2][e + 1]));
+    const float2 z3 = make_float2(__uint_as_float(z[3][e]), __uint_as_float(z[3][e + 1]));
+    const float2 s01 = __fadd2_rn(z0, z1), d01 = __ffma2_rn(z1, m1, z0);
+    const float2 s23 = __fadd2_rn(z2, z3), d23 = __ffma2_rn(z3, m1, z2);
+    y[0] = __fadd2_rn(s01, s23);
+    y[1] = __fadd2_rn(d01, d23);
+    y[2] = __ffma2_rn(s23, m1, s01);
+    y[3] = __ffma2_rn(d23, m1, d01);
+}
+
+// codes of 8 coordinates held in v[24 .. 31] at positions 8 pc .. 8 pc + 7 of a
+// 32-coordinate run (quantize_chunk on the top quarter of v, offset back by 24)
+template <int B, bool kClamp>
+__device__ __forceinline__ void quantize_piece(int pc, const uint32_t (&v)[32], float2 a2, float2 goff2,
+                                               float2 offm2, uint32_t tab, uint32_t bias, uint32_t *w)
+{
+    switch (pc) {
+    case 0: quantize_chunk<B, -24, 24, kClamp>(v, a2, goff2, offm2, tab, bias, w); break;
+    case 1: quantize_chunk<B, -16, 24, kClamp>(v, a2, goff2, offm2, tab, bias, w); break;
+    case 2: quantize_chunk<B, -8, 24, kClamp>(v, a2, goff2, offm2, tab, bias, w); break;
+    default: quantize_chunk<B, 0, 24, kClamp>(v, a2, goff2, offm2, tab, bias, w); break;
+    }
+}
+
+// NWQ packed words (32 coordinates) to global memory, streaming
+template <int NWQ>
+__device__ __forceinline__ void store_words(uint8_t *dst, const uint32_t *w)
+{
+    if constexpr (NWQ == 4) {
+        __stcs(reinterpret_cast<uint4 *>(dst), make_uint4(w[0], w[1], w[2], w[3]));
+    } else if constexpr (NWQ == 2) {
+        __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(w[0], w[1]));
+    } else {
+#pragma unroll
+        for (int i = 0; i < NWQ; ++i) __stcs(reinterpret_cast<unsigned int *>(dst) + i, w[i]);
+    }
+}
+
 // one run of NWH packed words (64 coordinates), 16- or 8-byte streaming stores
 template <int NWH>
 __device__ __forceinline__ void store_run(uint8_t *dst, const uint32_t *w)
@@ -148,13 +200,14 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
 {
     constexpr int D = kD * NH;
     constexpr int kTmemCols = tmem_cols<NH>();
+    constexpr int kSt = stages<NH>();
     constexpr int P = D * B / 8;             // packed bytes per key
     constexpr int NW = kD * B / 8 / 4;       // packed 32-bit words per 128 coordinates
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
     uint8_t *sA = base;                                      // kStages x 32 KB
-    uint8_t *sB = sA + kStages * kABytes;                    // NH x 32 KB
+    uint8_t *sB = sA + kSt * kABytes;                        // NH x 32 KB
     float2 *sTab = reinterpret_cast<float2 *>(sB + NH * kBBytes); // kMaxBuckets entries
     Smem &S = *reinterpret_cast<Smem *>(sTab + kMaxBuckets);
 
@@ -168,11 +221,12 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&S.acc_full[a]), 1);
-            mbar_init(smem_u32(&S.acc_empty[a]), kGroupWarps * 32);   // the group that drains it
+            // the group that drains it (d <= 256), or all epilogue warps (d = 512)
+            mbar_init(smem_u32(&S.acc_empty[a]), (NH == 4 ? kEpiWarps : kGroupWarps) * 32);
         }
         mbar_init(smem_u32(&S.drain), 1);
         for (int a = 0; a < 2; ++a)
-            for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&S.pair[a][q]), 64);   // two warps
+            for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&S.pair[a][q]), NH == 4 ? 128 : 64);   // warps of a quadrant
         fence_mbar_init();
     }
     if (warp == kWarpTma && lane == 0) prefetch_tensormap(&p.tmap);
@@ -223,8 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             bool stop = false;
             for (int t = blockIdx.x; t < p.ntiles && !stop; t += gridDim.x) {
                 for (int l = 0; l < NH; ++l, ++it) {         // one stage per 128 coordinates
-                    const int s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1;
+                    const int s = it % kSt;
+                    const uint32_t ph = (it / kSt) & 1;
                     if (!mbar_wait(smem_u32(&S.empty[s]), ph ^ 1)) {
                         atomicOr(&g_status, kErrTimeoutMma);
                         stop = true;
@@ -237,9 +291,9 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                 }
             }
             // let every load this thread issued land before the CTA exits
-            for (int k = 0; k < kStages && k < it; ++k) {
+            for (int k = 0; k < kSt && k < it; ++k) {
                 const int j = it - 1 - k;
-                mbar_wait(smem_u32(&S.full[j % kStages]), (j / kStages) & 1);
+                mbar_wait(smem_u32(&S.full[j % kSt]), (j / kSt) & 1);
             }
         }
     } else if (warp == kWarpMma) {
@@ -250,15 +304,15 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             int it = 0, st = 0;                               // tiles, stages
             bool stop = false;
             for (int t = blockIdx.x; t < p.ntiles && !stop; t += gridDim.x, ++it) {
-                const int acc = it & 1;
-                const uint32_t aph = (it >> 1) & 1;
+                const int acc = (acc_bufs<NH>() == 1) ? 0 : (it & 1);
+                const uint32_t aph = (acc_bufs<NH>() == 1) ? (it & 1) : ((it >> 1) & 1);
                 if (!mbar_wait(smem_u32(&S.acc_empty[acc]), aph ^ 1)) {
                     atomicOr(&g_status, kErrTimeoutDrain);
                     break;
                 }
                 for (int l = 0; l < NH; ++l, ++st) {
-                    const int s = st % kStages;
-                    const uint32_t ph = (st / kStages) & 1;
+                    const int s = st % kSt;
+                    const uint32_t ph = (st / kSt) & 1;
                     if (!mbar_wait(smem_u32(&S.full[s]), ph)) {
                         atomicOr(&g_status, kErrTimeoutLoad);
                         stop = true;
@@ -284,6 +338,110 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         }
     } else {
         // ---------------------------------------------------------- epilogue
+      if constexpr (NH == 4) {
+        // d = 512: y = (H_4 (x) H) diag(s) k, so y_q = sum_l (-1)^popcount(q & l) z_l over
+        // the four accumulators z_l = B_l k_l.  All 16 warps drain each tile: lane
+        // quadrant `quad`, 32-column quarter `cq` of every z_l, 8 columns at a time.
+        constexpr int NWQ = B;                       // packed words of 32 coordinates
+        const int quad = warp & 3, cq = warp >> 2;
+        const uint32_t col0 = tmem + (static_cast<uint32_t>(quad * 32) << 16) + cq * 32;
+        const int key = quad * 32 + lane;
+        float *ss4 = &S.ss[0][0][0];                 // [quarter][key]
+        constexpr uint32_t kCentral = (1u << (B - 1)) - 1u;
+        const uint32_t tab_u32 = smem_u32(sTab);
+        const uint32_t tab_bias = tab_u32 - kMagicBits * 8u;     // wraps mod 2^32 by design
+        int it = 0;
+        for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
+            const uint32_t aph = it & 1;
+            if (!mbar_wait_warp(smem_u32(&S.acc_full[0]), aph)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                break;
+            }
+            tc_fence_after_sync();
+            // pass 1: this quarter's sum of y^2 over the four outputs
+            float2 p01 = make_float2(0.0f, 0.0f), p23 = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int pc = 0; pc < 4; ++pc) {
+                uint32_t z[4][8];
+#pragma unroll
+                for (int l = 0; l < 4; ++l) tmem_ld8(col0 + l * kD + 8 * pc, z[l]);
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    float2 y[4];
+                    h4(z, e, y);
+                    p01 = __ffma2_rn(y[0], y[0], p01);
+                    p01 = __ffma2_rn(y[1], y[1], p01);
+                    p23 = __ffma2_rn(y[2], y[2], p23);
+                    p23 = __ffma2_rn(y[3], y[3], p23);
+                }
+            }
+            ss4[cq * kTileRows + key] = (p01.x + p01.y) + (p23.x + p23.y);
+            mbar_arrive(smem_u32(&S.pair[0][quad]));
+            if (!mbar_wait_warp(smem_u32(&S.pair[0][quad]), aph)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                break;
+            }
+            const float ss = (ss4[key] + ss4[kTileRows + key]) + (ss4[2 * kTileRows + key] + ss4[3 * kTileRows + key]);
+            const float norm = sqrtf(ss) * p.inv_sqrt_d;
+            const bool finite = ss <= 3.402823466e38f;
+            const bool clamp = !(ss >= 1e-36f);
+            const float a = (finite && ss > 0.0f) ? p.g_scale / sqrtf(ss) : 0.0f;
+            const float2 a2 = make_float2(a, a);
+            const float2 goff2 = make_float2(p.g_off, p.g_off);
+            const float2 offm2 = make_float2(p.g_off + kMagic, p.g_off + kMagic);
+            uint32_t w[4][NWQ + 1];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int i = 0; i <= NWQ; ++i) w[q][i] = 0;
+            // pass 2: codes of y_q at coordinates 128 q + 32 cq + (8 pc .. 8 pc + 7)
+#pragma unroll
+            for (int pc = 0; pc < 4; ++pc) {
+                uint32_t z[4][8];
+#pragma unroll
+                for (int l = 0; l < 4; ++l) tmem_ld8(col0 + l * kD + 8 * pc, z[l]);
+                uint32_t v[4][32];                   // y_q in v[q][24 .. 31]
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    float2 y[4];
+                    h4(z, e, y);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        v[q][24 + e] = __float_as_uint(y[q].x);
+                        v[q][25 + e] = __float_as_uint(y[q].y);
+                    }
+                }
+                if (pc == 3) {                       // every read of this tile's accumulators done
+                    tc_fence_before_sync();
+                    mbar_arrive(smem_u32(&S.acc_empty[0]));
+                }
+                if (finite) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (!clamp) quantize_piece<B, false>(pc, v[q], a2, goff2, offm2, tab_u32, tab_bias, w[q]);
+                        else quantize_piece<B, true>(pc, v[q], a2, goff2, offm2, tab_u32, tab_bias, w[q]);
+                    }
+                }
+            }
+            if (!finite) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int o = j * B;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        w[q][o >> 5] |= kCentral << (o & 31);
+                        if ((o & 31) + B > 32) w[q][(o >> 5) + 1] |= kCentral >> (32 - (o & 31));
+                    }
+                }
+            }
+            const int64_t row = static_cast<int64_t>(t) * kTileRows + key;
+            if (row < p.n) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) store_words<NWQ>(p.idx + row * P + (4 * q + cq) * NWQ * 4, w[q]);
+                if (cq == 0) __stcs(p.norms + row, norm);
+            }
+        }
+      } else {
         constexpr int kHalfCols = kD / 2;
         constexpr int NWH = NW / 2;                  // packed words per half row
         // group e drains accumulator e: the CTA's tiles 2m + e, so two tiles are
@@ -429,6 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                 if (half == 0) __stcs(p.norms + row, norm);
             }
         }
+      }
     }
 
     tc_fence_before_sync();
@@ -464,8 +623,8 @@ cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_
 {
     constexpr int D = kD * NH;
     auto kernel = quantize_keys_tc_kernel<B, kBF16, NH>;
-    const size_t smem = 1024 + kStages * kABytes + NH * kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem);
-    static_assert(1024 + kStages * kABytes + NH * kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem) <= 232448,
+    const size_t smem = 1024 + stages<NH>() * kABytes + NH * kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem);
+    static_assert(1024 + stages<NH>() * kABytes + NH * kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem) <= 232448,
                   "shared memory per block");
     static bool configured = false;
     if (!configured) {
@@ -525,7 +684,8 @@ cudaError_t launch_width(const QuantizeArgs &a, const BucketTable &tab, cudaStre
 
 bool quantize_tc_supported(const QuantizeArgs &a)
 {
-    return (a.d == kD || a.d == 2 * kD) && (a.kdtype == AXR_BF16 || a.kdtype == AXR_F16) && a.n > 0 &&
+    return (a.d == kD || a.d == 2 * kD || a.d == 4 * kD) && (a.kdtype == AXR_BF16 || a.kdtype == AXR_F16) &&
+           a.n > 0 &&
            a.out_stride == 1 &&
            a.out_offset == 0 &&
            a.n <= static_cast<int64_t>(0x7fffffff) - kTileRows && encode_tiled() != nullptr;
@@ -535,7 +695,11 @@ cudaError_t launch_quantize_keys_tc(const QuantizeArgs &a, cudaStream_t stream)
 {
     BucketTable tab;
     if (!get_bucket_table(a.d, a.b, &tab)) return cudaErrorInvalidValue;
-    return a.d == 2 * kD ? launch_width<2>(a, tab, stream) : launch_width<1>(a, tab, stream);
+    switch (a.d) {
+    case 2 * kD: return launch_width<2>(a, tab, stream);
+    case 4 * kD: return launch_width<4>(a, tab, stream);
+    default: return launch_width<1>(a, tab, stream);
+    }
 }
 
 unsigned int quantize_tc_status(bool clear)

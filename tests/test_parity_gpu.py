@@ -98,6 +98,40 @@ def test_scores_tile_ranges_cross_heads(heads, n, group, b):
     assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
 
 
+@pytest.mark.parametrize("d,b,heads,n,group", [
+    (256, 2, 40, 300, 4), (256, 4, 200, 77, 8), (256, 3, 30, 1000, 1), (256, 1, 64, 129, 3),
+    (512, 2, 40, 300, 4), (512, 4, 150, 77, 8), (512, 3, 20, 700, 2), (512, 1, 300, 64, 5),
+])
+def test_scores_wide_heads_cross_heads(d, b, heads, n, group):
+    """d = 256 and 512 run on the tensor-core kernel as 2 and 4 subtiles per tile,
+    with one B buffer per tile stream: a stream entering a new KV head waits for
+    its products on the last head before writing the new query digits.  Many
+    short heads make every CTA cross heads many times (n < 128: every tile a
+    head of its own), for G up to 8 (one stream per CTA at d = 512)."""
+    packed, norms = workloads.make_random_packed(heads, n, d, b, seed=heads + n + b + d, device=DEV)
+    wl = workloads.GQA_DECODE_128K.with_(d=d, batch=1, kv_heads=heads, group=group, T=n)
+    q = workloads.make_queries(wl, DEV)
+    s = workloads.make_signs(wl).to(DEV)
+    out = gpu_scores(q, packed, norms, group, b, s)
+    assert check_scores(q, packed, norms, out, group, b, s) <= 1e-4
+
+
+@pytest.mark.parametrize("d", [256, 512])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("n", [1, 127, 129, 1000])
+def test_quantize_wide_heads_tensor_core_tails(d, dtype, n):
+    """The d = 256 / 512 tensor-core write on partial tiles (the TMA zero-fills the
+    rows past n, the epilogue drops them).  Every code flip must lie inside the
+    boundary window; the in-window flip rate is not capped here, since a few
+    hundred rows hold too few coordinates for a rate of 1e-5 to mean anything
+    (the full-size sampled tests check it)."""
+    K, s = _keys(d, dtype, n, seed=9000 + d + n)
+    for b in (2, 3):
+        idx, norms = gpu_quantize(K, b, s)
+        rep = check_quantize(K, idx, norms, b, s)
+        assert rep.ok(flip_fraction=None), f"d={d} b={b} {dtype} n={n}: {rep}"
+
+
 @pytest.mark.parametrize("offset", [0, 1, 2, 3])
 def test_scores_norms_at_any_4_byte_offset(offset):
     """The tensor-core read kernel loads key norms by TMA from the 16-byte boundary

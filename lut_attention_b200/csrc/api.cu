@@ -319,7 +319,9 @@ extern "C" int axr_quantize_keys_block(const void *K, int kdtype, int64_t n, int
     QuantizeArgs a{K, kdtype, n, d, b, nullptr, idx, norms, Codebook{}};
     a.quats = quats;
     if (!get_codebook(d, b, &a.cb)) return fail(AXR_EUNSUPPORTED, "no codebook for d=%d b=%d", d, b);
-    const cudaError_t e = launch_quantize_keys_block(a, reinterpret_cast<cudaStream_t>(stream));
+    // bf16/fp16 keys of d = 128, 256, 512 on the tensor cores, the rest on CUDA cores
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = quantize_tc_supported(a) ? launch_quantize_keys_tc(a, st) : launch_quantize_keys_block(a, st);
     if (e != cudaSuccess) return fail(AXR_ECUDA, "block-rotation quantize launch: %s", cudaGetErrorString(e));
     return ok();
 }

@@ -90,7 +90,8 @@ cudaError_t launch_quantize_keys(const QuantizeArgs &a, cudaStream_t stream);
 // Write path with the block rotation (quantize_keys_block.cu): every d, dense output.
 cudaError_t launch_quantize_keys_block(const QuantizeArgs &a, cudaStream_t stream);
 
-// Tensor-core write path (quantize_keys_tc.cu): d = 128, bf16/fp16 keys.
+// Tensor-core write path (quantize_keys_tc.cu): d = 128, 256, 512, bf16/fp16 keys,
+// with the Walsh-Hadamard transform or (quats set) the block rotation.
 bool quantize_tc_supported(const QuantizeArgs &a);
 cudaError_t launch_quantize_keys_tc(const QuantizeArgs &a, cudaStream_t stream);
 unsigned int quantize_tc_status(bool clear);

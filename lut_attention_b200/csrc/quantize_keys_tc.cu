@@ -35,6 +35,7 @@
 #include <cuda_runtime.h>
 
 #include "axr_internal.cuh"
+#include "quat.cuh"
 #include "sm100.cuh"
 
 namespace axr {
@@ -73,6 +74,7 @@ struct TcParams {
     uint8_t *idx;
     float *norms;
     const int8_t *signs;
+    const float *quats;            // block rotation (d/4 x 8 floats) in place of the signs, or null
     int64_t n;
     int ntiles;
     float g_scale;
@@ -122,22 +124,28 @@ __device__ __forceinline__ void place_code(float g, float f, uint32_t tab, uint3
 // Quantize coordinates C0 + E, C0 + E + 1 (two at a time: one paired FMA gives
 // both bucket values g = y a + g_off, one more both f = y a + g_off + 1.5 * 2^23,
 // rounded exactly as two scalar FMAs would be).
+// The value compared with the bucket's threshold is g = y ag + goff: the bucket
+// value itself (ag = a, goff = g_off; thresholds in bucket units), or the unit
+// coordinate u (ag = 1 / |y|, goff = 0; thresholds in u units, the
+// block-rotation path), one paired FMA either way.
 template <int B, int C0, int E, bool kClamp>
-__device__ __forceinline__ void quantize_chunk(const uint32_t (&v)[32], float2 a2, float2 goff2, float2 offm2,
-                                               uint32_t tab, uint32_t bias, uint32_t *w)
+__device__ __forceinline__ void quantize_chunk(const uint32_t (&v)[32], float2 ag2, float2 goff2, float2 a2,
+                                               float2 offm2, uint32_t tab, uint32_t bias, uint32_t *w)
 {
     if constexpr (E < 32) {
         const float2 y = make_float2(__uint_as_float(v[E]), __uint_as_float(v[E + 1]));
-        const float2 g = __ffma2_rn(y, a2, goff2);
+        const float2 g = __ffma2_rn(y, ag2, goff2);
         const float2 f = __ffma2_rn(y, a2, offm2);
         place_code<B, (C0 + E) * B, kClamp>(g.x, f.x, tab, bias, w);
         place_code<B, (C0 + E + 1) * B, kClamp>(g.y, f.y, tab, bias, w);
-        quantize_chunk<B, C0, E + 2, kClamp>(v, a2, goff2, offm2, tab, bias, w);
+        quantize_chunk<B, C0, E + 2, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w);
     }
 }
 
 // y_q = sum_l (-1)^popcount(q & l) z_l (Sylvester H_4) for columns e, e + 1 of
 // the four accumulators' pieces z[l][0 .. 7]
+// (kIdentity: the block rotation, whose slices do not mix: y_q = z_q)
+template <bool kIdentity>
 __device__ __forceinline__ void h4(const uint32_t (&z)[4][8], int e, float2 (&y)[4])
 {
     const float2 m1 = make_float2(-1.0f, -1.0f);
@@ -145,6 +153,13 @@ __device__ __forceinline__ void h4(const uint32_t (&z)[4][8], int e, float2 (&y)
     const float2 z1 = make_float2(__uint_as_float(z[1][e]), __uint_as_float(z[1][e + 1]));
     const float2 z2 = make_float2(__uint_as_float(z[2][e]), __uint_as_float(z[2][e + 1]));
     const float2 z3 = make_float2(__uint_as_float(z[3][e]), __uint_as_float(z[3][e + 1]));
+    if constexpr (kIdentity) {
+        y[0] = z0;
+        y[1] = z1;
+        y[2] = z2;
+        y[3] = z3;
+        return;
+    }
     const float2 s01 = __fadd2_rn(z0, z1), d01 = __ffma2_rn(z1, m1, z0);
     const float2 s23 = __fadd2_rn(z2, z3), d23 = __ffma2_rn(z3, m1, z2);
     y[0] = __fadd2_rn(s01, s23);
@@ -156,14 +171,14 @@ __device__ __forceinline__ void h4(const uint32_t (&z)[4][8], int e, float2 (&y)
 // codes of 8 coordinates held in v[24 .. 31] at positions 8 pc .. 8 pc + 7 of a
 // 32-coordinate run (quantize_chunk on the top quarter of v, offset back by 24)
 template <int B, bool kClamp>
-__device__ __forceinline__ void quantize_piece(int pc, const uint32_t (&v)[32], float2 a2, float2 goff2,
+__device__ __forceinline__ void quantize_piece(int pc, const uint32_t (&v)[32], float2 ag2, float2 goff2, float2 a2,
                                                float2 offm2, uint32_t tab, uint32_t bias, uint32_t *w)
 {
     switch (pc) {
-    case 0: quantize_chunk<B, -24, 24, kClamp>(v, a2, goff2, offm2, tab, bias, w); break;
-    case 1: quantize_chunk<B, -16, 24, kClamp>(v, a2, goff2, offm2, tab, bias, w); break;
-    case 2: quantize_chunk<B, -8, 24, kClamp>(v, a2, goff2, offm2, tab, bias, w); break;
-    default: quantize_chunk<B, 0, 24, kClamp>(v, a2, goff2, offm2, tab, bias, w); break;
+    case 0: quantize_chunk<B, -24, 24, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w); break;
+    case 1: quantize_chunk<B, -16, 24, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w); break;
+    case 2: quantize_chunk<B, -8, 24, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w); break;
+    default: quantize_chunk<B, 0, 24, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w); break;
     }
 }
 
@@ -181,6 +196,39 @@ __device__ __forceinline__ void store_words(uint8_t *dst, const uint32_t *w)
     }
 }
 
+// Block rotation (IsoQuant, arXiv 2603.28430, abstract: 4-element blocks v turn
+// into qL v conj(qR)).  T is block diagonal, so each 16-coordinate group of a
+// 128-coordinate slice only mixes within itself: output columns 16 j .. 16 j + 15
+// of z_l are one M = 128, N = 16, K = 16 product of the keys' columns 16 j ..
+// with the group's 16 x 16 piece of T.  Those pieces are fp32; they enter the
+// tensor cores as kParts terms in the key type (bf16: 3 terms, 24 bits; fp16:
+// 2 terms, 22 bits), each product of a bf16/fp16 key with a term is exact, and
+// fp32 accumulation adds them, so y = T k comes out at fp32 accuracy.
+template <bool kBF16>
+__host__ __device__ constexpr int block_parts() { return kBF16 ? 3 : 2; }
+constexpr int kBlkBytes = 16 * 16 * 2;           // one 16 x 16 piece, no swizzle (core matrices)
+
+// byte offset of element (n = output, k = input) in a 16 x 16 K-major piece:
+// 8 x 8-element core matrices, K-adjacent ones 128 bytes apart, N-adjacent 256
+__device__ __forceinline__ int blk_offset(int n, int k)
+{
+    return ((n >> 3) * 2 + (k >> 3)) * 128 + (n & 7) * 16 + (k & 7) * 2;
+}
+
+template <bool kBF16>
+__device__ __forceinline__ uint16_t to_half_bits(float v, float &back)
+{
+    if constexpr (kBF16) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        back = __bfloat162float(h);
+        return __bfloat16_as_ushort(h);
+    } else {
+        const __half h = __float2half_rn(v);
+        back = __half2float(h);
+        return __half_as_ushort(h);
+    }
+}
+
 // one run of NWH packed words (64 coordinates), 16- or 8-byte streaming stores
 template <int NWH>
 __device__ __forceinline__ void store_run(uint8_t *dst, const uint32_t *w)
@@ -195,9 +243,11 @@ __device__ __forceinline__ void store_run(uint8_t *dst, const uint32_t *w)
     }
 }
 
-template <int B, bool kBF16, int NH>
+template <int B, bool kBF16, int NH, bool kBlock>
 __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __grid_constant__ TcParams p)
 {
+    constexpr int kParts = block_parts<kBF16>();
+    constexpr int kBRegion = kBlock ? kParts * NH * 8 * kBlkBytes : NH * kBBytes;
     constexpr int D = kD * NH;
     constexpr int kTmemCols = tmem_cols<NH>();
     constexpr int kSt = stages<NH>();
@@ -208,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
     uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
     uint8_t *sA = base;                                      // kStages x 32 KB
     uint8_t *sB = sA + kSt * kABytes;                        // NH x 32 KB
-    float2 *sTab = reinterpret_cast<float2 *>(sB + NH * kBBytes); // kMaxBuckets entries
+    float2 *sTab = reinterpret_cast<float2 *>(sB + kBRegion);     // kMaxBuckets entries
     Smem &S = *reinterpret_cast<Smem *>(sTab + kMaxBuckets);
 
     const int warp = threadIdx.x >> 5;
@@ -236,6 +286,30 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
     // of 128-byte swizzled rows (the layout TMA gives A).  For d = 256 the
     // Sylvester recursion H_256 = [[H, H], [H, -H]] gives y = (z_0 + z_1, z_0 - z_1)
     // with z_l = B_l k_l, which the epilogue forms.
+    if constexpr (kBlock) {
+        // piece (part, slice l, group j) at ((part * NH + l) * 8 + j) * kBlkBytes
+        for (int e = threadIdx.x; e < NH * 8 * 256; e += kThreads) {
+            const int l = e / (8 * 256), j = (e / 256) % 8, n = (e / 16) % 16, k = e % 16;
+            float v = 0.0f;
+            if ((n >> 2) == (k >> 2)) {
+                Quat qL, qRc;
+                block_quats(p.quats, 32 * l + 4 * j + (n >> 2), qL, qRc);
+                const int c = k & 3;
+                const Quat y = block_rotate(qL, qRc, {c == 0 ? 1.0f : 0.0f, c == 1 ? 1.0f : 0.0f,
+                                                      c == 2 ? 1.0f : 0.0f, c == 3 ? 1.0f : 0.0f});
+                const int r = n & 3;
+                v = r == 0 ? y.w : r == 1 ? y.x : r == 2 ? y.y : y.z;
+            }
+            float rest = v;
+#pragma unroll
+            for (int part = 0; part < kParts; ++part) {
+                float back;
+                const uint16_t bits = to_half_bits<kBF16>(rest, back);
+                rest -= back;
+                *reinterpret_cast<uint16_t *>(sB + ((part * NH + l) * 8 + j) * kBlkBytes + blk_offset(n, k)) = bits;
+            }
+        }
+    } else
     for (int chunk = threadIdx.x; chunk < NH * kD * (kD / 8); chunk += kThreads) {
         const int l = chunk / (kD * (kD / 8));
         const int n = (chunk / (kD / 8)) % kD;
@@ -300,6 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         // --------------------------------------------------------------- MMA
         if (lane == 0) {
             const uint32_t id = idesc(kAccF32, kBF16 ? kFmtBF16 : kFmtF16, kBF16 ? kFmtBF16 : kFmtF16, 128, kD);
+            const uint32_t id16 = idesc(kAccF32, kBF16 ? kFmtBF16 : kFmtF16, kBF16 ? kFmtBF16 : kFmtF16, 128, 16);
             const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
             int it = 0, st = 0;                               // tiles, stages
             bool stop = false;
@@ -321,11 +396,26 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                     tc_fence_after_sync();
                     // accumulator acc holds z_0 .. z_{NH-1}, 128 columns each
                     const uint32_t d = tmem + (acc * NH + l) * kD;
+                    if constexpr (kBlock) {
+                        // 16 output columns per group, from the group's 16 key columns
+                        // and the kParts terms of its piece of T
 #pragma unroll
-                    for (int k = 0; k < kD / 16; ++k) {
-                        const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
-                        mma_f16_ss(d, desc_k_sw128(a0 + s * kABytes + off), desc_k_sw128(b0 + l * kBBytes + off), id,
-                                   k > 0);
+                        for (int k = 0; k < kD / 16; ++k) {
+                            const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
+                            const uint64_t ad = desc_k_sw128(a0 + s * kABytes + off);
+#pragma unroll
+                            for (int part = 0; part < kParts; ++part)
+                                mma_f16_ss(d + 16 * k, ad,
+                                           desc_k_interleave(b0 + ((part * NH + l) * 8 + k) * kBlkBytes, 128, 256),
+                                           id16, part > 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < kD / 16; ++k) {
+                            const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
+                            mma_f16_ss(d, desc_k_sw128(a0 + s * kABytes + off), desc_k_sw128(b0 + l * kBBytes + off),
+                                       id, k > 0);
+                        }
                     }
                     mma_commit(smem_u32(&S.empty[s]));
                 }
@@ -368,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     float2 y[4];
-                    h4(z, e, y);
+                    h4<kBlock>(z, e, y);
                     p01 = __ffma2_rn(y[0], y[0], p01);
                     p01 = __ffma2_rn(y[1], y[1], p01);
                     p23 = __ffma2_rn(y[2], y[2], p23);
@@ -389,6 +479,10 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const float2 a2 = make_float2(a, a);
             const float2 goff2 = make_float2(p.g_off, p.g_off);
             const float2 offm2 = make_float2(p.g_off + kMagic, p.g_off + kMagic);
+            // the compared value: the bucket value, or u itself for the block rotation
+            const float ug = (finite && ss > 0.0f) ? 1.0f / sqrtf(ss) : 0.0f;
+            const float2 ag2 = kBlock ? make_float2(ug, ug) : a2;
+            const float2 gofs2 = kBlock ? make_float2(0.0f, 0.0f) : goff2;
             uint32_t w[4][NWQ + 1];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
@@ -404,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     float2 y[4];
-                    h4(z, e, y);
+                    h4<kBlock>(z, e, y);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         v[q][24 + e] = __float_as_uint(y[q].x);
@@ -418,8 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                 if (finite) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        if (!clamp) quantize_piece<B, false>(pc, v[q], a2, goff2, offm2, tab_u32, tab_bias, w[q]);
-                        else quantize_piece<B, true>(pc, v[q], a2, goff2, offm2, tab_u32, tab_bias, w[q]);
+                        if (!clamp) quantize_piece<B, false>(pc, v[q], ag2, gofs2, a2, offm2, tab_u32, tab_bias, w[q]);
+                        else quantize_piece<B, true>(pc, v[q], ag2, gofs2, a2, offm2, tab_u32, tab_bias, w[q]);
                     }
                 }
             }
@@ -488,8 +582,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                     for (int e = 0; e < 32; e += 2) {
                         const float2 z0 = make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
                         const float2 z1 = make_float2(__uint_as_float(v1[e]), __uint_as_float(v1[e + 1]));
-                        const float2 ya = __fadd2_rn(z0, z1);
-                        const float2 yb = __ffma2_rn(z1, make_float2(-1.0f, -1.0f), z0);
+                        const float2 ya = kBlock ? z0 : __fadd2_rn(z0, z1);
+                        const float2 yb = kBlock ? z1 : __ffma2_rn(z1, make_float2(-1.0f, -1.0f), z0);
                         p01 = __ffma2_rn(ya, ya, p01);
                         p23 = __ffma2_rn(yb, yb, p23);
                     }
@@ -518,14 +612,18 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const float2 a2 = make_float2(a, a);
             const float2 goff2 = make_float2(p.g_off, p.g_off);
             const float2 offm2 = make_float2(p.g_off + kMagic, p.g_off + kMagic);
+            // the compared value: the bucket value, or u itself for the block rotation
+            const float ug = (finite && ss > 0.0f) ? 1.0f / sqrtf(ss) : 0.0f;
+            const float2 ag2 = kBlock ? make_float2(ug, ug) : a2;
+            const float2 gofs2 = kBlock ? make_float2(0.0f, 0.0f) : goff2;
             if constexpr (NH == 1) {
                 uint32_t v[32];
                 tmem_ld32(col_addr, v);
-                if (finite && !clamp) quantize_chunk<B, 0, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
-                else if (finite) quantize_chunk<B, 0, 0, true>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
+                if (finite && !clamp) quantize_chunk<B, 0, 0, false>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 0, 0, true>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
                 tmem_ld32(col_addr + 32, v);
-                if (finite && !clamp) quantize_chunk<B, 32, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
-                else if (finite) quantize_chunk<B, 32, 0, true>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
+                if (finite && !clamp) quantize_chunk<B, 32, 0, false>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 32, 0, true>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
             } else {
 #pragma unroll
                 for (int c = 0; c < kHalfCols / 32; ++c) {
@@ -536,8 +634,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                     for (int e = 0; e < 32; e += 2) {
                         const float2 z0 = make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
                         const float2 z1 = make_float2(__uint_as_float(v1[e]), __uint_as_float(v1[e + 1]));
-                        const float2 ya = __fadd2_rn(z0, z1);
-                        const float2 yb = __ffma2_rn(z1, make_float2(-1.0f, -1.0f), z0);
+                        const float2 ya = kBlock ? z0 : __fadd2_rn(z0, z1);
+                        const float2 yb = kBlock ? z1 : __ffma2_rn(z1, make_float2(-1.0f, -1.0f), z0);
                         v[e] = __float_as_uint(ya.x);
                         v[e + 1] = __float_as_uint(ya.y);
                         v1[e] = __float_as_uint(yb.x);
@@ -545,19 +643,19 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                     }
                     if (c == 0) {
                         if (finite && !clamp) {
-                            quantize_chunk<B, 0, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
-                            quantize_chunk<B, 0, 0, false>(v1, a2, goff2, offm2, tab_u32, tab_bias, w1);
+                            quantize_chunk<B, 0, 0, false>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 0, 0, false>(v1, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w1);
                         } else if (finite) {
-                            quantize_chunk<B, 0, 0, true>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
-                            quantize_chunk<B, 0, 0, true>(v1, a2, goff2, offm2, tab_u32, tab_bias, w1);
+                            quantize_chunk<B, 0, 0, true>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 0, 0, true>(v1, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w1);
                         }
                     } else {
                         if (finite && !clamp) {
-                            quantize_chunk<B, 32, 0, false>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
-                            quantize_chunk<B, 32, 0, false>(v1, a2, goff2, offm2, tab_u32, tab_bias, w1);
+                            quantize_chunk<B, 32, 0, false>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 32, 0, false>(v1, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w1);
                         } else if (finite) {
-                            quantize_chunk<B, 32, 0, true>(v, a2, goff2, offm2, tab_u32, tab_bias, w);
-                            quantize_chunk<B, 32, 0, true>(v1, a2, goff2, offm2, tab_u32, tab_bias, w1);
+                            quantize_chunk<B, 32, 0, true>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 32, 0, true>(v1, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w1);
                         }
                     }
                 }
@@ -618,13 +716,14 @@ EncodeTiledFn encode_tiled()
     return fn;
 }
 
-template <int B, bool kBF16, int NH>
+template <int B, bool kBF16, int NH, bool kBlock>
 cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_t stream)
 {
     constexpr int D = kD * NH;
-    auto kernel = quantize_keys_tc_kernel<B, kBF16, NH>;
-    const size_t smem = 1024 + stages<NH>() * kABytes + NH * kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem);
-    static_assert(1024 + stages<NH>() * kABytes + NH * kBBytes + kMaxBuckets * sizeof(float2) + sizeof(Smem) <= 232448,
+    auto kernel = quantize_keys_tc_kernel<B, kBF16, NH, kBlock>;
+    constexpr size_t kBReg = kBlock ? block_parts<kBF16>() * NH * 8 * kBlkBytes : NH * kBBytes;
+    const size_t smem = 1024 + stages<NH>() * kABytes + kBReg + kMaxBuckets * sizeof(float2) + sizeof(Smem);
+    static_assert(1024 + stages<NH>() * kABytes + kBReg + kMaxBuckets * sizeof(float2) + sizeof(Smem) <= 232448,
                   "shared memory per block");
     static bool configured = false;
     if (!configured) {
@@ -652,10 +751,16 @@ cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_
     p.ntiles = static_cast<int>((a.n + kTileRows - 1) / kTileRows);
     p.g_scale = tab.g_scale;
     p.g_off = tab.g_off;
-    p.inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+    // |y|^2 = d |k|^2 for the unnormalised Walsh-Hadamard product, |k|^2 for the
+    // (orthonormal) block rotation
+    p.inv_sqrt_d = kBlock ? 1.0f : 1.0f / sqrtf(static_cast<float>(D));
+    p.quats = a.quats;
     p.nt = tab.nt;
+    // thresholds in bucket units, or (block rotation, which compares u itself) the
+    // codebook boundary each bucket holds, in u units
     for (int j = 0; j < kMaxBuckets; ++j) {
-        p.tau[j] = tab.tau[j];
+        const bool has = j < tab.nt && tab.tau[j] < INFINITY;
+        p.tau[j] = kBlock ? (has ? a.cb.boundaries[tab.base[j]] : INFINITY) : tab.tau[j];
         p.base[j] = tab.base[j];
     }
     const int grid = p.ntiles < device_sm_count() ? p.ntiles : device_sm_count();
@@ -663,21 +768,32 @@ cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_
     return cudaGetLastError();
 }
 
-template <bool kBF16, int NH>
+template <bool kBF16, int NH, bool kBlock>
 cudaError_t launch_typed(const QuantizeArgs &a, const BucketTable &tab, cudaStream_t stream)
 {
     switch (a.b) {
-    case 1: return launch_tc<1, kBF16, NH>(a, tab, stream);
-    case 2: return launch_tc<2, kBF16, NH>(a, tab, stream);
-    case 3: return launch_tc<3, kBF16, NH>(a, tab, stream);
-    default: return launch_tc<4, kBF16, NH>(a, tab, stream);
+    case 1: return launch_tc<1, kBF16, NH, kBlock>(a, tab, stream);
+    case 2: return launch_tc<2, kBF16, NH, kBlock>(a, tab, stream);
+    case 3: return launch_tc<3, kBF16, NH, kBlock>(a, tab, stream);
+    default: return launch_tc<4, kBF16, NH, kBlock>(a, tab, stream);
     }
 }
 
-template <int NH>
+template <int NH, bool kBlock>
 cudaError_t launch_width(const QuantizeArgs &a, const BucketTable &tab, cudaStream_t stream)
 {
-    return a.kdtype == AXR_BF16 ? launch_typed<true, NH>(a, tab, stream) : launch_typed<false, NH>(a, tab, stream);
+    return a.kdtype == AXR_BF16 ? launch_typed<true, NH, kBlock>(a, tab, stream)
+                                : launch_typed<false, NH, kBlock>(a, tab, stream);
+}
+
+template <bool kBlock>
+cudaError_t launch_transform(const QuantizeArgs &a, const BucketTable &tab, cudaStream_t stream)
+{
+    switch (a.d) {
+    case 2 * kD: return launch_width<2, kBlock>(a, tab, stream);
+    case 4 * kD: return launch_width<4, kBlock>(a, tab, stream);
+    default: return launch_width<1, kBlock>(a, tab, stream);
+    }
 }
 
 }  // namespace
@@ -695,11 +811,7 @@ cudaError_t launch_quantize_keys_tc(const QuantizeArgs &a, cudaStream_t stream)
 {
     BucketTable tab;
     if (!get_bucket_table(a.d, a.b, &tab)) return cudaErrorInvalidValue;
-    switch (a.d) {
-    case 2 * kD: return launch_width<2>(a, tab, stream);
-    case 4 * kD: return launch_width<4>(a, tab, stream);
-    default: return launch_width<1>(a, tab, stream);
-    }
+    return a.quats ? launch_transform<true>(a, tab, stream) : launch_transform<false>(a, tab, stream);
 }
 
 unsigned int quantize_tc_status(bool clear)

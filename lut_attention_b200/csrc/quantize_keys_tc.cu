@@ -1,24 +1,32 @@
-// Quantize-on-write on the 5th-generation tensor cores, head dimension 128,
-// bf16 or fp16 keys (AXELRAM, arXiv 2604.02638, abstract: keys are transformed
-// once on write and stored as indices into a design-time codebook).
+// Quantize-on-write on the 5th-generation tensor cores, head dimension 128, 256
+// or 512, bf16 or fp16 keys (AXELRAM, arXiv 2604.02638, abstract: keys are
+// transformed once on write and stored as indices into a design-time codebook).
 //
 // The sign-flipped Walsh-Hadamard transform is a matrix product:
 //     y = H diag(s) k   for every key   <=>   Y = K (H diag(s))^T
 // H diag(s) has entries +-1, exact in bf16/fp16, and the keys are bf16/fp16, so
 // every product is exact and tcgen05 accumulates in fp32: the same arithmetic as
-// a butterfly transform, without spending CUDA-core instructions on it.
+// a butterfly transform, without spending CUDA-core instructions on it.  Wider
+// heads follow Sylvester's recursion: with H_256 = [[H, H], [H, -H]] and
+// H_512 = H_4 (x) H, y is a signed sum of z_l = H diag(s_l) k_l over the
+// 128-coordinate slices l of the key, which the tensor cores compute slice by
+// slice and the epilogue combines.  The IsoQuant block rotation (quats) takes
+// the same path with another B (see the block-rotation helpers below).
 //
 // One CTA per SM, persistent over 128-key tiles:
-//   warp 16 (TMA) : streams key tiles HBM -> shared memory (4-stage ring,
-//                   128-byte swizzle, one 32 KB tile per stage);
-//   warp 17 (MMA) : 8 tcgen05.mma (M=128, N=128, K=16) per tile into one of two
-//                   128-column fp32 accumulators in tensor memory;
-//   warps 0-15    : two epilogue groups of 8 warps, group e draining
-//                   accumulator e (the CTA's even or odd tiles), so two tiles are
-//                   in the epilogue at once.  In a group, two warps per 32 keys
-//                   (a tensor-memory lane quadrant), one per half of the 128
-//                   columns: read y, exchange the partial sums of y^2
-//                   (= d ||k||^2 in total), quantize, pack, store.
+//   warp 16 (TMA) : streams key slices HBM -> shared memory (a ring of 32 KB
+//                   stages, 128-byte swizzle, one 128-coordinate slice of a
+//                   tile per stage);
+//   warp 17 (MMA) : 8 tcgen05.mma (M=128, N=128, K=16) per slice into the
+//                   tile's 128-column fp32 accumulator for that slice;
+//   warps 0-15    : at d = 128 and 256, two epilogue groups of 8 warps, group e
+//                   draining the accumulators of the CTA's even or odd tiles, so
+//                   two tiles are in the epilogue at once.  In a group, two warps
+//                   per 32 keys (a tensor-memory lane quadrant), one per half of
+//                   the 128 columns: read y, exchange the partial sums of y^2
+//                   (= d ||k||^2 in total), quantize, pack, store.  At d = 512
+//                   the four accumulators fill tensor memory: one tile at a time,
+//                   drained by all 16 warps (a 32-column quarter each).
 // Quantization: u = y / sqrt(sum y^2); with g = u * G_SCALE + G_OFF every
 // bucket [j - 0.5, j + 0.5) of g holds at most one decision boundary, so
 //     idx = base[j] + (g > tau[j]),   j = round(g)

@@ -1,6 +1,9 @@
-// Score-on-read on the 5th-generation tensor cores, head dimension 128 (AXELRAM,
-// arXiv 2604.02638, abstract: scores come from table lookups on the stored
-// indices, never from dequantized keys).
+// Score-on-read on the 5th-generation tensor cores, head dimension 128, 256 or
+// 512 (AXELRAM, arXiv 2604.02638, abstract: scores come from table lookups on
+// the stored indices, never from dequantized keys).  Wider heads run each tile
+// as 2 or 4 subtiles of 128 coordinates into one accumulator (see Cfg); the
+// queries are rotated by the Walsh-Hadamard transform or, for keys written with
+// it, by the IsoQuant block rotation.
 //
 // For the G query heads of a KV head the scores of a tile of 128 keys form one
 // small contraction, s[t][g] = norm_t * sum_j c[idx_t[j]] * q''_g[j], so the

@@ -261,7 +261,9 @@ int axr_select_signs(const void *K, int kdtype, const void *q, int qdtype, int64
  * Device-side status of the tensor-core kernels (no counterpart in the method;
  * a diagnostic).  Every wait inside those kernels is bounded; a wait that runs
  * out records a bit here instead of hanging: 1 = a tile load never arrived,
- * 2 = a matrix product never completed, 4 = an accumulator was never released.
+ * 2 = a matrix product never completed, 4 = an accumulator was never released;
+ * 8 = the read kernel found its shared-memory window laid out so that its stages
+ * do not fit, and scored nothing.
  * Synchronizes the current device, writes the OR of the recorded bits to
  * *status (0 = none) and clears them if `clear` is non-zero.
  */

@@ -66,7 +66,11 @@ using namespace sm100;
 constexpr int kD = 128;
 constexpr float kInvSqrtD = 0.08838834764831845f;   // 1 / sqrt(128), the attention temperature
 constexpr int kTileRows = 128;
-constexpr int kStages = 6;            // a multiple of every stream count: a stream owns whole stages
+// Stages of packed rows in flight per CTA: 6 at d = 128 (6 tiles), 12 for wider
+// heads, whose tiles take NH stages each.  Stages 0-5 sit in the gap below the
+// lookup table when it holds them (otherwise after it), stages 6-11 after it.
+constexpr int kStagesMax = 12;
+constexpr int kLowStages = 6;
 constexpr int kGroupThreads = 128;    // worker threads of one stream (one per key of a tile)
 constexpr int kK = 2 * kD;            // two digits per coordinate
 constexpr int kACols = kK / 4;        // tensor-memory columns of one A buffer
@@ -102,6 +106,7 @@ struct Cfg {
     static constexpr int kDOff = S * 2 * kACols;      // A buffers first, then D buffers
     static constexpr int kSliceB = N * kK;            // B bytes of one subtile's K block
     static constexpr int kBBytes = kSliceB * NH;      // one B buffer
+    static constexpr int kStages = (NH == 1) ? kLowStages : kStagesMax;
     static_assert(kStages % S == 0, "streams must own whole stages");
     static_assert(kDOff + S * 2 * N <= kTmemCols, "tensor memory budget");
     static_assert(kSliceB <= kBBytesMax, "B buffer");
@@ -149,7 +154,7 @@ struct TcParams {
 
 constexpr int kMaxStreams = 3;
 struct Smem {
-    uint64_t full[kStages], empty[kStages];
+    uint64_t full[kStagesMax], empty[kStagesMax];
     // per stream and buffer: A written (workers); products done (one commit: A
     // may be overwritten, D may be read)
     uint64_t a_full[kMaxStreams][2], mma_done[kMaxStreams][2];
@@ -404,9 +409,20 @@ __device__ __forceinline__ uint32_t lut_addr(const uint32_t *w, int l, uint32_t 
 // (so one PRMT forms a full address), the rest below it when the gap is large
 // enough, else after it.
 constexpr int kBRegion = 32768;       // two B buffers per stream, for every stream
-constexpr int kRestBytes = kStages * kStageBytes + kBRegion + kSmemBook;
+constexpr int kRestBytes = kLowStages * kStageBytes + kBRegion + kSmemBook;
 constexpr size_t kSmemRequest = 1024 + 65536 + kLutBytes + kRestBytes;
 static_assert(kSmemRequest <= 232448, "shared memory per block");
+
+// Addresses of the NS stages: the first kLowStages from `lo`, the rest from `hi`.
+template <int NS>
+struct StageMap {
+    uint8_t *lo, *hi;
+    __device__ __forceinline__ uint8_t *at(int s) const
+    {
+        if constexpr (NS <= kLowStages) return lo + s * kStageBytes;
+        return s < kLowStages ? lo + s * kStageBytes : hi + (s - kLowStages) * kStageBytes;
+    }
+};
 template <int NQ, int NH>
 constexpr bool b_fits()
 {
@@ -464,7 +480,8 @@ struct Worker {
         for (int c = 0; c < NL; ++c) tmem_ld16(taddr + 16 * c, acc[c]);
     }
 
-    static __device__ void run(const TcParams &p, Smem &S, int g, uint8_t *sStage, uint8_t *sB, uint32_t lut_base,
+    static __device__ void run(const TcParams &p, Smem &S, int g, const StageMap<C::kStages> &sm, uint8_t *sB,
+                               uint32_t lut_base,
                                uint32_t tmem, int t0, int t1)
     {
         const int lane = threadIdx.x & 31;
@@ -491,8 +508,8 @@ struct Worker {
                 if constexpr (NH > 1) {
                     // the CTA's load of (tile, slice) went to stage i mod kStages
                     const int i = (tile - t0) * NH + sl;
-                    s = i % kStages;
-                    sph = static_cast<uint32_t>(i / kStages) & 1u;
+                    s = i % C::kStages;
+                    sph = static_cast<uint32_t>(i / C::kStages) & 1u;
                 }
                 if (!mbar_wait_warp(smem_u32(&S.full[s]), sph)) {
                     if (lane == 0) atomicOr(&g_status, kErrTimeoutLoad);
@@ -501,7 +518,7 @@ struct Worker {
                 }
                 uint32_t w[NW + 1];
                 {
-                    const uint8_t *st = sStage + s * kStageBytes;
+                    const uint8_t *st = sm.at(s);
 #pragma unroll
                     for (int c = 0; c < P / 16; ++c) {
                         const uint4 x = *reinterpret_cast<const uint4 *>(st + chunk_offset<P>(r, c));
@@ -511,7 +528,7 @@ struct Worker {
                 }
                 // this tile's key norm, with its first slice (its scores are due two tiles from now)
                 if (sl == 0)
-                    nk = reinterpret_cast<const float *>(sStage + s * kStageBytes + kStageCodeBytes)
+                    nk = reinterpret_cast<const float *>(sm.at(s) + kStageCodeBytes)
                         [((h * p.head_stride + ti * kTileRows + p.nshift) & 3) + r];
                 mbar_arrive(smem_u32(&S.empty[s]));
 
@@ -598,8 +615,8 @@ struct Worker {
                 mbar_arrive(smem_u32(&S.a_full[g][ab]));
                 if constexpr (NH == 1) {
                     s += C::S;
-                    if (s >= kStages) {
-                        s -= kStages;
+                    if (s >= C::kStages) {
+                        s -= C::kStages;
                         sph ^= 1;
                     }
                 }
@@ -647,11 +664,21 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base1k = (raw + 1023u) & ~1023u;
     const uint32_t lut_pos = (base1k + 65535u) & ~65535u;
-    const bool rest_first = lut_pos - base1k >= static_cast<uint32_t>(kRestBytes);
-    const uint32_t rest_pos = rest_first ? base1k : lut_pos + kLutBytes;
+    // stages 0-5 in the gap below the table when it holds them, else after it;
+    // then stages 6-11 (wide heads), B and the bookkeeping.  A shared window whose
+    // gap is neither large nor small enough is refused before any barrier exists.
+    const bool low = lut_pos - base1k >= static_cast<uint32_t>(kLowStages * kStageBytes);
+    const uint32_t hi_pos = lut_pos + kLutBytes;
+    const uint32_t st_lo = low ? base1k : hi_pos;
+    const uint32_t st_hi = low ? hi_pos : hi_pos + kLowStages * kStageBytes;
+    const uint32_t b_pos = st_hi + (C::kStages - kLowStages) * kStageBytes;
+    if (b_pos + kBRegion + kSmemBook > raw + static_cast<uint32_t>(kSmemRequest)) {
+        if (threadIdx.x == 0) atomicOr(&g_status, kErrLayout);
+        return;
+    }
     uint8_t *sLut = smem_raw + (lut_pos - raw);
-    uint8_t *sStage = smem_raw + (rest_pos - raw);                  // kStages x 8 KB
-    uint8_t *sB = sStage + kStages * kStageBytes;                    // S streams x 2 B buffers
+    const StageMap<C::kStages> sm{smem_raw + (st_lo - raw), smem_raw + (st_hi - raw)};
+    uint8_t *sB = smem_raw + (b_pos - raw);                          // S streams x 2 B buffers
     Smem &S = *reinterpret_cast<Smem *>(sB + kBRegion);
 
     const int warp = threadIdx.x >> 5;
@@ -660,7 +687,7 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
     const int t1 = min(p.total_tiles, t0 + p.tiles_per_cta);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&S.full[s]), 1);
             mbar_init(smem_u32(&S.empty[s]), kGroupThreads);     // consumed by one stream
         }
@@ -706,11 +733,12 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
                     }
                     const uint32_t full = smem_u32(&S.full[s]);
                     mbar_arrive_expect_tx(full, kTileRows * P + (sl == 0 ? kNormBox * 4 : 0));
-                    tma_load_2d(smem_u32(sStage + s * kStageBytes), &p.tmap, sl * P, row, full);
+                    const uint32_t stg = smem_u32(sm.at(s));
+                    tma_load_2d(stg, &p.tmap, sl * P, row, full);
                     if (sl == 0)
-                        tma_load_1d(smem_u32(sStage + s * kStageBytes + kStageCodeBytes), &p.nmap,
+                        tma_load_1d(stg + kStageCodeBytes, &p.nmap,
                                     (row + p.nshift) & ~3, full);
-                    if (++s == kStages) {
+                    if (++s == C::kStages) {
                         s = 0;
                         ph ^= 1;
                     }
@@ -721,9 +749,9 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
                 }
             }
             // every load issued has landed before the CTA may exit
-            for (int k = 0; k < kStages && k < it; ++k) {
+            for (int k = 0; k < C::kStages && k < it; ++k) {
                 const int j = it - 1 - k;
-                mbar_wait(smem_u32(&S.full[j % kStages]), (j / kStages) & 1);
+                mbar_wait(smem_u32(&S.full[j % C::kStages]), (j / C::kStages) & 1);
             }
         }
     } else if (warp >= C::kWarpMma0) {
@@ -778,7 +806,7 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
         }
     } else {
         // ----------------------------------------------------------- workers
-        Worker<B, NQ, NH>::run(p, S, warp / 4, sStage, sB, lut_pos, tmem, t0, t1);
+        Worker<B, NQ, NH>::run(p, S, warp / 4, sm, sB, lut_pos, tmem, t0, t1);
     }
 
     tc_fence_before_sync();

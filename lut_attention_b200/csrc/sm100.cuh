@@ -22,6 +22,7 @@ namespace sm100 {
 constexpr unsigned kErrTimeoutLoad = 1u;     // a TMA stage never arrived
 constexpr unsigned kErrTimeoutMma = 2u;      // an MMA commit never arrived
 constexpr unsigned kErrTimeoutDrain = 4u;    // the epilogue never released a buffer
+constexpr unsigned kErrLayout = 8u;          // the shared-memory window cannot hold the stages
 constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)

@@ -406,10 +406,13 @@ __device__ __forceinline__ uint32_t lut_addr(const uint32_t *w, int l, uint32_t 
 }
 
 // Dynamic shared memory: the table on a 64 KB boundary of the shared window
-// (so one PRMT forms a full address), the rest below it when the gap is large
-// enough, else after it.
+// (so one PRMT forms a full address).  The request covers the table's
+// alignment gap (at most 64 KB, which holds stages 0-5 when it is large
+// enough), the table, and after it kRestBytes: stages 6-11, B and the
+// bookkeeping.
 constexpr int kBRegion = 32768;       // two B buffers per stream, for every stream
-constexpr int kRestBytes = kLowStages * kStageBytes + kBRegion + kSmemBook;
+constexpr int kRestBytes = (kStagesMax - kLowStages) * kStageBytes + kBRegion + kSmemBook;
+static_assert(kLowStages * kStageBytes == (kStagesMax - kLowStages) * kStageBytes, "either half of the stages");
 constexpr size_t kSmemRequest = 1024 + 65536 + kLutBytes + kRestBytes;
 static_assert(kSmemRequest <= 232448, "shared memory per block");
 

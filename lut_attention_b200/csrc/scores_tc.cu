@@ -122,6 +122,12 @@ struct Lookup {
     static constexpr int FB = C * B;              // 8, 6, 8, 4
     static constexpr int EB = 2 * C;              // entry bytes: C hi digits, C lo digits
     static constexpr int NF = 1 << FB;            // table fields
+    // b = 3: the table is indexed by a whole byte, and a second one sits in the
+    // unused upper half of every 256-byte row (lane offsets 128 + 4 lane):
+    // the first reads the 6-bit field in bits 0..5 of the byte, the second in
+    // bits 2..7, so a field that starts 0 or 2 bits into a byte costs one PRMT
+    static constexpr bool kByteTables = (B == 3);
+    static constexpr int kRows = kByteTables ? 256 : NF;
 };
 
 struct TcParams {
@@ -354,8 +360,10 @@ __device__ void build_lut(const TcParams &p, uint8_t *lut)
 {
     using LK = Lookup<B>;
     constexpr uint32_t mask = (1u << B) - 1u;
-    for (int e = threadIdx.x; e < LK::NF * 32; e += kWorkers) {
-        const int field = e / 32, ln = e % 32;
+    constexpr int kTables = LK::kByteTables ? 2 : 1;
+    for (int e = threadIdx.x; e < LK::kRows * 32 * kTables; e += kWorkers) {
+        const int row = e / (32 * kTables), ln = e % 32, tab = (e / 32) % kTables;
+        const int field = LK::kByteTables ? ((tab == 0) ? (row & (LK::NF - 1)) : (row >> 2)) : row;
         uint8_t bytes[LK::EB];
 #pragma unroll
         for (int i = 0; i < LK::C; ++i) {
@@ -363,7 +371,7 @@ __device__ void build_lut(const TcParams &p, uint8_t *lut)
             bytes[i] = static_cast<uint8_t>(p.hi[code]);
             bytes[LK::C + i] = static_cast<uint8_t>(p.lo[code]);
         }
-        uint8_t *dst = lut + field * 256 + ln * LK::EB;
+        uint8_t *dst = lut + row * 256 + tab * 128 + ln * LK::EB;
 #pragma unroll
         for (int i = 0; i < LK::EB; ++i) dst[i] = bytes[i];
     }
@@ -381,8 +389,9 @@ __device__ __forceinline__ int chunk_offset(int r, int c)
 
 // shared-memory address of the table entry for lookup l of a row held in w[].
 // base_lane = table base (64 KB aligned) | lane * entry size, so the field
-// only has to be placed in bits 8.. of it: one PRMT for byte fields, a shift
-// and one LOP3 otherwise.
+// only has to be placed in bits 8.. of it: one PRMT for byte fields (and, at
+// b = 3, for fields starting 0 or 2 bits into a byte), a shift and one LOP3
+// otherwise.
 template <int B>
 __device__ __forceinline__ uint32_t lut_addr(const uint32_t *w, int l, uint32_t base_lane)
 {
@@ -393,6 +402,11 @@ __device__ __forceinline__ uint32_t lut_addr(const uint32_t *w, int l, uint32_t 
         // bytes: [lane offset, field, table base bits 16..23, 24..31]
         const uint32_t sel = 0x7604u | (static_cast<uint32_t>(sh >> 3) << 4);
         return __byte_perm(w[wi], base_lane, sel);
+    } else if (LK::kByteTables && ((sh & 7) == 0 || (sh & 7) == 2)) {
+        // the byte holding the field indexes the first table (field in bits
+        // 0..5) or the second (bits 2..7, lane offsets + 128)
+        const uint32_t sel = 0x7604u | (static_cast<uint32_t>(sh >> 3) << 4);
+        return __byte_perm(w[wi], (sh & 7) == 0 ? base_lane : (base_lane | 128u), sel);
     } else {
         constexpr uint32_t fmask = ((1u << LK::FB) - 1u) << 8;
         uint32_t x;
@@ -662,7 +676,7 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
     constexpr int P = kD * B / 8;             // bytes of one 128-coordinate slice of a packed row
     static_assert(kTileRows * P <= kStageCodeBytes && kStageCodeBytes + kNormBox * 4 <= kStageBytes,
                   "stage too small for a tile of packed rows and its norms");
-    static_assert(LK::NF * 256 <= kLutBytes, "lookup table too large");
+    static_assert(LK::kRows * 256 <= kLutBytes, "lookup table too large");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base1k = (raw + 1023u) & ~1023u;

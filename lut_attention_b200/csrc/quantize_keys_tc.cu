@@ -571,19 +571,25 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             // (partial sums 0,1 and 2,3 in paired FMAs: coordinates e = 0, 1 mod 4 and 2, 3 mod 4;
             // at d = 256, 0,1 for y = z_0 + z_1 and 2,3 for y = z_0 - z_1)
             float2 p01 = make_float2(0.0f, 0.0f), p23 = make_float2(0.0f, 0.0f);
+            // d = 128: the half's 64 columns are read once, with one wait, and held
+            // for pass 2; the accumulator is released as soon as they are read
+            uint32_t vh[NH == 1 ? 2 * 32 : 1];
+            if constexpr (NH == 1) {
+                tmem_ld64(col_addr, vh);
+                tc_fence_before_sync();
+                mbar_arrive(smem_u32(&S.acc_empty[acc]));
 #pragma unroll
-            for (int c = 0; c < kHalfCols / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(col_addr + 32 * c, v);
-                if constexpr (NH == 1) {
+                for (int e = 0; e < 2 * 32; e += 4) {
+                    const float2 x01 = make_float2(__uint_as_float(vh[e]), __uint_as_float(vh[e + 1]));
+                    const float2 x23 = make_float2(__uint_as_float(vh[e + 2]), __uint_as_float(vh[e + 3]));
+                    p01 = __ffma2_rn(x01, x01, p01);
+                    p23 = __ffma2_rn(x23, x23, p23);
+                }
+            } else {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const float2 x01 = make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                        const float2 x23 = make_float2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                        p01 = __ffma2_rn(x01, x01, p01);
-                        p23 = __ffma2_rn(x23, x23, p23);
-                    }
-                } else {
+                for (int c = 0; c < kHalfCols / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(col_addr + 32 * c, v);
                     uint32_t v1[32];
                     tmem_ld32(col_addr + kD + 32 * c, v1);
 #pragma unroll
@@ -625,13 +631,12 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const float2 ag2 = kBlock ? make_float2(ug, ug) : a2;
             const float2 gofs2 = kBlock ? make_float2(0.0f, 0.0f) : goff2;
             if constexpr (NH == 1) {
-                uint32_t v[32];
-                tmem_ld32(col_addr, v);
-                if (finite && !clamp) quantize_chunk<B, 0, 0, false>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                else if (finite) quantize_chunk<B, 0, 0, true>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                tmem_ld32(col_addr + 32, v);
-                if (finite && !clamp) quantize_chunk<B, 32, 0, false>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                else if (finite) quantize_chunk<B, 32, 0, true>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                const uint32_t(&va)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&vh[0]);
+                const uint32_t(&vb)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&vh[32]);
+                if (finite && !clamp) quantize_chunk<B, 0, 0, false>(va, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 0, 0, true>(va, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                if (finite && !clamp) quantize_chunk<B, 32, 0, false>(vb, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 32, 0, true>(vb, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
             } else {
 #pragma unroll
                 for (int c = 0; c < kHalfCols / 32; ++c) {
@@ -680,8 +685,10 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                     }
                 }
             }
-            tc_fence_before_sync();
-            mbar_arrive(smem_u32(&S.acc_empty[acc]));
+            if constexpr (NH != 1) {
+                tc_fence_before_sync();
+                mbar_arrive(smem_u32(&S.acc_empty[acc]));
+            }
 
             const int64_t row = static_cast<int64_t>(t) * kTileRows + key;
             if (row < p.n) {

@@ -1,6 +1,7 @@
 // Internal declarations shared by the libaxr translation units (not installed).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -146,5 +147,11 @@ cudaError_t launch_sign_select(const SignSelectArgs &a, cudaStream_t stream);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device.  The limit belongs to the kernel's instance in each device's context,
+// so it is set once per device; `done` holds one bit per device (devices 64 and
+// up are set on every call).  Safe to call from several host threads.
+cudaError_t allow_dynamic_smem(const void *kernel, size_t bytes, std::atomic<unsigned long long> &done);
 
 }  // namespace axr

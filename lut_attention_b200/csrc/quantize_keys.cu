@@ -182,12 +182,16 @@ template <int D, int B, typename T>
 cudaError_t launch_typed(const QuantizeArgs &a, cudaStream_t stream)
 {
     auto kernel = quantize_keys_kernel<D, B, T>;
-    static int blocks_per_sm = 0;
+    // resident blocks per SM (the same on every device of one model; it sizes the
+    // grid, and the kernel strides over the rows, so any value is correct)
+    static std::atomic<int> blocks_cached{0};
+    int blocks_per_sm = blocks_cached.load(std::memory_order_relaxed);
     if (blocks_per_sm == 0) {
         int v = 0;
         cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, kThreads, 0);
         if (e != cudaSuccess) return e;
         blocks_per_sm = v > 0 ? v : 1;
+        blocks_cached.store(blocks_per_sm, std::memory_order_relaxed);
     }
     constexpr int E = D >= 32 ? 32 : D;
     constexpr int RW = 32 / (D / E);

@@ -740,13 +740,10 @@ cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_
     const size_t smem = 1024 + stages<NH>() * kABytes + kBReg + kMaxBuckets * sizeof(float2) + sizeof(Smem);
     static_assert(1024 + stages<NH>() * kABytes + kBReg + kMaxBuckets * sizeof(float2) + sizeof(Smem) <= 232448,
                   "shared memory per block");
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> smem_allowed{0};     // one bit per device
+    if (cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(kernel), smem, smem_allowed);
+        e != cudaSuccess)
+        return e;
     TcParams p{};
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return cudaErrorNotSupported;

@@ -861,13 +861,10 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     constexpr int PT = P * NH;                // the whole packed row
     auto kernel = scores_tc_kernel<B, NQ, NH>;
     const size_t smem = kSmemRequest;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> smem_allowed{0};     // one bit per device
+    if (cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(kernel), smem, smem_allowed);
+        e != cudaSuccess)
+        return e;
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return cudaErrorNotSupported;
     TcParams p{};

@@ -108,10 +108,11 @@ def job_scores_per_s(wl: workloads.Workload, world: int, ms_per_step: float) -> 
 
 def kernel_file(kind: str, wl: workloads.Workload) -> str:
     """Source file of the kernel the library runs for this workload (api.cu takes the
-    tensor-core kernels at d = 128, for the write path with bf16/f16 keys)."""
+    tensor-core kernels at d = 128, 256 and 512, for the write path with bf16/f16 keys)."""
+    tc_width = wl.d in (128, 256, 512)
     if kind == "quantize_keys":
-        return "quantize_keys_tc.cu" if wl.d == 128 and wl.dtype in ("bf16", "f16") else "quantize_keys.cu"
-    return "scores_tc.cu" if wl.d == 128 else "scores.cu"
+        return "quantize_keys_tc.cu" if tc_width and wl.dtype in ("bf16", "f16") else "quantize_keys.cu"
+    return "scores_tc.cu" if tc_width else "scores.cu"
 
 
 def profiled_traffic(kernel_file: str, workload: str, b: int):

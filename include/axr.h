@@ -13,7 +13,8 @@
  *   - All buffers are owned by the caller.  The library never allocates device
  *     memory; it keeps only a host-side, thread-safe cache of codebooks.
  *   - Device-pointer arguments must be device (or managed) memory of the current
- *     device.  Calls enqueue work on `stream` and return without synchronising;
+ *     device; memory of another device is refused with AXR_EINVAL.  Calls
+ *     enqueue work on `stream` and return without synchronising;
  *     results are valid once the stream has reached that point.
  *   - Argument errors are detected on the host before any launch and return
  *     AXR_EINVAL / AXR_EUNSUPPORTED with nothing enqueued.  A failed launch

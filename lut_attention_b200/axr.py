@@ -75,10 +75,19 @@ def _raise(rc: int, where: str) -> None:
         raise AxrError(rc, where, detail)
 
 
-def _stream_handle(stream) -> int:
+def _stream_handle(stream, device=None) -> int:
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _call(name: str, device: torch.device, stream, *args) -> None:
+    """Call libaxr's `name` with the tensors' device current (the library checks its
+    pointers against, and launches on, the current device), on `stream` or that
+    device's current stream; a status other than AXR_OK raises."""
+    with torch.cuda.device(device):
+        rc = getattr(library(), name)(*args, _stream_handle(stream, device))
+    _raise(rc, name)
 
 
 def _require_cuda(t: torch.Tensor, name: str) -> None:
@@ -124,9 +133,8 @@ def axr_quantize_keys(K: torch.Tensor, b: int, signs: torch.Tensor,
     _require_cuda(norms, "norms")
     if idx.numel() < n * P or norms.numel() < n:
         raise ValueError("idx/norms too small")
-    rc = library().axr_quantize_keys(K.data_ptr(), _DTYPE_CODE[K.dtype], n, d, b, signs.data_ptr(),
-                                     idx.data_ptr(), norms.data_ptr(), _stream_handle(stream))
-    _raise(rc, "axr_quantize_keys")
+    _call("axr_quantize_keys", K.device, stream,
+          K.data_ptr(), _DTYPE_CODE[K.dtype], n, d, b, signs.data_ptr(), idx.data_ptr(), norms.data_ptr())
     return idx, norms
 
 
@@ -155,10 +163,9 @@ def axr_scores(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, group: i
     _require_cuda(scores, "scores")
     if scores.numel() < hg * n or scores.dtype != torch.float32:
         raise ValueError("scores must be float32 with (heads*group)*n elements")
-    rc = library().axr_scores(q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), n,
-                              heads, group, d, b, signs.data_ptr(), scores.data_ptr(),
-                              _stream_handle(stream))
-    _raise(rc, "axr_scores")
+    _call("axr_scores", q.device, stream,
+          q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), n, heads, group, d, b,
+          signs.data_ptr(), scores.data_ptr())
     return scores
 
 
@@ -188,9 +195,8 @@ def axr_quantize_keys_block(K: torch.Tensor, b: int, quats: torch.Tensor, idx: t
     _require_cuda(norms, "norms")
     if idx.numel() < n * P or norms.numel() < n:
         raise ValueError("idx/norms too small")
-    rc = library().axr_quantize_keys_block(K.data_ptr(), _DTYPE_CODE[K.dtype], n, d, b, quats.data_ptr(),
-                                           idx.data_ptr(), norms.data_ptr(), _stream_handle(stream))
-    _raise(rc, "axr_quantize_keys_block")
+    _call("axr_quantize_keys_block", K.device, stream,
+          K.data_ptr(), _DTYPE_CODE[K.dtype], n, d, b, quats.data_ptr(), idx.data_ptr(), norms.data_ptr())
     return idx, norms
 
 
@@ -219,9 +225,9 @@ def axr_scores_block(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, gr
     _require_cuda(scores, "scores")
     if scores.numel() < hg * n or scores.dtype != torch.float32:
         raise ValueError("scores must be float32 with (heads*group)*n elements")
-    rc = library().axr_scores_block(q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), n,
-                                    heads, group, d, b, quats.data_ptr(), scores.data_ptr(), _stream_handle(stream))
-    _raise(rc, "axr_scores_block")
+    _call("axr_scores_block", q.device, stream,
+          q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), n, heads, group, d, b,
+          quats.data_ptr(), scores.data_ptr())
     return scores
 
 
@@ -254,11 +260,9 @@ def axr_append_scores(k_new: torch.Tensor, q: torch.Tensor, idx: torch.Tensor, n
     _require_cuda(scores, "scores")
     if scores.numel() < hg * (pos + 1) or scores.dtype != torch.float32:
         raise ValueError("scores must be float32 with (heads*group)*(pos+1) elements")
-    rc = library().axr_append_scores(k_new.data_ptr(), _DTYPE_CODE[k_new.dtype], q.data_ptr(),
-                                     _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), capacity, pos,
-                                     heads, group, d, b, signs.data_ptr(), scores.data_ptr(),
-                                     _stream_handle(stream))
-    _raise(rc, "axr_append_scores")
+    _call("axr_append_scores", k_new.device, stream,
+          k_new.data_ptr(), _DTYPE_CODE[k_new.dtype], q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(),
+          norms.data_ptr(), capacity, pos, heads, group, d, b, signs.data_ptr(), scores.data_ptr())
     return scores
 
 
@@ -304,11 +308,10 @@ def axr_attention(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, V: to
             or out.dtype != torch.float32:
         raise ValueError("scores and out must be float32 and large enough")
     ws_bytes = workspace.numel() * workspace.element_size()
-    rc = library().axr_attention(q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(),
-                                 V.data_ptr(), _DTYPE_CODE[V.dtype], n, heads, group, d, b, signs.data_ptr(),
-                                 scores.data_ptr(), workspace.data_ptr(), ws_bytes, out.data_ptr(),
-                                 _stream_handle(stream))
-    _raise(rc, "axr_attention")
+    _call("axr_attention", q.device, stream,
+          q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), V.data_ptr(),
+          _DTYPE_CODE[V.dtype], n, heads, group, d, b, signs.data_ptr(), scores.data_ptr(),
+          workspace.data_ptr(), ws_bytes, out.data_ptr())
     return out, scores
 
 
@@ -335,11 +338,9 @@ def axr_attention_static(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor
     if scores.dtype != torch.float32 or out.dtype != torch.float32 or scores.numel() < hg * n \
             or out.numel() < hg * d:
         raise ValueError("scores and out must be float32 and large enough")
-    rc = library().axr_attention_static(q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(),
-                                        V.data_ptr(), _DTYPE_CODE[V.dtype], n, heads, group, d, b,
-                                        signs.data_ptr(), scores.data_ptr(), out.data_ptr(),
-                                        _stream_handle(stream))
-    _raise(rc, "axr_attention_static")
+    _call("axr_attention_static", q.device, stream,
+          q.data_ptr(), _DTYPE_CODE[q.dtype], idx.data_ptr(), norms.data_ptr(), V.data_ptr(),
+          _DTYPE_CODE[V.dtype], n, heads, group, d, b, signs.data_ptr(), scores.data_ptr(), out.data_ptr())
     return out, scores
 
 
@@ -374,10 +375,9 @@ def axr_select_signs(K: torch.Tensor, q: torch.Tensor, group: int, b: int, candi
         _require_cuda(t, name)
     if errors.dtype != torch.float32 or errors.numel() < C * heads or best.dtype != torch.int32:
         raise ValueError("errors must be float32 with C*heads elements, best int32")
-    rc = library().axr_select_signs(K.data_ptr(), _DTYPE_CODE[K.dtype], q.data_ptr(), _DTYPE_CODE[q.dtype], n,
-                                    samples, heads, group, d, b, candidates.data_ptr(), C, errors.data_ptr(),
-                                    best.data_ptr(), _stream_handle(stream))
-    _raise(rc, "axr_select_signs")
+    _call("axr_select_signs", K.device, stream,
+          K.data_ptr(), _DTYPE_CODE[K.dtype], q.data_ptr(), _DTYPE_CODE[q.dtype], n, samples, heads, group, d,
+          b, candidates.data_ptr(), C, errors.data_ptr(), best.data_ptr())
     return errors, best
 
 

@@ -42,20 +42,29 @@ int elem_size(int dtype)
     }
 }
 
-// A device pointer the current device's kernels can dereference: device memory,
-// managed memory, or host memory mapped into the device address space.
-bool device_accessible(const void *p)
+// Where a pointer lives, for the current device's kernels: device memory of the
+// current device, managed memory, or host memory mapped into the device address
+// space are usable; memory of another device is reported as such (a kernel here
+// would fault on it without peer access).
+enum class Access { kUsable, kOtherDevice, kNone };
+
+Access device_access(const void *p, int *owner)
 {
     cudaPointerAttributes attr;
     if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
         cudaGetLastError();
-        return false;
+        return Access::kNone;
     }
     switch (attr.type) {
-    case cudaMemoryTypeDevice:
-    case cudaMemoryTypeManaged: return true;
-    case cudaMemoryTypeHost: return attr.devicePointer != nullptr;
-    default: return false;
+    case cudaMemoryTypeDevice: {
+        int cur = 0;
+        if (cudaGetDevice(&cur) != cudaSuccess) return Access::kNone;
+        *owner = attr.device;
+        return attr.device == cur ? Access::kUsable : Access::kOtherDevice;
+    }
+    case cudaMemoryTypeManaged: return Access::kUsable;
+    case cudaMemoryTypeHost: return attr.devicePointer != nullptr ? Access::kUsable : Access::kNone;
+    default: return Access::kNone;
     }
 }
 
@@ -63,8 +72,13 @@ int check_device_ptr(const void *p, uintptr_t align, const char *name)
 {
     if (!p) return fail(AXR_EINVAL, "%s is NULL", name);
     if (!aligned(p, align)) return fail(AXR_EINVAL, "%s is not %u-byte aligned", name, (unsigned)align);
-    if (!device_accessible(p)) return fail(AXR_EINVAL, "%s is not device-accessible memory", name);
-    return AXR_OK;
+    int owner = -1;
+    switch (device_access(p, &owner)) {
+    case Access::kUsable: return AXR_OK;
+    case Access::kOtherDevice:
+        return fail(AXR_EINVAL, "%s is memory of device %d, not of the current device", name, owner);
+    default: return fail(AXR_EINVAL, "%s is not device-accessible memory", name);
+    }
 }
 
 int check_shape(int d, int b)

@@ -60,3 +60,18 @@ def test_two_ranks_shard_and_take_the_slowest_time():
     assert s0 != s1 and k0 != k1                                  # each rank draws its own batch
     # whole-job rate: both ranks' scores over the slowest rank's time
     assert res[0]["value"] == pytest.approx(1 * 4 * 64 * 2 / (11.0e-3))
+
+
+@pytest.mark.timeout(120)
+def test_reference_arm_other_ranks_exit_without_work():
+    """Under torchrun the reference arm runs on rank 0 alone: another rank prints
+    nothing and exits 0 (no process group, no oracle)."""
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2", MASTER_ADDR="127.0.0.1", MASTER_PORT="1")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=110)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""

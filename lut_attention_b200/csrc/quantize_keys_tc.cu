@@ -572,12 +572,10 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             // at d = 256, 0,1 for y = z_0 + z_1 and 2,3 for y = z_0 - z_1)
             float2 p01 = make_float2(0.0f, 0.0f), p23 = make_float2(0.0f, 0.0f);
             // d = 128: the half's 64 columns are read once, with one wait, and held
-            // for pass 2; the accumulator is released as soon as they are read
+            // for pass 2; the accumulator is released once both halves' sums are read
             uint32_t vh[NH == 1 ? 2 * 32 : 1];
             if constexpr (NH == 1) {
                 tmem_ld64(col_addr, vh);
-                tc_fence_before_sync();
-                mbar_arrive(smem_u32(&S.acc_empty[acc]));
 #pragma unroll
                 for (int e = 0; e < 2 * 32; e += 4) {
                     const float2 x01 = make_float2(__uint_as_float(vh[e]), __uint_as_float(vh[e + 1]));
@@ -610,6 +608,14 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                 break;
             }
             const float ss = S.ss[acc][0][key] + S.ss[acc][1][key];
+            if constexpr (NH == 1) {
+                // the accumulator is in registers.  Releasing it only now, after the
+                // read of the other half's sum, keeps the group's next tile on this
+                // accumulator (which needs every thread's release) from overwriting
+                // S.ss[acc] before that read
+                tc_fence_before_sync();
+                mbar_arrive(smem_u32(&S.acc_empty[acc]));
+            }
             const float norm = sqrtf(ss) * p.inv_sqrt_d;
 
             uint32_t w[NWH + 1], w1[NWH + 1];      // codes of y (z_0 + z_1 at d = 256) and of z_0 - z_1

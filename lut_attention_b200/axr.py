@@ -97,6 +97,21 @@ def _require_cuda(t: torch.Tensor, name: str) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
+def _check_signs(signs: torch.Tensor, d: int) -> None:
+    """The sign pattern D: int8, one entry per coordinate (the kernels read d of them)."""
+    if signs.dtype != torch.int8:
+        raise ValueError("signs must be int8")
+    if signs.numel() != d:
+        raise ValueError(f"signs must have d={d} entries, got {signs.numel()}")
+
+
+def _check_read_operands(idx: torch.Tensor, norms: torch.Tensor) -> None:
+    """Packed codes are bytes and key norms fp32: the kernels read n*P bytes and
+    4*n bytes through these pointers, whatever dtype the tensor carries."""
+    if idx.dtype != torch.uint8 or norms.dtype != torch.float32:
+        raise ValueError("idx must be uint8 and norms float32")
+
+
 def axr_make_codebook(d: int, b: int) -> tuple[np.ndarray, np.ndarray]:
     """fp32 centroids (2^b, ascending) and boundaries (2^b - 1) for (d, b)."""
     L = 1 << b if 0 < b < 31 else 1
@@ -119,9 +134,8 @@ def axr_quantize_keys(K: torch.Tensor, b: int, signs: torch.Tensor,
     _require_cuda(signs, "signs")
     if K.dtype not in _DTYPE_CODE:
         raise ValueError(f"K dtype {K.dtype} not supported")
-    if signs.dtype != torch.int8:
-        raise ValueError("signs must be int8")
     d = K.shape[-1]
+    _check_signs(signs, d)
     lead = K.shape[:-1]
     n = K.numel() // d if d else 0
     P = packed_row_bytes(d, b)
@@ -131,6 +145,7 @@ def axr_quantize_keys(K: torch.Tensor, b: int, signs: torch.Tensor,
         norms = torch.empty(lead, dtype=torch.float32, device=K.device)
     _require_cuda(idx, "idx")
     _require_cuda(norms, "norms")
+    _check_read_operands(idx, norms)
     if idx.numel() < n * P or norms.numel() < n:
         raise ValueError("idx/norms too small")
     _call("axr_quantize_keys", K.device, stream,
@@ -147,9 +162,9 @@ def axr_scores(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, group: i
         _require_cuda(t, name)
     if q.dtype not in _DTYPE_CODE:
         raise ValueError(f"q dtype {q.dtype} not supported")
-    if idx.dtype != torch.uint8 or norms.dtype != torch.float32 or signs.dtype != torch.int8:
-        raise ValueError("idx must be uint8, norms float32, signs int8")
+    _check_read_operands(idx, norms)
     hg, d = q.shape
+    _check_signs(signs, d)
     if group < 1 or hg % group:
         raise ValueError("q must have heads*group rows")
     heads = hg // group
@@ -193,6 +208,7 @@ def axr_quantize_keys_block(K: torch.Tensor, b: int, quats: torch.Tensor, idx: t
         norms = torch.empty(lead, dtype=torch.float32, device=K.device)
     _require_cuda(idx, "idx")
     _require_cuda(norms, "norms")
+    _check_read_operands(idx, norms)
     if idx.numel() < n * P or norms.numel() < n:
         raise ValueError("idx/norms too small")
     _call("axr_quantize_keys_block", K.device, stream,
@@ -208,8 +224,7 @@ def axr_scores_block(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, gr
         _require_cuda(t, name)
     if q.dtype not in _DTYPE_CODE:
         raise ValueError(f"q dtype {q.dtype} not supported")
-    if idx.dtype != torch.uint8 or norms.dtype != torch.float32:
-        raise ValueError("idx must be uint8, norms float32")
+    _check_read_operands(idx, norms)
     hg, d = q.shape
     _check_quats(quats, d)
     if group < 1 or hg % group:
@@ -242,9 +257,9 @@ def axr_append_scores(k_new: torch.Tensor, q: torch.Tensor, idx: torch.Tensor, n
         _require_cuda(t, name)
     if k_new.dtype not in _DTYPE_CODE or q.dtype not in _DTYPE_CODE:
         raise ValueError("k_new and q must be float32, float16 or bfloat16")
-    if idx.dtype != torch.uint8 or norms.dtype != torch.float32 or signs.dtype != torch.int8:
-        raise ValueError("idx must be uint8, norms float32, signs int8")
+    _check_read_operands(idx, norms)
     heads, d = k_new.shape
+    _check_signs(signs, d)
     hg, dq = q.shape
     if dq != d or group < 1 or hg != heads * group:
         raise ValueError(f"q must be ({heads}*{group}, {d})")
@@ -284,9 +299,9 @@ def axr_attention(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor, V: to
         _require_cuda(t, name)
     if q.dtype not in _DTYPE_CODE or V.dtype not in _DTYPE_CODE:
         raise ValueError("q and V must be float32, float16 or bfloat16")
-    if idx.dtype != torch.uint8 or norms.dtype != torch.float32 or signs.dtype != torch.int8:
-        raise ValueError("idx must be uint8, norms float32, signs int8")
+    _check_read_operands(idx, norms)
     hg, d = q.shape
+    _check_signs(signs, d)
     if group < 1 or hg % group:
         raise ValueError("q must have heads*group rows")
     heads = hg // group
@@ -326,7 +341,9 @@ def axr_attention_static(q: torch.Tensor, idx: torch.Tensor, norms: torch.Tensor
         _require_cuda(t, name)
     if q.dtype not in _DTYPE_CODE or V.dtype not in _DTYPE_CODE:
         raise ValueError("q and V must be float32, float16 or bfloat16")
+    _check_read_operands(idx, norms)
     hg, d = q.shape
+    _check_signs(signs, d)
     if group < 1 or hg % group:
         raise ValueError("q must have heads*group rows")
     heads = hg // group

@@ -109,3 +109,69 @@ def test_sign_choice_call(fake):
     errors, best = axr.axr_select_signs(K, q, G, b, cand)
     assert errors.shape == (C, H) and best.shape == (1,)
     _check(fake, "axr_select_signs", {4: n, 5: S, 6: H, 7: G, 8: d, 9: b, 11: C})
+
+
+def _decode_inputs(d=128, b=4, heads=2, group=4, n=300):
+    idx = torch.zeros((heads, n, d * b // 8), dtype=torch.uint8)
+    norms = torch.zeros((heads, n), dtype=torch.float32)
+    q = torch.zeros((heads * group, d), dtype=torch.bfloat16)
+    V = torch.zeros((heads, n, d), dtype=torch.bfloat16)
+    scores = torch.zeros((heads * group, n), dtype=torch.float32)
+    out = torch.zeros((heads * group, d), dtype=torch.float32)
+    return idx, norms, q, V, scores, out
+
+
+def test_static_attention_refuses_wrongly_typed_operands(fake):
+    """The kernels read 4*n bytes of norms and n*P bytes of codes through raw
+    pointers: a half-precision norms tensor of the right shape would be read past
+    its end, so the binding refuses it before any call."""
+    d, b, group = 128, 4, 4
+    idx, norms, q, V, scores, out = _decode_inputs(d, b, group=group)
+    signs = torch.ones(d, dtype=torch.int8)
+    for bad in (dict(norms=norms.half()), dict(norms=norms.bfloat16()), dict(idx=idx.to(torch.int16)),
+                dict(signs=signs.to(torch.int32))):
+        a = dict(idx=idx, norms=norms, signs=signs) | bad
+        with pytest.raises(ValueError):
+            axr.axr_attention_static(q, a["idx"], a["norms"], V, group, b, a["signs"], scores, out)
+    assert not fake.calls
+
+
+def test_every_call_refuses_a_short_sign_pattern(fake):
+    """The kernels read d entries of the sign pattern D."""
+    d, b, group = 128, 4, 4
+    idx, norms, q, V, scores, out = _decode_inputs(d, b, group=group)
+    short = torch.ones(d - 1, dtype=torch.int8)
+    K = torch.zeros((5, d), dtype=torch.bfloat16)
+    k_new = torch.zeros((idx.shape[0], d), dtype=torch.bfloat16)
+    calls = [
+        lambda: axr.axr_quantize_keys(K, b, short),
+        lambda: axr.axr_scores(q, idx, norms, group, b, short),
+        lambda: axr.axr_append_scores(k_new, q, idx, norms, 3, group, b, short),
+        lambda: axr.axr_attention(q, idx, norms, V, group, b, short),
+        lambda: axr.axr_attention_static(q, idx, norms, V, group, b, short, scores, out),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="signs"):
+            call()
+    assert not fake.calls
+
+
+def test_read_calls_refuse_wrongly_typed_codes_and_norms(fake):
+    d, b, group = 128, 4, 4
+    idx, norms, q, V, scores, out = _decode_inputs(d, b, group=group)
+    signs = torch.ones(d, dtype=torch.int8)
+    quats = workloads.make_block_quats(workloads.GQA_DECODE_128K.with_(d=d))
+    k_new = torch.zeros((idx.shape[0], d), dtype=torch.bfloat16)
+    for bad_idx, bad_norms in ((idx, norms.half()), (idx.to(torch.int8), norms)):
+        calls = [
+            lambda: axr.axr_scores(q, bad_idx, bad_norms, group, b, signs),
+            lambda: axr.axr_scores_block(q, bad_idx, bad_norms, group, b, quats),
+            lambda: axr.axr_append_scores(k_new, q, bad_idx, bad_norms, 3, group, b, signs),
+            lambda: axr.axr_attention(q, bad_idx, bad_norms, V, group, b, signs),
+            lambda: axr.axr_quantize_keys(torch.zeros((idx.shape[0], idx.shape[1], d), dtype=torch.bfloat16),
+                                          b, signs, idx=bad_idx, norms=bad_norms),
+        ]
+        for call in calls:
+            with pytest.raises(ValueError):
+                call()
+    assert not fake.calls

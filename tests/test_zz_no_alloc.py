@@ -15,19 +15,32 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _inputs(heads, n, d, b, group, seed):
+def _inputs(heads, n, d, b, group, seed, vdtype=torch.bfloat16):
     packed, norms = workloads.make_random_packed(heads, n, d, b, seed=seed, device=DEV)
-    wl = workloads.GQA_DECODE_128K.with_(batch=1, kv_heads=heads, group=group, T=n, seed=seed)
+    wl = workloads.GQA_DECODE_128K.with_(d=d, batch=1, kv_heads=heads, group=group, T=n, seed=seed)
     q = workloads.make_queries(wl, DEV)
     s = workloads.make_signs(wl).to(DEV)
     g = torch.Generator(device=DEV).manual_seed(seed + 17)
-    V = torch.randn((heads, n, d), generator=g, device=DEV).to(torch.bfloat16)
+    V = torch.randn((heads, n, d), generator=g, device=DEV).to(vdtype)
     return packed, norms, q, s, V
 
 
-def test_two_consecutive_calls_match_the_workspace_entry_point(axr_lib):
-    heads, n, d, b, group = 4, 9000, 128, 4, 4
-    packed, norms, q, s, V = _inputs(heads, n, d, b, group, seed=5)
+# (KV heads, keys, d, b, queries per KV head, value dtype): the padded group of
+# 3 queries, a single query, eight queries, the narrow CUDA-core read (d = 32)
+# and the widest head, with every value dtype; all fit the fixed scratch.
+CASES = [
+    (4, 9000, 128, 4, 4, torch.bfloat16),
+    (3, 5000, 128, 3, 3, torch.float16),
+    (2, 7001, 512, 2, 3, torch.float32),
+    (5, 3000, 256, 4, 8, torch.bfloat16),
+    (6, 4097, 32, 2, 1, torch.float16),
+    (2, 130, 64, 1, 2, torch.float32),
+]
+
+
+@pytest.mark.parametrize("heads,n,d,b,group,vdtype", CASES)
+def test_two_consecutive_calls_match_the_workspace_entry_point(axr_lib, heads, n, d, b, group, vdtype):
+    packed, norms, q, s, V = _inputs(heads, n, d, b, group, seed=5 + n + d, vdtype=vdtype)
     ref_out, ref_scores = axr.axr_attention(q, packed, norms, V, group, b, s)
     for _ in range(2):
         scores = torch.full((heads * group, n), float("nan"), device=DEV)

@@ -39,3 +39,13 @@ def axr_lib():
     if not os.path.exists(axr.LIB_PATH):
         build.build()
     return axr.library()
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Full-size parity counts (tests/full_parity.py), one line per workload, at
+    the end of the run's output."""
+    mod = sys.modules.get("full_parity")
+    if mod is not None and mod.REPORTS:
+        terminalreporter.write_sep("-", "full-size parity with the oracle (boundary window 1e-6)")
+        for line in mod.REPORTS:
+            terminalreporter.write_line(line)

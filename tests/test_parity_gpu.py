@@ -122,14 +122,16 @@ def test_scores_wide_heads_cross_heads(d, b, heads, n, group):
 def test_quantize_wide_heads_tensor_core_tails(d, dtype, n):
     """The d = 256 / 512 tensor-core write on partial tiles (the TMA zero-fills the
     rows past n, the epilogue drops them).  Every code flip must lie inside the
-    boundary window; the in-window flip rate is not capped here, since a few
-    hundred rows hold too few coordinates for a rate of 1e-5 to mean anything
-    (the full-size sampled tests check it)."""
+    boundary window.  The in-window flip rate is capped at 1e-5 from n = 1000
+    (2.6e5 and 5.1e5 coordinates, where the cap allows 2 and 5 flips); one or
+    127 rows hold too few coordinates for a rate of 1e-5 to mean anything (the
+    full-size tests check the rate on at least 2^20 rows)."""
     K, s = _keys(d, dtype, n, seed=9000 + d + n)
     for b in (2, 3):
         idx, norms = gpu_quantize(K, b, s)
         rep = check_quantize(K, idx, norms, b, s)
-        assert rep.ok(flip_fraction=None), f"d={d} b={b} {dtype} n={n}: {rep}"
+        cap = None if n < 1000 else 1e-5
+        assert rep.ok(flip_fraction=cap), f"d={d} b={b} {dtype} n={n}: {rep}"
 
 
 @pytest.mark.parametrize("offset", [0, 1, 2, 3])

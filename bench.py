@@ -139,7 +139,7 @@ class ClockSampler:
         "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.period = period_s
         self.samples = []
         self.max_mhz = None
@@ -199,20 +199,48 @@ class ClockSampler:
         if self._thread:
             self._thread.join()
 
-    def summary(self):
-        if not self.samples:
+    def mark(self) -> int:
+        """Index of the next sample, to summarise a later window on its own."""
+        return len(self.samples)
+
+    def summary(self, start: int = 0, stop: int | None = None):
+        window = self.samples[start:stop]
+        if not window:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
-        mhz = statistics.median(s[0] for s in self.samples)
+        mhz = statistics.median(s[0] for s in window)
         active = set()
-        for _, r in self.samples:
+        for _, r in window:
             for name, bit in self.REASONS.items():
                 if r & bit:
                     active.add(name)
         return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": sorted(active),
-                "samples": len(self.samples)}
+                "samples": len(window)}
 
 
 # ----------------------------------------------------------------- the step --
+
+def timed_steps(path, stream, steps: int, barrier):
+    """K steps between CUDA events on the launching stream, with a barrier and a
+    synchronize on both sides: (elapsed ms, mean write ms, mean read ms).  Each
+    kernel is also bracketed by its own events."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    start.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        path.quantize(i % 2)
+        ev[i][1].record(stream)
+        path.score((i + 1) % 2)
+        ev[i][2].record(stream)
+    end.record(stream)
+    barrier()
+    elapsed_ms = start.elapsed_time(end)
+    t_write = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    t_read = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    return elapsed_ms, t_write, t_read
+
 
 class Path:
     """Device buffers and the two kernels of one step."""
@@ -558,6 +586,8 @@ def main():
     ap.add_argument("--workload", default="gqa_decode_128k", choices=sorted(workloads.BY_NAME))
     ap.add_argument("--b", type=int, default=None, help="bits per coordinate (default: the workload's)")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--sustain-seconds", type=float, default=1.5,
+                    help="length of the extra window of steps timed after the K steps (0: none)")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-legs", action="store_true",
@@ -604,26 +634,28 @@ def main():
         path.score((i + 1) % 2)
     barrier()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
     barrier()
-    start.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        path.quantize(i % 2)
-        ev[i][1].record(stream)
-        path.score((i + 1) % 2)
-        ev[i][2].record(stream)
-    end.record(stream)
-    barrier()
-    clocks.busy(False)
-    elapsed_ms = start.elapsed_time(end)
-    t_write = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
-    t_read = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
-
+    mark0 = clocks.mark()
+    elapsed_ms, t_write, t_read = timed_steps(path, stream, args.steps, barrier)
+    clock_window = clocks.summary(mark0)
     elapsed_ms, t_write, t_read = max_over_ranks([elapsed_ms, t_write, t_read], world, device)
     ms_per_step = elapsed_ms / args.steps
+
+    # a longer window of the same steps (at least --sustain-seconds), so that the
+    # power-capped clock the kernels settle at is measured even for a short run;
+    # every rank runs the same number of steps
+    sus_steps = max(1, math.ceil(args.sustain_seconds * 1e3 / max(ms_per_step, 1e-3)))
+    sus_steps = int(max_over_ranks([float(sus_steps)], world, device)[0])
+    sustained = None
+    if args.sustain_seconds > 0:
+        barrier()
+        mark1 = clocks.mark()
+        s_el, s_w, s_r = timed_steps(path, stream, sus_steps, barrier)
+        s_clocks = clocks.summary(mark1)
+        s_el, s_w, s_r = max_over_ranks([s_el, s_w, s_r], world, device)
+        sustained = {"steps": sus_steps, "seconds": s_el * 1e-3, "ms_per_step": s_el / sus_steps,
+                     "write_ms": s_w, "read_ms": s_r, "clocks": s_clocks}
+    clocks.busy(False)
 
     # end to end through the public API with host buffers
     e2e = run_e2e(wl, path, device, args.e2e_steps, world)
@@ -655,8 +687,25 @@ def main():
                    "bytes_per_row": algo["read_per_row"]},
     }
     dominant = "quantize_keys" if t_write >= t_read else "scores"
-    dk = kernels[dominant]
-    src = kernel_file(dominant, wl)
+
+    def roofline(kind):
+        k = kernels[kind]
+        src = kernel_file(kind, wl)
+        return {"bound": "hbm", "kernel": kind, "source": src, "achieved": k["gbs"], "peak": peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": k["gbs"] / peak,
+                "frac_of_8tbs": k["gbs"] / NOMINAL_HBM_GBS, "traffic": profiled_traffic(src, wl.name, wl.b)}
+
+    if sustained is not None:
+        mhz = sustained["clocks"].get("sm_mhz")
+        top = sustained["clocks"].get("sm_max_mhz") or mhz
+        for kind, key, byts in (("quantize_keys", "write", algo["write"]), ("scores", "read", algo["read"])):
+            ms = sustained[f"{key}_ms"]
+            gbs = byts / (ms * 1e-3) / 1e9
+            sustained[key] = {"ms": ms, "gbs": gbs, "frac_of_measured": gbs / peak,
+                              "frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
+                              # the time at the median clock scaled to the maximum clock
+                              "ms_at_max_clock": ms * mhz / top if mhz and top else None}
+        sustained["value"] = job_scores_per_s(wl, world, sustained["ms_per_step"])
     line = {
         "metric": "lut_attention_scores_per_s",
         "value": job_scores_per_s(wl, world, ms_per_step),
@@ -673,12 +722,12 @@ def main():
         "config": config_dict(wl, world),
         "keys_per_s": keys_per_step / (ms_per_step * 1e-3),
         "kernels": kernels,
-        "roofline": {"bound": "hbm", "kernel": dominant, "source": src, "achieved": dk["gbs"], "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": dk["gbs"] / peak,
-                     "frac_of_8tbs": dk["gbs"] / NOMINAL_HBM_GBS,
-                     "traffic": profiled_traffic(src, wl.name, wl.b)},
+        "roofline": roofline(dominant),
+        "roofline_write": roofline("quantize_keys"),
+        "roofline_read": roofline("scores"),
         "gpu_launches": 2 * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clock_window,
+        "sustained": sustained,
         "e2e": e2e,
         "decode_step": decode_step,
         "attention": attention,

@@ -108,10 +108,13 @@ def job_scores_per_s(wl: workloads.Workload, world: int, ms_per_step: float) -> 
 
 def kernel_file(kind: str, wl: workloads.Workload) -> str:
     """Source file of the kernel the library runs for this workload (api.cu takes the
-    tensor-core kernels at d = 128, 256 and 512, for the write path with bf16/f16 keys)."""
+    tensor-core kernels at d = 128, 256 and 512, for the write path with bf16/f16 keys;
+    the read path at d = 128 has a kernel of its own)."""
     tc_width = wl.d in (128, 256, 512)
     if kind == "quantize_keys":
         return "quantize_keys_tc.cu" if tc_width and wl.dtype in ("bf16", "f16") else "quantize_keys.cu"
+    if wl.d == 128:
+        return "scores_tc128.cu"
     return "scores_tc.cu" if tc_width else "scores.cu"
 
 

@@ -23,7 +23,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(PKG, "libaxr.so")
 
 SOURCES = ["api.cu", "attention.cu", "codebook.cpp", "quantize_keys.cu", "quantize_keys_block.cu",
-           "quantize_keys_tc.cu", "scores.cu", "scores_tc.cu", "sign_select.cu"]
+           "quantize_keys_tc.cu", "scores.cu", "scores_tc.cu", "scores_tc128.cu", "sign_select.cu"]
 HEADERS = [os.path.join(INCLUDE, "axr.h")] + [
     os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))
 ]

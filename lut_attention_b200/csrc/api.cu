@@ -107,6 +107,19 @@ int device_sm_count()
     return counts[dev];
 }
 
+EncodeTiledFn encode_tiled()
+{
+    static const EncodeTiledFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return static_cast<EncodeTiledFn>(nullptr);
+    }();
+    return fn;
+}
+
 cudaError_t allow_dynamic_smem(const void *kernel, size_t bytes, std::atomic<unsigned long long> &done)
 {
     int dev = 0;

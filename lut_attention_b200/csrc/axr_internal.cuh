@@ -3,6 +3,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "axr.h"
@@ -98,10 +99,14 @@ cudaError_t launch_quantize_keys_tc(const QuantizeArgs &a, cudaStream_t stream);
 unsigned int quantize_tc_status(bool clear);
 cudaError_t launch_scores(const ScoresArgs &a, cudaStream_t stream);
 
-// Tensor-core read path (scores_tc.cu): d = 128.
+// Tensor-core read path: d = 128 (scores_tc128.cu), d = 256 and 512
+// (scores_tc.cu).  scores_tc_* dispatch on d and cover both.
 bool scores_tc_supported(const ScoresArgs &a);
 cudaError_t launch_scores_tc(const ScoresArgs &a, cudaStream_t stream);
 unsigned int scores_tc_status(bool clear);
+bool scores_tc128_supported(const ScoresArgs &a);
+cudaError_t launch_scores_tc128(const ScoresArgs &a, cudaStream_t stream);
+unsigned int scores_tc128_status(bool clear);
 
 // Decode attention after the scores (attention.cu): softmax over each query
 // head's n scores, weighted sum of its KV head's value rows.
@@ -147,6 +152,14 @@ cudaError_t launch_sign_select(const SignSelectArgs &a, cudaStream_t stream);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
+
+// cuTensorMapEncodeTiled from the driver, looked up once; nullptr when the
+// driver does not provide it (the tensor-core kernels are then not used).
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled();
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current
 // device.  The limit belongs to the kernel's instance in each device's context,

@@ -1,32 +1,14 @@
-// Score-on-read on the 5th-generation tensor cores, head dimension 128, 256 or
-// 512 (AXELRAM, arXiv 2604.02638, abstract: scores come from table lookups on
-// the stored indices, never from dequantized keys).  Wider heads run each tile
-// as 2 or 4 subtiles of 128 coordinates into one accumulator (see Cfg); the
-// queries are rotated by the Walsh-Hadamard transform or, for keys written with
-// it, by the IsoQuant block rotation.
+// Score-on-read on the 5th-generation tensor cores, head dimension 256 or 512
+// (AXELRAM, arXiv 2604.02638, abstract: scores come from table lookups on the
+// stored indices, never from dequantized keys).  Each 128-key tile runs as 2 or
+// 4 subtiles of 128 coordinates into one accumulator (see Cfg); the queries are
+// rotated by the Walsh-Hadamard transform or, for keys written with it, by the
+// IsoQuant block rotation.  128-wide heads have their own kernel
+// (scores_tc128.cu); the digits and lookup tables are shared (lut_read.cuh).
 //
-// For the G query heads of a KV head the scores of a tile of 128 keys form one
-// small contraction, s[t][g] = norm_t * sum_j c[idx_t[j]] * q''_g[j], so the
-// lookups feed the tensor cores instead of G FMAs per coordinate:
-//   * every centroid becomes two signed 8-bit digits of a fixed-point number,
-//     c * 128 * S_c = 128 * hi + lo  (|hi| <= 127, |lo| <= 64);
-//   * every rotated query coordinate becomes three signed 8-bit digits,
-//     q'' * S_q = D0 + D1/128 + D2/128^2  (|D| <= 64);
-//   * A (tensor memory) holds the hi and lo digits of the looked-up centroids,
-//     K = 2 * 128; B (shared memory) holds the query digits, N = 4 columns per
-//     query with weights (128, 1, 1/128, 1/128^2):
-//         hi rows (D0, D1, D2, 0),   lo rows (0, D0, D1, D2)
-//     so one kind::i8 product per 32-wide K step yields, for every query,
-//     sum_j q'' c * 128 * S_q * S_c as four exact int32 partial sums.
-// The digit error is at most 0.5 / (128 * 127) of the largest centroid per
-// coordinate, so |score error| <= 8.5e-5 * ||q|| * ||k|| / sqrt(d) in the worst
-// case, inside the 1e-4 the method's tests use; query digits add < 1e-6.
-//
-// Decoding a packed index row into A is a table walk: each lookup takes one
-// field of the row (one byte = 2 codes at b = 4 or 4 codes at b = 2, a 6-bit
-// pair at b = 3, a nibble of 4 codes at b = 1) and reads the digits of all its
-// codes from a table replicated per lane (address = field * 256 + lane * entry
-// size), which is conflict-free in shared memory.
+// The lookups become fixed-point digits that feed an exact int32 tcgen05.mma
+// kind::i8 contraction over a tile of 128 keys and the G queries of a KV head
+// (lut_read.cuh states the digits and their error bound).
 //
 // One CTA per SM, persistent over a contiguous range of 128-key tiles, which it
 // deals round-robin to S tile streams (S = 3 for up to 4 queries per KV head,
@@ -37,11 +19,9 @@
 //                    them by the key norm and the query scale and store the
 //                    scores; then look up tile k's digits and store them to
 //                    A in the same buffer.  On entering a new KV head they
-//                    rotate its queries (sign flip, Walsh-Hadamard
-//                    butterflies, 1/d) and write their digits into the other
-//                    of the stream's two B buffers.  In a decode step they
-//                    first quantize the head's new key when tile k is the
-//                    head's last (the one that holds it).
+//                    wait for the stream's last products, rotate the head's
+//                    queries (sign flip, Walsh-Hadamard butterflies, 1/d) and
+//                    write their digits into the stream's B buffer.
 //   1 MMA warp     : 8 tcgen05.mma (M = 128, N = 4G, K = 32) per tile and one
 //                    commit, which frees A and publishes D at once.
 // plus one TMA warp loading each tile's packed rows and key norms HBM -> shared
@@ -55,6 +35,7 @@
 #include <cuda_runtime.h>
 
 #include "axr_internal.cuh"
+#include "lut_read.cuh"
 #include "quat.cuh"
 #include "sm100.cuh"
 
@@ -62,17 +43,18 @@ namespace axr {
 namespace {
 
 using namespace sm100;
+using lut::kD;
+using lut::kK;
+using lut::kLutBytes;
+using lut::Lookup;
 
-constexpr int kD = 128;
-constexpr float kInvSqrtD = 0.08838834764831845f;   // 1 / sqrt(128), the attention temperature
 constexpr int kTileRows = 128;
-// Stages of packed rows in flight per CTA: 6 at d = 128 (6 tiles), 12 for wider
-// heads, whose tiles take NH stages each.  Stages 0-5 sit in the gap below the
-// lookup table when it holds them (otherwise after it), stages 6-11 after it.
+// Stages of packed rows in flight per CTA: 12, each one slice of a tile (a tile
+// takes NH of them).  Stages 0-5 sit in the gap below the lookup table when it
+// holds them (otherwise after it), stages 6-11 after it.
 constexpr int kStagesMax = 12;
 constexpr int kLowStages = 6;
 constexpr int kGroupThreads = 128;    // worker threads of one stream (one per key of a tile)
-constexpr int kK = 2 * kD;            // two digits per coordinate
 constexpr int kACols = kK / 4;        // tensor-memory columns of one A buffer
 constexpr int kTmemCols = 512;
 // One stage: the packed rows of a tile (P <= 64 bytes each), then its key norms.
@@ -82,23 +64,20 @@ constexpr int kTmemCols = 512;
 constexpr int kStageCodeBytes = kTileRows * 64;
 constexpr int kNormBox = kTileRows + 4;
 constexpr int kStageBytes = kStageCodeBytes + 1024;   // keeps every stage 512-byte aligned
-constexpr int kLutBytes = 256 * 256;          // up to 256 fields x 256 bytes
 constexpr int kInvSlots = 8;          // per-stream ring of query scales, one slot per head
 constexpr int kBBytesMax = 32 * kK;   // one B buffer at most: 8 queries x 4 digit rows x K bytes
 
 // launch shape for NQ query columns per KV head (G <= NQ) and head dimension
-// 128 * NH.  A tile of 128 keys is processed as NH subtiles of 128 coordinates
-// (one stage, one A buffer and one K = 256 block of B each) accumulating into one
-// D.  At NH = 1 each stream double-buffers B (the next head's digits are written
-// while the last head's products run); wider heads keep one B buffer per stream
-// (shared memory), and the streams wait for their products before a new head.
+// 128 * NH (NH = 2 or 4).  A tile of 128 keys is processed as NH subtiles of 128
+// coordinates (one stage, one A buffer and one K = 256 block of B each)
+// accumulating into one D.  Each stream keeps one B buffer (shared memory), and
+// waits for its products before writing a new head's digits.
 template <int NQ, int NH>
 struct Cfg {
+    static_assert(NH == 2 || NH == 4, "128-wide heads run in scores_tc128.cu");
     static constexpr int N = 4 * NQ;                  // B rows = D columns
-    static constexpr int S = (NH == 1) ? ((NQ <= 4) ? 3 : 2)
-                           : (NH == 2) ? ((NQ <= 4) ? 3 : 2)
-                                       : ((NQ <= 4) ? 2 : 1);   // tile streams
-    static constexpr int kBBufs = (NH == 1) ? 2 : 1;  // B buffers per stream
+    static constexpr int S = (NH == 2) ? ((NQ <= 4) ? 3 : 2) : ((NQ <= 4) ? 2 : 1);   // tile streams
+    static constexpr int kBBufs = 1;                  // B buffers per stream
     static constexpr int kWorkerWarps = 4 * S;
     static constexpr int kWarpTma = kWorkerWarps;
     static constexpr int kWarpMma0 = kWorkerWarps + 1;
@@ -106,29 +85,14 @@ struct Cfg {
     static constexpr int kDOff = S * 2 * kACols;      // A buffers first, then D buffers
     static constexpr int kSliceB = N * kK;            // B bytes of one subtile's K block
     static constexpr int kBBytes = kSliceB * NH;      // one B buffer
-    static constexpr int kStages = (NH == 1) ? kLowStages : kStagesMax;
+    static constexpr int kStages = kStagesMax;
     static_assert(kStages % S == 0, "streams must own whole stages");
     static_assert(kDOff + S * 2 * N <= kTmemCols, "tensor memory budget");
     static_assert(kSliceB <= kBBytesMax, "B buffer");
-    static_assert(NH == 1 || kBBytes >= NQ * kD * NH * 4, "a wide head's B buffer holds its rotation scratch");
+    static_assert(kBBytes >= NQ * kD * NH * 4, "a wide head's B buffer holds its rotation scratch");
 };
 
 __device__ unsigned int g_status;
-
-// geometry of one lookup for b bits: C codes per lookup, FB field bits
-template <int B>
-struct Lookup {
-    static constexpr int C = (B >= 3) ? 2 : 4;
-    static constexpr int FB = C * B;              // 8, 6, 8, 4
-    static constexpr int EB = 2 * C;              // entry bytes: C hi digits, C lo digits
-    static constexpr int NF = 1 << FB;            // table fields
-    // b = 3: the table is indexed by a whole byte, and a second one sits in the
-    // unused upper half of every 256-byte row (lane offsets 128 + 4 lane):
-    // the first reads the 6-bit field in bits 0..5 of the byte, the second in
-    // bits 2..7, so a field that starts 0 or 2 bits into a byte costs one PRMT
-    static constexpr bool kByteTables = (B == 3);
-    static constexpr int kRows = kByteTables ? 256 : NF;
-};
 
 struct TcParams {
     CUtensorMap tmap;          // packed rows as a [heads*n, P] byte tensor, box P x 128
@@ -148,14 +112,6 @@ struct TcParams {
     float inv_sc;              // 1 / (128 * S_c)
     int8_t hi[kMaxLevels];     // centroid digits
     int8_t lo[kMaxLevels];
-    // decode step: the key of KV head h in k_new (heads x 128, kdtype) is quantized
-    // into row append_pos of that head (the last key scored) before it is read
-    int append_pos;            // -1: no key to append
-    int kdtype;
-    const void *k_new;
-    uint8_t *idx_out;          // the packed rows and norms, writable
-    float *norms_out;
-    float bnd[kMaxLevels - 1]; // codebook decision boundaries (unit-vector scale)
 };
 
 constexpr int kMaxStreams = 3;
@@ -168,21 +124,10 @@ struct Smem {
     uint64_t wsync[kMaxStreams];       // the threads of one stream (query rotation steps)
     uint32_t tmem_base;
     float inv[kMaxStreams][kInvSlots][8];   // per stream, head slot and query: 1 / (128 * S_q * S_c)
-    float q[2048];                           // rotation scratch: S * NQ <= 16 query rows of d floats
     float qmax[kMaxStreams][4][8];           // per stream, warp and query: max |q''|
-    uint32_t arow[kMaxStreams][17];          // per stream: packed row of an appended key
 };
 constexpr int kSmemBook = 10240;
 static_assert(sizeof(Smem) <= kSmemBook, "bookkeeping area too small");
-
-__device__ __forceinline__ float load_q(const void *q, int dtype, int64_t i)
-{
-    switch (dtype) {
-    case AXR_F32: return static_cast<const float *>(q)[i];
-    case AXR_F16: return __half2float(static_cast<const __half *>(q)[i]);
-    default: return __bfloat162float(static_cast<const __nv_bfloat16 *>(q)[i]);
-    }
-}
 
 // bounded barrier of the threads of stream g; `phase` counts the syncs so far
 __device__ __forceinline__ bool stream_sync(Smem &S, int g, int &phase)
@@ -193,27 +138,19 @@ __device__ __forceinline__ bool stream_sync(Smem &S, int g, int &phase)
     return ok;
 }
 
-// B offset of element (n, k) in the no-swizzle K-major layout: 8-row x 16-byte
-// core matrices, K-adjacent ones 128 bytes apart, N-adjacent ones kK*8 bytes apart
-__device__ __forceinline__ int b_offset(int n, int k)
-{
-    return ((n >> 3) * (kK / 16) + (k >> 4)) * 128 + (n & 7) * 16 + (k & 15);
-}
-
 // Rotate the G queries of KV head h and write their digits into B buffer `b`
 // of stream g (the stream's 128 threads; thread j owns coordinates j + 128 l of
 // the NH slices l).  Slice l's digits form their own K = 256 block of B, at
-// l * N * kK bytes.  The rotation works in S.q at d = 128; for wider heads the
-// B buffer itself is the scratch (it is free, and every byte of it is written
-// with digits only after the last read of the rotated values).
+// l * N * kK bytes.  The B buffer itself is the rotation scratch (it is free,
+// and every byte of it is written with digits only after the last read of the
+// rotated values).
 template <int B, int NQ, int NH>
 __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *inv, int h, int &phase)
 {
-    using LK = Lookup<B>;
     constexpr int D = kD * NH;
     constexpr int kSliceB = 4 * NQ * kK;        // bytes of one slice's digits (N rows x K)
     const int tid = threadIdx.x & (kGroupThreads - 1);
-    float(*q)[D] = reinterpret_cast<float(*)[D]>(NH == 1 ? S.q + g * NQ * kD : reinterpret_cast<float *>(b));
+    float(*q)[D] = reinterpret_cast<float(*)[D]>(b);
 #pragma unroll
     for (int sl = 0; sl < NH; ++sl) {
         const int j = tid + kD * sl;
@@ -221,7 +158,7 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
 #pragma unroll
         for (int qi = 0; qi < NQ; ++qi)
             q[qi][j] = (qi < p.group)
-                           ? sg * load_q(p.q, p.qdtype, (static_cast<int64_t>(h) * p.group + qi) * D + j)
+                           ? sg * lut::load_q(p.q, p.qdtype, (static_cast<int64_t>(h) * p.group + qi) * D + j)
                            : 0.0f;
     }
     if (!stream_sync(S, g, phase)) return false;
@@ -229,7 +166,7 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
     if (p.quats) {
         // q'' = T q / sqrt(d): the IsoQuant block rotation T (orthonormal) times the
         // temperature; each coordinate from its 4-element block
-        const float inv_sqrt_d = (NH == 1) ? kInvSqrtD : 1.0f / sqrtf(static_cast<float>(D));
+        const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
 #pragma unroll
         for (int sl = 0; sl < NH; ++sl) {
             const int j = tid + kD * sl;
@@ -270,9 +207,9 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
         if ((tid & 31) == 0) S.qmax[g][tid >> 5][qi] = m;
     }
     if (!stream_sync(S, g, phase)) return false;
-    // this coordinate's hi and lo K rows: lookup l = j / C covers K indices EB*l ..
-    const int l = tid / LK::C, t = tid % LK::C;
-    const int k_hi = LK::EB * l + t, k_lo = LK::EB * l + LK::C + t;
+    // this coordinate's hi and lo K rows (the same in every slice)
+    int k_hi, k_lo;
+    lut::digit_rows<B>(tid, k_hi, k_lo);
 #pragma unroll
     for (int qi = 0; qi < NQ; ++qi) {
         float m = 0.0f;
@@ -282,99 +219,11 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
         if (tid == 0) inv[qi] = p.inv_sc / sq;
 #pragma unroll
         for (int sl = 0; sl < NH; ++sl) {
-            uint8_t *bs = b + sl * kSliceB;
-            const float Q = qq[qi][sl] * sq;                  // |Q| <= 64
-            const float d0 = rintf(Q);
-            const float r1 = (Q - d0) * 128.0f;
-            const float d1 = rintf(r1);
-            const float d2 = rintf((r1 - d1) * 128.0f);
-            const uint8_t D0 = static_cast<uint8_t>(static_cast<int8_t>(d0));
-            const uint8_t D1 = static_cast<uint8_t>(static_cast<int8_t>(d1));
-            const uint8_t D2 = static_cast<uint8_t>(static_cast<int8_t>(d2));
-            // column weights (128, 1, 1/128, 1/128^2): hi rows (D0, D1, D2, 0), lo rows (0, D0, D1, D2)
-            bs[b_offset(4 * qi + 0, k_hi)] = D0;
-            bs[b_offset(4 * qi + 1, k_hi)] = D1;
-            bs[b_offset(4 * qi + 2, k_hi)] = D2;
-            bs[b_offset(4 * qi + 3, k_hi)] = 0;
-            bs[b_offset(4 * qi + 0, k_lo)] = 0;
-            bs[b_offset(4 * qi + 1, k_lo)] = D0;
-            bs[b_offset(4 * qi + 2, k_lo)] = D1;
-            bs[b_offset(4 * qi + 3, k_lo)] = D2;
+            lut::write_query_digits(b + sl * kSliceB, qi, k_hi, k_lo, qq[qi][sl] * sq);   // |Q| <= 64
         }
     }
     fence_proxy_async_smem();
     return stream_sync(S, g, phase);
-}
-
-// Decode step: quantize the appended key of KV head h, exactly as the write path
-// defines it (sign flip, Walsh-Hadamard, norm, nearest centroid, packing), with
-// the stream's 128 threads (thread j owns coordinate j).  Stores its codes and
-// norm in the cache and leaves the packed row in S.arow[g] and the norm in *norm.
-template <int B, int NQ>
-__device__ bool append_key(const TcParams &p, Smem &S, int g, int h, float *norm, int &phase)
-{
-    constexpr int P = kD * B / 8;
-    constexpr int L = 1 << B;
-    const int tid = threadIdx.x & (kGroupThreads - 1);
-    float *y = S.q + g * NQ * kD;
-    const float x = (p.signs[tid] < 0 ? -1.0f : 1.0f) *
-                    load_q(p.k_new, p.kdtype, static_cast<int64_t>(h) * kD + tid);
-    y[tid] = x;
-    float ss = x * x;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if ((tid & 31) == 0) S.qmax[g][tid >> 5][0] = ss;
-    if (tid <= P / 4) S.arow[g][tid] = 0u;
-    if (!stream_sync(S, g, phase)) return false;
-    for (int hh = 1; hh < kD; hh <<= 1) {
-        if (tid < kD / 2) {
-            const int i = (tid / hh) * 2 * hh + (tid % hh);
-            const float a = y[i], c = y[i + hh];
-            y[i] = a + c;
-            y[i + hh] = a - c;
-        }
-        if (!stream_sync(S, g, phase)) return false;
-    }
-    const float nk = sqrtf((S.qmax[g][0][0] + S.qmax[g][1][0]) + (S.qmax[g][2][0] + S.qmax[g][3][0]));
-    // u = y / (sqrt(d) ||k||); idx = number of boundaries below u (a zero key has
-    // u = 0 and takes the central index)
-    const float u = (nk > 0.0f) ? y[tid] / (sqrtf(static_cast<float>(kD)) * nk) : 0.0f;
-    uint32_t code = 0;
-#pragma unroll
-    for (int i = 0; i < L - 1; ++i) code += (u > p.bnd[i]) ? 1u : 0u;
-    const int bit = tid * B;
-    atomicOr(&S.arow[g][bit >> 5], code << (bit & 31));
-    if ((bit & 31) + B > 32) atomicOr(&S.arow[g][(bit >> 5) + 1], code >> (32 - (bit & 31)));
-    if (!stream_sync(S, g, phase)) return false;
-    const int64_t row = static_cast<int64_t>(h) * p.head_stride + p.append_pos;
-    if (tid < P / 4) reinterpret_cast<uint32_t *>(p.idx_out + row * P)[tid] = S.arow[g][tid];
-    if (tid == 0) p.norms_out[row] = nk;
-    *norm = nk;
-    return true;
-}
-
-// table entry of one field value: C hi digits then C lo digits, replicated for
-// the 32 lanes (entry (field, lane) at field * 256 + lane * EB)
-template <int B, int kWorkers>
-__device__ void build_lut(const TcParams &p, uint8_t *lut)
-{
-    using LK = Lookup<B>;
-    constexpr uint32_t mask = (1u << B) - 1u;
-    constexpr int kTables = LK::kByteTables ? 2 : 1;
-    for (int e = threadIdx.x; e < LK::kRows * 32 * kTables; e += kWorkers) {
-        const int row = e / (32 * kTables), ln = e % 32, tab = (e / 32) % kTables;
-        const int field = LK::kByteTables ? ((tab == 0) ? (row & (LK::NF - 1)) : (row >> 2)) : row;
-        uint8_t bytes[LK::EB];
-#pragma unroll
-        for (int i = 0; i < LK::C; ++i) {
-            const int code = (field >> (B * i)) & mask;
-            bytes[i] = static_cast<uint8_t>(p.hi[code]);
-            bytes[LK::C + i] = static_cast<uint8_t>(p.lo[code]);
-        }
-        uint8_t *dst = lut + row * 256 + tab * 128 + ln * LK::EB;
-#pragma unroll
-        for (int i = 0; i < LK::EB; ++i) dst[i] = bytes[i];
-    }
 }
 
 // byte offset of 16-byte chunk c of tile row r in a stage, with the swizzle
@@ -385,38 +234,6 @@ __device__ __forceinline__ int chunk_offset(int r, int c)
     if constexpr (P == 64) return r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
     else if constexpr (P == 32) return r * 32 + ((c ^ ((r >> 2) & 1)) << 4);
     else return r * P + (c << 4);
-}
-
-// shared-memory address of the table entry for lookup l of a row held in w[].
-// base_lane = table base (64 KB aligned) | lane * entry size, so the field
-// only has to be placed in bits 8.. of it: one PRMT for byte fields (and, at
-// b = 3, for fields starting 0 or 2 bits into a byte), a shift and one LOP3
-// otherwise.
-template <int B>
-__device__ __forceinline__ uint32_t lut_addr(const uint32_t *w, int l, uint32_t base_lane)
-{
-    using LK = Lookup<B>;
-    const int bit = l * LK::FB;
-    const int wi = bit >> 5, sh = bit & 31;
-    if constexpr (LK::FB == 8) {
-        // bytes: [lane offset, field, table base bits 16..23, 24..31]
-        const uint32_t sel = 0x7604u | (static_cast<uint32_t>(sh >> 3) << 4);
-        return __byte_perm(w[wi], base_lane, sel);
-    } else if (LK::kByteTables && ((sh & 7) == 0 || (sh & 7) == 2)) {
-        // the byte holding the field indexes the first table (field in bits
-        // 0..5) or the second (bits 2..7, lane offsets + 128)
-        const uint32_t sel = 0x7604u | (static_cast<uint32_t>(sh >> 3) << 4);
-        return __byte_perm(w[wi], (sh & 7) == 0 ? base_lane : (base_lane | 128u), sel);
-    } else {
-        constexpr uint32_t fmask = ((1u << LK::FB) - 1u) << 8;
-        uint32_t x;
-        if (sh >= 8) {
-            x = (sh + LK::FB <= 32) ? (w[wi] >> (sh - 8)) : __funnelshift_r(w[wi], w[wi + 1], sh - 8);
-        } else {
-            x = w[wi] << (8 - sh);
-        }
-        return (x & fmask) | base_lane;
-    }
 }
 
 // Dynamic shared memory: the table on a 64 KB boundary of the shared window
@@ -445,8 +262,7 @@ constexpr bool b_fits()
 {
     return Cfg<NQ, NH>::S * Cfg<NQ, NH>::kBBufs * Cfg<NQ, NH>::kBBytes <= kBRegion;
 }
-static_assert(b_fits<4, 1>() && b_fits<8, 1>() && b_fits<4, 2>() && b_fits<8, 2>() && b_fits<4, 4>() &&
-                  b_fits<8, 4>(),
+static_assert(b_fits<4, 2>() && b_fits<8, 2>() && b_fits<4, 4>() && b_fits<8, 4>(),
               "B buffers of every stream fit");
 
 // Worker threads of tile stream g (local tiles k = 0, 1, ... are the CTA's
@@ -567,18 +383,14 @@ struct Worker {
                         store_sums(p, S, g, acc, nk2, hs2, h2, t2k + r, inv_hc, inv);
                     }
                     if (h != prev_h) {
-                        if constexpr (C::kBBufs == 1) {
-                            // one B buffer: the last head's products must be done with it
-                            if (m >= 1 && !mbar_wait_warp(smem_u32(&S.mma_done[g][(m - 1) & 1]), ((m - 1) >> 1) & 1)) {
-                                if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after_sync();
-                            bsel = 0;
-                        } else {
-                            bsel = (bsel < 0) ? 0 : (bsel ^ 1);
+                        // one B buffer: the last head's products must be done with it
+                        if (m >= 1 && !mbar_wait_warp(smem_u32(&S.mma_done[g][(m - 1) & 1]), ((m - 1) >> 1) & 1)) {
+                            if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                            ok = false;
+                            break;
                         }
+                        tc_fence_after_sync();
+                        bsel = 0;
                         prev_h = h;
                         ++hc;
                         if (!build_b<B, NQ, NH>(p, S, g, sB + (C::kBBufs * g + bsel) * C::kBBytes,
@@ -586,23 +398,6 @@ struct Worker {
                             if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
                             ok = false;
                             break;
-                        }
-                    }
-                    // decode step: this head's last tile holds the appended key, whose row
-                    // the stage has only as it was before this launch
-                    if constexpr (NH == 1) {
-                        if (p.append_pos >= 0 && ti == (p.append_pos >> 7)) {
-                            float nka;
-                            if (!append_key<B, NQ>(p, S, g, h, &nka, sync_phase)) {
-                                if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
-                                ok = false;
-                                break;
-                            }
-                            if (r == (p.append_pos & (kTileRows - 1))) {
-#pragma unroll
-                                for (int i = 0; i < NW; ++i) w[i] = S.arow[g][i];
-                                nk = nka;
-                            }
                         }
                     }
                 }
@@ -615,13 +410,13 @@ struct Worker {
                     if constexpr (LK::EB == 4) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const uint32_t ad = lut_addr<B>(w, 16 * qt + i, base_lane);
+                            const uint32_t ad = lut::lut_addr<B>(w, 16 * qt + i, base_lane);
                             asm("ld.shared.u32 %0, [%1];" : "=r"(a[i]) : "r"(ad));
                         }
                     } else {
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            const uint32_t ad = lut_addr<B>(w, 8 * qt + i, base_lane);
+                            const uint32_t ad = lut::lut_addr<B>(w, 8 * qt + i, base_lane);
                             asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a[2 * i]), "=r"(a[2 * i + 1]) : "r"(ad));
                         }
                     }
@@ -630,13 +425,6 @@ struct Worker {
                 tmem_wait_st();
                 tc_fence_before_sync();
                 mbar_arrive(smem_u32(&S.a_full[g][ab]));
-                if constexpr (NH == 1) {
-                    s += C::S;
-                    if (s >= C::kStages) {
-                        s -= C::kStages;
-                        sph ^= 1;
-                    }
-                }
             }
             if (!ok) break;
 
@@ -722,7 +510,7 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
         prefetch_tensormap(&p.tmap);
         prefetch_tensormap(&p.nmap);
     }
-    if (warp < C::kWorkerWarps) build_lut<B, C::kWorkerWarps * 32>(p, sLut);
+    if (warp < C::kWorkerWarps) lut::build_lut<B>(p.hi, p.lo, sLut, threadIdx.x, C::kWorkerWarps * 32);
     if (warp == 0) {
         tmem_alloc(smem_u32(&S.tmem_base), kTmemCols);
         tmem_relinquish();
@@ -836,24 +624,6 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
 
 // ------------------------------------------------------------------ host side
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                   CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
 template <int B, int NQ, int NH>
 cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
 {
@@ -900,30 +670,13 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     p.scores = a.scores;
     p.n = static_cast<int>(a.n);
     p.head_stride = static_cast<int>(a.head_stride);
-    p.append_pos = a.k_new ? static_cast<int>(a.append_pos) : -1;
-    p.kdtype = a.kdtype;
-    p.k_new = a.k_new;
-    p.idx_out = a.idx_out;
-    p.norms_out = a.norms_out;
-    for (int i = 0; i < kMaxLevels - 1; ++i) p.bnd[i] = a.cb.boundaries[i];
     p.group = a.group;
     p.tiles_per_head = static_cast<int>((a.n + kTileRows - 1) / kTileRows);
     p.total_tiles = p.tiles_per_head * a.heads;
     const int sms = device_sm_count();
     const int grid = p.total_tiles < sms ? p.total_tiles : sms;
     p.tiles_per_cta = (p.total_tiles + grid - 1) / grid;
-    // centroid digits: c * 128 * S_c = 128 * hi + lo, S_c = 127 / max |c|
-    const int L = 1 << a.b;
-    const float cmax = fabsf(a.cb.centroids[L - 1]);
-    const double sc = 127.0 / cmax;
-    p.inv_sc = static_cast<float>(1.0 / (128.0 * sc));
-    for (int i = 0; i < kMaxLevels; ++i) {
-        const double v = (i < L) ? a.cb.centroids[i] * 128.0 * sc : 0.0;
-        const long vi = lrint(v);
-        const long hi = lrint(static_cast<double>(vi) / 128.0);
-        p.hi[i] = static_cast<int8_t>(hi);
-        p.lo[i] = static_cast<int8_t>(vi - 128 * hi);
-    }
+    lut::centroid_digits(a.cb, p.hi, p.lo, &p.inv_sc);
     const int used = (p.total_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
     kernel<<<used, Cfg<NQ, NH>::kThreads, smem, stream>>>(p);
     return cudaGetLastError();
@@ -950,9 +703,10 @@ cudaError_t launch_h(const ScoresArgs &a, cudaStream_t stream)
 
 bool scores_tc_supported(const ScoresArgs &a)
 {
+    if (a.d == kD) return scores_tc128_supported(a);
     // d = 256 and 512 run as 2 and 4 slices of 128 coordinates; the fused decode
     // step (one appended key quantized in the kernel) exists for d = 128 only
-    const bool width = a.d == kD || ((a.d == 2 * kD || a.d == 4 * kD) && a.k_new == nullptr);
+    const bool width = (a.d == 2 * kD || a.d == 4 * kD) && a.k_new == nullptr;
     return width && a.b >= 1 && a.b <= 4 && a.group <= 8 && a.n > 0 &&
            static_cast<int64_t>(a.heads) * a.head_stride < (static_cast<int64_t>(1) << 31) - kTileRows &&
            encode_tiled() != nullptr;
@@ -963,7 +717,7 @@ cudaError_t launch_scores_tc(const ScoresArgs &a, cudaStream_t stream)
     switch (a.d) {
     case 2 * kD: return launch_h<2>(a, stream);
     case 4 * kD: return launch_h<4>(a, stream);
-    default: return launch_h<1>(a, stream);
+    default: return launch_scores_tc128(a, stream);
     }
 }
 
@@ -975,7 +729,7 @@ unsigned int scores_tc_status(bool clear)
         const unsigned int z = 0;
         cudaMemcpyToSymbol(g_status, &z, sizeof(z));
     }
-    return v;
+    return v | scores_tc128_status(clear);
 }
 
 }  // namespace axr

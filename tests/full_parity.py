@@ -138,11 +138,11 @@ def _check_chunk(K: np.ndarray, g_idx: np.ndarray, g_norms: np.ndarray, g_scores
 
 
 def sample_tokens(T: int, per_head: int, seed: int, h: int) -> torch.Tensor:
-    """First, last and seeded random tokens of one KV head, sorted and distinct."""
+    """First, last and per_head other seeded tokens of one KV head (drawn without
+    replacement), sorted and distinct."""
     g = torch.Generator(device="cpu").manual_seed(seed * 100_003 + h)
-    pick = torch.randint(0, T, (per_head,), generator=g)
-    pick = torch.cat([pick, torch.tensor([0, T - 1])])
-    return torch.unique(pick)
+    pick = torch.randperm(T - 2, generator=g)[:per_head] + 1
+    return torch.unique(torch.cat([pick, torch.tensor([0, T - 1])]))
 
 
 def run(wl: workloads.Workload, device, min_rows: int | None = None) -> FullReport:

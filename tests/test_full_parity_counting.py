@@ -53,6 +53,6 @@ def test_planted_changes_are_counted(oracle_lib):
 
 
 def test_sample_tokens_hold_first_and_last():
-    tok = full_parity.sample_tokens(65536, 100, seed=5, h=3)
-    assert tok[0] == 0 and tok[-1] == 65535
+    tok = full_parity.sample_tokens(65536, 8192, seed=5, h=3)
+    assert tok[0] == 0 and tok[-1] == 65535 and len(tok) == 8192 + 2
     assert bool((tok[1:] > tok[:-1]).all())

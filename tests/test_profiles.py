@@ -28,9 +28,24 @@ def test_default_workload_kernels_have_current_traffic():
         assert 0.85 * algorithmic <= traffic <= 1.02 * algorithmic, (src, traffic, algorithmic)
 
 
+def test_traffic_lines_carry_the_hash_they_were_captured_on():
+    """Every line of profiles/traffic.txt names the source hash listed on its
+    `# captured:` line: a line is never relabelled to a later source."""
+    text = open(os.path.join(ROOT, "profiles", "traffic.txt")).read()
+    cap = [ln for ln in text.splitlines() if ln.startswith("# captured:")]
+    assert len(cap) == 1, "traffic.txt needs exactly one '# captured:' line"
+    words = cap[0].split(":", 1)[1].split()
+    captured = dict(zip(words[0::2], words[1::2]))
+    lines = [ln.split() for ln in text.splitlines() if ln.strip() and not ln.startswith("#")]
+    assert lines
+    for parts in lines:
+        assert len(parts) == 5, parts
+        assert parts[0] in captured and parts[3] == captured[parts[0]], parts
+
+
 def test_kernel_files_follow_the_library_dispatch():
     assert bench.kernel_file("quantize_keys", workloads.GQA_DECODE_128K) == "quantize_keys_tc.cu"
-    assert bench.kernel_file("scores", workloads.GQA_DECODE_128K) == "scores_tc.cu"
+    assert bench.kernel_file("scores", workloads.GQA_DECODE_128K) == "scores_tc128.cu"
     assert bench.kernel_file("quantize_keys", workloads.WIDE_D512) == "quantize_keys_tc.cu"
     assert bench.kernel_file("scores", workloads.WIDE_D256) == "scores_tc.cu"
     assert bench.kernel_file("quantize_keys", workloads.PR1_REF) == "quantize_keys.cu"     # fp32 keys
@@ -42,5 +57,20 @@ def test_profile_summaries_name_existing_sources_and_commands():
         text = open(os.path.join(ROOT, "profiles", name)).read()
         for src in set(re.findall(r"\b([a-z_]+\.cu)\b", text)):
             assert os.path.exists(os.path.join(csrc, src)), (name, src)
-        if name.endswith(".md"):
-            assert "--clock-control none" in text, f"{name}: the ncu command is missing or locks clocks"
+        if name.endswith(".md") and "ncu" in text:
+            for cmd in re.findall(r"^\s*ncu --.*$", text, flags=re.M):
+                assert "--clock-control none" in cmd, f"{name}: an ncu command locks clocks"
+            assert re.search(r"^\s*ncu --.*$", text, flags=re.M), f"{name}: the ncu command is missing"
+
+
+def test_full_size_parity_report_is_of_the_current_kernels():
+    """profiles/parity_full_size.md (the every-row comparison with the oracle) was
+    produced by the current write and read kernel sources."""
+    text = open(os.path.join(ROOT, "profiles", "parity_full_size.md")).read()
+    line = [ln for ln in text.splitlines() if ln.startswith("sources: ")]
+    assert len(line) == 1
+    words = line[0].split()[1:]
+    recorded = dict(zip(words[0::2], words[1::2]))
+    assert set(recorded) == {"quantize_keys_tc.cu", "quantize_keys.cu", "scores_tc128.cu", "scores_tc.cu"}
+    for src, h in recorded.items():
+        assert bench.kernel_source_hash(src) == h, f"{src} changed since the full-size parity run"

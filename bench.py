@@ -588,6 +588,9 @@ def main():
     ap.add_argument("--impl", choices=["axr", "reference"], default="axr")
     ap.add_argument("--workload", default="gqa_decode_128k", choices=sorted(workloads.BY_NAME))
     ap.add_argument("--b", type=int, default=None, help="bits per coordinate (default: the workload's)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="keys per KV head instead of the workload's context: a reduced case for profiler "
+                         "captures (its line is not the workload's figure and carries no profiled traffic)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--sustain-seconds", type=float, default=1.5,
                     help="length of the extra window of steps timed after the K steps (0: none)")
@@ -602,6 +605,8 @@ def main():
     base = workloads.BY_NAME[args.workload]
     if args.b is not None:
         base = base.with_(b=args.b)
+    if args.tokens is not None:
+        base = base.with_(T=args.tokens)
 
     if args.impl == "reference":
         reference_arm(args, base, world, rank)
@@ -696,7 +701,8 @@ def main():
         src = kernel_file(kind, wl)
         return {"bound": "hbm", "kernel": kind, "source": src, "achieved": k["gbs"], "peak": peak,
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": k["gbs"] / peak,
-                "frac_of_8tbs": k["gbs"] / NOMINAL_HBM_GBS, "traffic": profiled_traffic(src, wl.name, wl.b)}
+                "frac_of_8tbs": k["gbs"] / NOMINAL_HBM_GBS,
+                "traffic": None if args.tokens is not None else profiled_traffic(src, wl.name, wl.b)}
 
     if sustained is not None:
         mhz = sustained["clocks"].get("sm_mhz")

@@ -259,16 +259,34 @@ int axr_select_signs(const void *K, int kdtype, const void *q, int qdtype, int64
                      int32_t *best, axr_stream stream);
 
 /*
- * Device-side status of the tensor-core kernels (no counterpart in the method;
- * a diagnostic).  Every wait inside those kernels is bounded; a wait that runs
- * out records a bit here instead of hanging: 1 = a tile load never arrived,
+ * Device-side status of the kernels (no counterpart in the method; a
+ * diagnostic).  Every wait inside the tensor-core kernels is bounded; a wait that
+ * runs out records a bit here instead of hanging: 1 = a tile load never arrived,
  * 2 = a matrix product never completed, 4 = an accumulator was never released;
  * 8 = the read kernel found its shared-memory window laid out so that its stages
- * do not fit, and scored nothing.
+ * do not fit, and scored nothing.  In the debug build (libaxr_debug.so) every
+ * kernel also checks each plain global load and store against the buffer the
+ * call's arguments describe, skips one that falls outside (a load reads zeros)
+ * and records 16.
  * Synchronizes the current device, writes the OR of the recorded bits to
  * *status (0 = none) and clears them if `clear` is non-zero.
  */
 int axr_device_status(int clear, unsigned int *status);
+
+/* 1 in the debug build (libaxr_debug.so, compiled with AXR_DEBUG: device-side
+ * bounds checks, status bit 16), 0 in the release build (libaxr.so). */
+int axr_debug_build(void);
+
+/*
+ * Debug build only: shorten, for every later launch, each buffer span the bounds
+ * checks allow by `bytes` (>= 0; 0 restores the exact spans), so that the last
+ * accesses of every buffer count as outside and are skipped with status bit 16
+ * although they lie in the real allocation.  For testing that the checks fire
+ * without any access leaving its buffer.  Process-wide, not thread-safe against
+ * concurrent launches.  AXR_EINVAL for bytes < 0; AXR_EUNSUPPORTED in the
+ * release build.
+ */
+int axr_debug_set_span_slack(int64_t bytes);
 
 /* Static string naming a status code. */
 const char *axr_status_string(int status);

@@ -11,6 +11,8 @@ from .axr import (  # noqa: F401
     axr_attention,
     axr_attention_static,
     axr_attention_workspace_bytes,
+    axr_debug_build,
+    axr_debug_set_span_slack,
     axr_device_status,
     axr_make_codebook,
     axr_quantize_keys,
@@ -28,6 +30,8 @@ __all__ = [
     "axr_attention",
     "axr_attention_static",
     "axr_attention_workspace_bytes",
+    "axr_debug_build",
+    "axr_debug_set_span_slack",
     "axr_device_status",
     "axr_make_codebook",
     "axr_quantize_keys",

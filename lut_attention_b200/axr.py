@@ -15,7 +15,9 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libaxr.so")
+# AXR_DEBUG=1 selects the debug build (device-side bounds checks, status bit 16)
+DEBUG = os.environ.get("AXR_DEBUG", "") == "1"
+LIB_PATH = os.path.join(_HERE, "libaxr_debug.so" if DEBUG else "libaxr.so")
 
 AXR_OK, AXR_EINVAL, AXR_EUNSUPPORTED, AXR_ECUDA = 0, -1, -2, -3
 AXR_F32, AXR_F16, AXR_BF16 = 0, 1, 2
@@ -38,6 +40,8 @@ SIGNATURES = {
     "axr_last_error": (ctypes.c_char_p, []),
     "axr_version": (_I32, []),
     "axr_device_status": (_I32, [_I32, _P]),
+    "axr_debug_build": (_I32, []),
+    "axr_debug_set_span_slack": (_I32, [_I64]),
 }
 
 _lock = threading.Lock()
@@ -57,8 +61,8 @@ def library() -> ctypes.CDLL:
         if _lib is None:
             if not os.path.exists(LIB_PATH):
                 raise RuntimeError(
-                    f"libaxr.so is missing at {LIB_PATH}: build it with "
-                    "`python -m lut_attention_b200.build` (needs nvcc)")
+                    f"{os.path.basename(LIB_PATH)} is missing at {LIB_PATH}: build it with "
+                    f"`python -m lut_attention_b200.build{' --debug' if DEBUG else ''}` (needs nvcc)")
             lib = ctypes.CDLL(LIB_PATH)
             for name, (res, args) in SIGNATURES.items():
                 fn = getattr(lib, name)
@@ -399,7 +403,20 @@ def axr_select_signs(K: torch.Tensor, q: torch.Tensor, group: int, b: int, candi
 
 
 def axr_device_status(clear: bool = True) -> int:
-    """Bits recorded by a bounded wait that ran out in a tensor-core kernel (0 = none)."""
+    """Bits recorded on the device (0 = none): 1, 2, 4 a bounded wait that ran out
+    in a tensor-core kernel, 8 a read kernel whose stages did not fit, 16 (debug
+    build only) a load or store outside its buffer, skipped."""
     out = ctypes.c_uint(0)
     _raise(library().axr_device_status(1 if clear else 0, ctypes.byref(out)), "axr_device_status")
     return out.value
+
+
+def axr_debug_build() -> bool:
+    """True when the loaded library is the debug build (libaxr_debug.so)."""
+    return bool(library().axr_debug_build())
+
+
+def axr_debug_set_span_slack(nbytes: int) -> None:
+    """Debug build: shorten every buffer span the bounds checks allow by nbytes
+    (0 restores them); raises in the release build."""
+    _raise(library().axr_debug_set_span_slack(int(nbytes)), "axr_debug_set_span_slack")

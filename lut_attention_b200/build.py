@@ -1,10 +1,16 @@
 """Build libaxr.so in-tree with nvcc for sm_100a.
 
-    python -m lut_attention_b200.build [--force] [--ptxas-verbose]
+    python -m lut_attention_b200.build [--force] [--ptxas-verbose] [--debug]
 
 Each source compiles to an object under ``_build/`` (in parallel), then nvcc
 links them into ``lut_attention_b200/libaxr.so`` with the CUDA runtime linked
 statically, so the library does not depend on which libcudart PyTorch loads.
+
+``--debug`` builds ``lut_attention_b200/libaxr_debug.so`` from the same sources
+with ``-DAXR_DEBUG`` (objects under ``_build/debug/``): every kernel then
+checks its plain global loads and stores against the buffers the call
+describes and records status bit 16 instead of making one that falls outside.
+The binding loads it instead of libaxr.so when ``AXR_DEBUG=1`` is set.
 """
 from __future__ import annotations
 
@@ -21,6 +27,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(PKG, "libaxr.so")
+DEBUG_LIB_PATH = os.path.join(PKG, "libaxr_debug.so")
 
 SOURCES = ["api.cu", "attention.cu", "codebook.cpp", "quantize_keys.cu", "quantize_keys_block.cu",
            "quantize_keys_tc.cu", "scores.cu", "scores_tc.cu", "scores_tc128.cu", "sign_select.cu"]
@@ -46,16 +53,18 @@ def _stale(target: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, jobs: int | None = None) -> str:
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(force: bool = False, ptxas_verbose: bool = False, jobs: int | None = None, debug: bool = False) -> str:
+    build_dir = os.path.join(BUILD_DIR, "debug") if debug else BUILD_DIR
+    lib_path = DEBUG_LIB_PATH if debug else LIB_PATH
+    os.makedirs(build_dir, exist_ok=True)
     cc = nvcc()
     objs, cmds = [], []
     for src in SOURCES:
         src_path = os.path.join(CSRC, src)
-        obj = os.path.join(BUILD_DIR, os.path.splitext(src)[0] + ".o")
+        obj = os.path.join(build_dir, os.path.splitext(src)[0] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src_path] + HEADERS):
-            flags = list(COMMON) + ARCH
+            flags = list(COMMON) + ARCH + (["-DAXR_DEBUG"] if debug else [])
             if ptxas_verbose and src.endswith(".cu"):
                 flags += ["-Xptxas", "-v"]
             cmds.append([cc, *flags, "-c", src_path, "-o", obj])
@@ -75,19 +84,20 @@ def build(force: bool = False, ptxas_verbose: bool = False, jobs: int | None = N
     if failed:
         raise RuntimeError(f"nvcc failed on: {', '.join(failed)}")
 
-    if force or cmds or _stale(LIB_PATH, objs):
-        tmp = f"{LIB_PATH}.{os.getpid()}.tmp"
+    if force or cmds or _stale(lib_path, objs):
+        tmp = f"{lib_path}.{os.getpid()}.tmp"
         subprocess.check_call([cc, "-shared", *ARCH, "-o", tmp, *objs, "-cudart", "static"])
-        os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 def main() -> None:
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build libaxr_debug.so (-DAXR_DEBUG)")
     args = ap.parse_args()
-    print(build(force=args.force, ptxas_verbose=args.ptxas_verbose))
+    print(build(force=args.force, ptxas_verbose=args.ptxas_verbose, debug=args.debug))
 
 
 if __name__ == "__main__":

@@ -32,15 +32,7 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 bool pow2_in_range(int d) { return d >= 8 && d <= 512 && (d & (d - 1)) == 0; }
 
-int elem_size(int dtype)
-{
-    switch (dtype) {
-    case AXR_F32: return 4;
-    case AXR_F16: return 2;
-    case AXR_BF16: return 2;
-    default: return 0;
-    }
-}
+int elem_size(int dtype) { return dtype_bytes(dtype); }
 
 // Where a pointer lives, for the current device's kernels: device memory of the
 // current device, managed memory, or host memory mapped into the device address
@@ -131,6 +123,49 @@ cudaError_t allow_dynamic_smem(const void *kernel, size_t bytes, std::atomic<uns
     if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
     return e;
 }
+
+namespace dbg {
+namespace {
+std::mutex g_reader_mu;
+std::vector<Reader> &readers()
+{
+    static std::vector<Reader> v;
+    return v;
+}
+#ifdef AXR_DEBUG
+std::atomic<int64_t> g_slack{0};
+#endif
+}  // namespace
+
+bool register_reader(Reader r)
+{
+    std::lock_guard<std::mutex> lock(g_reader_mu);
+    readers().push_back(r);
+    return true;
+}
+
+unsigned read_all(bool clear)
+{
+    std::lock_guard<std::mutex> lock(g_reader_mu);
+    unsigned v = 0;
+    for (Reader r : readers()) {
+        const unsigned x = r(clear);
+        if (x == ~0u) return ~0u;
+        v |= x;
+    }
+    return v;
+}
+
+#ifdef AXR_DEBUG
+void set_slack(int64_t bytes) { g_slack.store(bytes, std::memory_order_relaxed); }
+
+Span span(const void *base, uint64_t bytes)
+{
+    const uint64_t slack = static_cast<uint64_t>(g_slack.load(std::memory_order_relaxed));
+    return Span{reinterpret_cast<uintptr_t>(base), bytes > slack ? bytes - slack : 0};
+}
+#endif
+}  // namespace dbg
 
 }  // namespace axr
 
@@ -244,6 +279,7 @@ extern "C" int axr_append_scores(const void *k_new, int kdtype, const void *q, i
         QuantizeArgs qa{k_new, kdtype, heads, d, b, signs, idx, norms, cb};
         qa.out_stride = capacity;
         qa.out_offset = pos;
+        qa.out_rows = static_cast<int64_t>(heads) * capacity;
         e = launch_quantize_keys(qa, st);
         if (e == cudaSuccess) e = scores_tc_supported(sa) ? launch_scores_tc(sa, st) : launch_scores(sa, st);
     }
@@ -441,9 +477,30 @@ extern "C" int axr_device_status(int clear, unsigned int *status)
     if (e != cudaSuccess) return fail(AXR_ECUDA, "device synchronize: %s", cudaGetErrorString(e));
     const unsigned int q = quantize_tc_status(clear != 0);
     const unsigned int r = scores_tc_status(clear != 0);
-    if (q == ~0u || r == ~0u) return fail(AXR_ECUDA, "reading the device status words failed");
-    *status = q | r;
+    const unsigned int bnd = dbg::read_all(clear != 0);
+    if (q == ~0u || r == ~0u || bnd == ~0u) return fail(AXR_ECUDA, "reading the device status words failed");
+    *status = q | r | bnd;
     return ok();
+}
+
+extern "C" int axr_debug_build(void)
+{
+#ifdef AXR_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+extern "C" int axr_debug_set_span_slack(int64_t bytes)
+{
+    if (bytes < 0) return fail(AXR_EINVAL, "bytes=%lld must be >= 0", (long long)bytes);
+#ifdef AXR_DEBUG
+    dbg::set_slack(bytes);
+    return ok();
+#else
+    return fail(AXR_EUNSUPPORTED, "span slack exists only in the debug build (libaxr_debug.so)");
+#endif
 }
 
 extern "C" const char *axr_last_error(void) { return g_last_error; }

@@ -85,6 +85,7 @@ struct AttnParams {
     int n;
     int group;
     int splits;
+    AXR_DEBUG_ONLY(dbg::Span sp_scores, sp_V, sp_part, sp_out;)
 };
 
 // partial sums of one chunk of keys for the query heads of one KV head
@@ -109,7 +110,8 @@ __global__ void __launch_bounds__(kThreads) attention_partial_kernel(const AttnP
     for (int i = threadIdx.x; i < len; i += kThreads) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float v = (g < p.group) ? p.scores[(static_cast<int64_t>(h) * p.group + g) * p.n + t0 + i] : 0.0f;
+            const float *src = p.scores + (static_cast<int64_t>(h) * p.group + g) * p.n + t0 + i;
+            const float v = (g < p.group && AXR_IN(p.sp_scores, src, 4)) ? *src : 0.0f;
             s_w[g][i] = v;
             red[g] = fmaxf(red[g], v);
         }
@@ -170,7 +172,13 @@ __global__ void __launch_bounds__(kThreads) attention_partial_kernel(const AttnP
     const T *Vh = static_cast<const T *>(p.V) + (static_cast<int64_t>(h) * p.n + t0) * D + lane * E;
     for (int i = warp; i < len; i += kWarps) {
         float v[E];
-        load_values<T, E>(Vh + static_cast<int64_t>(i) * D, v);
+        const T *src = Vh + static_cast<int64_t>(i) * D;
+        if (AXR_IN(p.sp_V, src, E * sizeof(T))) {
+            load_values<T, E>(src, v);
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) v[e] = 0.0f;
+        }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             const float w = s_w[g][i];
@@ -189,10 +197,16 @@ __global__ void __launch_bounds__(kThreads) attention_partial_kernel(const AttnP
         __syncthreads();
     }
     float *part = p.part + (static_cast<int64_t>(h) * p.splits + c) * G * (D + 2);
-    for (int i = threadIdx.x; i < G * D; i += kThreads) part[(i / D) * (D + 2) + i % D] = s_o[i / D][i % D];
+    for (int i = threadIdx.x; i < G * D; i += kThreads) {
+        float *dst = part + (i / D) * (D + 2) + i % D;
+        if (AXR_IN(p.sp_part, dst, 4)) *dst = s_o[i / D][i % D];
+    }
     if (threadIdx.x < G) {
-        part[threadIdx.x * (D + 2) + D] = s_m[threadIdx.x];
-        part[threadIdx.x * (D + 2) + D + 1] = s_l[threadIdx.x];
+        float *dst = part + threadIdx.x * (D + 2) + D;
+        if (AXR_IN(p.sp_part, dst, 8)) {
+            dst[0] = s_m[threadIdx.x];
+            dst[1] = s_l[threadIdx.x];
+        }
     }
 }
 
@@ -204,16 +218,21 @@ __global__ void attention_combine_kernel(const AttnParams p)
     const int h = hq / p.group, g = hq % p.group;
     const float *part = p.part + static_cast<int64_t>(h) * p.splits * G * (D + 2) + g * (D + 2);
     float M = -INFINITY;
-    for (int c = 0; c < p.splits; ++c) M = fmaxf(M, part[static_cast<int64_t>(c) * G * (D + 2) + D]);
+    for (int c = 0; c < p.splits; ++c) {
+        const float *pm = part + static_cast<int64_t>(c) * G * (D + 2) + D;
+        if (AXR_IN(p.sp_part, pm, 4)) M = fmaxf(M, *pm);
+    }
     for (int j = threadIdx.x; j < D; j += blockDim.x) {
         float o = 0.0f, l = 0.0f;
         for (int c = 0; c < p.splits; ++c) {
             const float *pc = part + static_cast<int64_t>(c) * G * (D + 2);
+            if (!AXR_IN(p.sp_part, pc + j, 4) || !AXR_IN(p.sp_part, pc + D, 8)) continue;
             const float sc = expf(pc[D] - M);
             o = fmaf(sc, pc[j], o);
             l = fmaf(sc, pc[D + 1], l);
         }
-        p.out[static_cast<int64_t>(hq) * D + j] = o / l;
+        float *dst = p.out + static_cast<int64_t>(hq) * D + j;
+        if (AXR_IN(p.sp_out, dst, 4)) *dst = o / l;
     }
 }
 
@@ -229,6 +248,11 @@ cudaError_t launch_dgt(const AttentionArgs &a, cudaStream_t stream)
     p.n = static_cast<int>(a.n);
     p.group = a.group;
     p.splits = attention_splits(a.n, a.group);
+    AXR_DEBUG_ONLY(const uint64_t rows_q = static_cast<uint64_t>(a.heads) * a.group;
+                   p.sp_scores = dbg::span(a.scores, rows_q * a.n * sizeof(float));
+                   p.sp_V = dbg::span(a.V, static_cast<uint64_t>(a.heads) * a.n * D * sizeof(T));
+                   p.sp_part = dbg::span(a.workspace, attention_workspace_bytes(a.n, a.heads, a.group, D));
+                   p.sp_out = dbg::span(a.out, rows_q * D * sizeof(float));)
     attention_partial_kernel<D, G, T><<<dim3(p.splits, a.heads), kThreads, 0, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

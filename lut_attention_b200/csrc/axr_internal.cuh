@@ -7,12 +7,19 @@
 #include <cuda_runtime.h>
 
 #include "axr.h"
+#include "bounds.cuh"
 
 namespace axr {
 
 constexpr int kMaxBits = 4;
 constexpr int kMaxLevels = 1 << kMaxBits;
 constexpr int kMaxGroup = 8;
+
+// bytes of one element of an axr_dtype, 0 for anything else
+__host__ __device__ inline int dtype_bytes(int dtype)
+{
+    return dtype == AXR_F32 ? 4 : (dtype == AXR_F16 || dtype == AXR_BF16) ? 2 : 0;
+}
 
 // fp32 codebook for one (d, b): what the kernels receive by value.
 struct Codebook {
@@ -55,6 +62,7 @@ struct QuantizeArgs {
     // key per head is appended)
     int64_t out_stride = 1;
     int64_t out_offset = 0;
+    int64_t out_rows = 0;      // rows of idx and norms (0: n); what the bounds checks of the debug build allow
     // IsoQuant block rotation in place of diag(signs) and H: (d/4) x 8 floats,
     // qL then qR of every 4-element block (quantize_keys_block.cu)
     const float *quats = nullptr;

@@ -39,6 +39,7 @@ struct QParams {
     int64_t out_stride;        // key r goes to row r * out_stride + out_offset
     int64_t out_offset;
     float bnd[kMaxLevels - 1];
+    AXR_DEBUG_ONLY(dbg::Span sp_K, sp_signs, sp_idx, sp_norms;)
 };
 
 template <int D, int B, typename T>
@@ -71,7 +72,10 @@ __global__ void __launch_bounds__(kThreads) quantize_keys_kernel(QParams p)
 #pragma unroll
     for (int k = 0; k < NCH; ++k)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) sg[8 * k + e] = (p.signs[8 * t + 8 * TPR * k + e] < 0) ? -1.0f : 1.0f;
+        for (int e = 0; e < 8; ++e) {
+            const int8_t *sp = p.signs + 8 * t + 8 * TPR * k + e;
+            sg[8 * k + e] = (AXR_IN(p.sp_signs, sp, 1) && *sp < 0) ? -1.0f : 1.0f;
+        }
 
     const float sqrt_d = sqrtf(static_cast<float>(D));
     const int64_t nsteps = (p.n + RW - 1) / RW;
@@ -85,8 +89,9 @@ __global__ void __launch_bounds__(kThreads) quantize_keys_kernel(QParams p)
         float v[E];
 #pragma unroll
         for (int k = 0; k < NCH; ++k) {
-            if (valid) {
-                Load8<T>::run(p.K, row * D + 8 * t + 8 * TPR * k, v + 8 * k);
+            const int64_t at = row * D + 8 * t + 8 * TPR * k;
+            if (valid && AXR_IN(p.sp_K, static_cast<const T *>(p.K) + at, 8 * sizeof(T))) {
+                Load8<T>::run(p.K, at, v + 8 * k);
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v[8 * k + e] = 0.0f;
@@ -160,20 +165,23 @@ __global__ void __launch_bounds__(kThreads) quantize_keys_kernel(QParams p)
             // the warp step's rows are contiguous in idx: write them out
             uint8_t *dst = p.idx + first * P;
             if (rows_here == RW) {
-                if (lane < WBYTES / 16)
+                if (lane < WBYTES / 16 && AXR_IN(p.sp_idx, reinterpret_cast<uint4 *>(dst) + lane, 16))
                     __stcs(reinterpret_cast<uint4 *>(dst) + lane, reinterpret_cast<const uint4 *>(stage)[lane]);
             } else {
                 const int nbytes = static_cast<int>(rows_here) * P;
-                for (int i = lane; i < nbytes; i += 32) dst[i] = stage[i];
+                for (int i = lane; i < nbytes; i += 32)
+                    if (AXR_IN(p.sp_idx, dst + i, 1)) dst[i] = stage[i];
             }
         } else {
             // rows land out_stride rows apart (one key appended per cache head)
             for (int i = lane; i < static_cast<int>(rows_here) * P; i += 32) {
                 const int64_t rr = first + i / P;
-                p.idx[(rr * p.out_stride + p.out_offset) * P + i % P] = stage[i];
+                uint8_t *o = p.idx + (rr * p.out_stride + p.out_offset) * P + i % P;
+                if (AXR_IN(p.sp_idx, o, 1)) *o = stage[i];
             }
         }
-        if (valid && t == 0) __stcs(p.norms + row * p.out_stride + p.out_offset, norm);
+        float *nd = p.norms + row * p.out_stride + p.out_offset;
+        if (valid && t == 0 && AXR_IN(p.sp_norms, nd, 4)) __stcs(nd, norm);
         __syncwarp();
     }
 }
@@ -209,6 +217,11 @@ cudaError_t launch_typed(const QuantizeArgs &a, cudaStream_t stream)
     p.out_stride = a.out_stride;
     p.out_offset = a.out_offset;
     for (int i = 0; i < kMaxLevels - 1; ++i) p.bnd[i] = a.cb.boundaries[i];
+    AXR_DEBUG_ONLY(const int64_t rows = a.out_rows ? a.out_rows : a.n;
+                   p.sp_K = dbg::span(a.K, static_cast<uint64_t>(a.n) * D * sizeof(T));
+                   p.sp_signs = dbg::span(a.signs, D);
+                   p.sp_idx = dbg::span(a.idx, static_cast<uint64_t>(rows) * (D * B / 8));
+                   p.sp_norms = dbg::span(a.norms, static_cast<uint64_t>(rows) * sizeof(float));)
     kernel<<<grid, kThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }

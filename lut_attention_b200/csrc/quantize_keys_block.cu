@@ -61,6 +61,7 @@ struct BParams {
     float bnd[kMaxLevels];
     float tau[kMaxBuckets];
     int base[kMaxBuckets];
+    AXR_DEBUG_ONLY(dbg::Span sp_K, sp_quats, sp_idx, sp_norms;)
 };
 
 // Code of one rotated unit coordinate u, given the bits of f = round(g) + 1.5 * 2^23
@@ -167,7 +168,11 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const 
 #pragma unroll
     for (int i = 0; i < NB; ++i) {
         Quat qL, qRc;
-        block_quats(p.quats, t * NB + i, qL, qRc);
+        if (AXR_IN(p.sp_quats, p.quats + 8 * (t * NB + i), 32)) {
+            block_quats(p.quats, t * NB + i, qL, qRc);
+        } else {
+            unit_quats(qL, qRc);
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const Quat e = {c == 0 ? 1.0f : 0.0f, c == 1 ? 1.0f : 0.0f, c == 2 ? 1.0f : 0.0f, c == 3 ? 1.0f : 0.0f};
@@ -192,7 +197,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const 
 #pragma unroll
         for (int uu = 0; uu < U; ++uu) {
             const int64_t row = (grp * U + uu) * RW + slot;
-            load_row<T, EPT>(p.K, row * D + t * EPT, row < p.n, cur[uu]);
+            const bool ok = row < p.n && AXR_IN(p.sp_K, static_cast<const T *>(p.K) + row * D + t * EPT, EPT * sizeof(T));
+            load_row<T, EPT>(p.K, row * D + t * EPT, ok, cur[uu]);
         }
     }
     for (; grp < ngroups; grp += stride) {
@@ -202,7 +208,9 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const 
 #pragma unroll
             for (int uu = 0; uu < U; ++uu) {
                 const int64_t row = (gn * U + uu) * RW + slot;
-                load_row<T, EPT>(p.K, row * D + t * EPT, row < p.n, nxt[uu]);
+                const bool ok =
+                    row < p.n && AXR_IN(p.sp_K, static_cast<const T *>(p.K) + row * D + t * EPT, EPT * sizeof(T));
+                load_row<T, EPT>(p.K, row * D + t * EPT, ok, nxt[uu]);
             }
         }
 #pragma unroll
@@ -244,8 +252,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const 
             const Word word = (ss >= 1e-36f && ss <= 3.402823466e38f)
                                   ? pack_codes<B, EPT, false, Word>(y, inv, a, offm2, tab, bias, last)
                                   : pack_codes<B, EPT, true, Word>(y, inv, a, offm2, tab, bias, last);
-            if (valid) {
-                uint8_t *dst = p.idx + row * P + t * TB;
+            uint8_t *dst = p.idx + row * P + t * TB;
+            if (valid && AXR_IN(p.sp_idx, dst, TB)) {
                 if constexpr (TB == 8) {
                     *reinterpret_cast<uint2 *>(dst) = make_uint2(static_cast<uint32_t>(word),
                                                                  static_cast<uint32_t>(word >> 32));
@@ -257,8 +265,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_keys_block_kernel(const 
 #pragma unroll
                     for (int i = 0; i < TB; ++i) dst[i] = static_cast<uint8_t>(word >> (8 * i));
                 }
-                if (t == 0) p.norms[row] = norm;
             }
+            if (valid && t == 0 && AXR_IN(p.sp_norms, p.norms + row, 4)) p.norms[row] = norm;
         }
 #pragma unroll
         for (int uu = 0; uu < U; ++uu) cur[uu] = nxt[uu];
@@ -303,6 +311,10 @@ cudaError_t launch_typed(const QuantizeArgs &a, const BucketTable &tab, cudaStre
         p.tau[j] = tab.tau[j];
         p.base[j] = tab.base[j];
     }
+    AXR_DEBUG_ONLY(p.sp_K = dbg::span(a.K, static_cast<uint64_t>(a.n) * D * sizeof(T));
+                   p.sp_quats = dbg::span(a.quats, (D / 4) * 8 * sizeof(float));
+                   p.sp_idx = dbg::span(a.idx, static_cast<uint64_t>(a.n) * (D * B / 8));
+                   p.sp_norms = dbg::span(a.norms, static_cast<uint64_t>(a.n) * sizeof(float));)
     kernel<<<grid, kThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }

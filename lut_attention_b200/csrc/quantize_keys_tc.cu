@@ -29,14 +29,17 @@
 //                   drained by all 16 warps (a 32-column quarter each).
 // Quantization: u = y / sqrt(sum y^2); with g = u * G_SCALE + G_OFF every
 // bucket [j - 0.5, j + 0.5) of g holds at most one decision boundary, so
-//     idx = base[j] + (g > tau[j]),   j = round(g)
+//     idx = base[j] + (u > tau[j]),   j = round(g)
 // is the count of boundaries below u (one table lookup and one compare instead
 // of a b-level binary search).  tau[j] is the boundary inside bucket j (+inf if
 // none); no boundary lies near a bucket edge, so the rounding of j never
-// changes the result.  Zero keys and exact zeros land on tau = G_OFF, the
-// central boundary, and take the lower index, as ties do.  A key with a
-// non-finite entry (outside the contract) stores its non-finite norm and the
-// central index instead of reading the table out of range.
+// changes the result.  Each bucket is one 32-bit word in shared memory (tau with
+// base in its low 4 bits, see place_code): one wavefront per warp-wide lookup,
+// which buckets 32 apart would have to share a bank to conflict.  Zero keys and
+// exact zeros land on the central boundary (0) and take the lower index, as
+// ties do.  A key with a non-finite entry (outside the contract) stores its
+// non-finite norm and the central index instead of reading the table out of
+// range.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -91,6 +94,7 @@ struct TcParams {
     int nt;
     float tau[kMaxBuckets];
     int base[kMaxBuckets];
+    AXR_DEBUG_ONLY(dbg::Span sp_idx, sp_norms, sp_signs, sp_quats;)
 };
 
 struct Smem {
@@ -100,53 +104,62 @@ struct Smem {
     float ss[2][2][kTileRows];     // [accumulator][column half][key]: partial sums of y^2
 };
 
-// Add the code of one coordinate into the packed words at bit offset O, given its
-// bucket value g and the bits of f = round(g) + 1.5 * 2^23 (bucket table at
-// shared address tab, bias folded so that the entry address is bits(f) * 8 +
-// bias).  Codes occupy disjoint bit fields, so adding the bucket's base and then
-// the compare bit is the same as or-ing the code.
+// Insert the code of one coordinate (unit value u) into the packed words at bit
+// offset O.  Its bucket is round(g) for g = u g_scale + g_off, read from the
+// bits of f = g + 1.5 * 2^23 (entry address bits(f) * 4 + bias, or the clamped
+// bucket).  An entry is the codebook boundary the bucket holds (u units, +inf
+// if none) with its low 4 mantissa bits replaced by the bucket's base code (the
+// number of boundaries below the bucket).  Compared with u as a float it is the
+// boundary moved by at most 15 ulp (at most 2.3e-7 for d >= 128, inside the
+// 1e-6 boundary window); +inf with a base is a NaN and compares false.  The
+// code is the low bits of entry + (u > entry).  At b = 1, 2, 4 the codes of a
+// 32-bit word arrive in coordinate order and each enters at the top of the word
+// with one funnel shift, moving the earlier ones down; at b = 3 they are
+// masked and added at their offsets.
 template <int B, int O, bool kClamp>
-__device__ __forceinline__ void place_code(float g, float f, uint32_t tab, uint32_t bias, uint32_t *w)
+__device__ __forceinline__ void place_code(float u, float f, uint32_t tab, uint32_t bias, uint32_t *w)
 {
     uint32_t addr;
     if constexpr (kClamp) {
         const uint32_t bucket = min(__float_as_uint(f) - kMagicBits, static_cast<uint32_t>(kMaxBuckets - 1));
-        addr = tab + bucket * 8u;
+        addr = tab + bucket * 4u;
     } else {
-        addr = __float_as_uint(f) * 8u + bias;
+        addr = __float_as_uint(f) * 4u + bias;
     }
-    float tau;
-    uint32_t base;
-    asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(tau), "=r"(base) : "r"(addr));
+    uint32_t e;
+    asm("ld.shared.b32 %0, [%1];" : "=r"(e) : "r"(addr));
+    if (u > __uint_as_float(e)) ++e;
     constexpr int k = O >> 5, sh = O & 31;
-    if constexpr (sh + B <= 32) {
-        w[k] += base << sh;
-        if (g > tau) w[k] += 1u << sh;
+    if constexpr (32 % B == 0) {
+        w[k] = __funnelshift_r(w[k], e, B);
     } else {
-        const uint32_t code = base + (g > tau ? 1u : 0u);
+        const uint32_t code = e & ((1u << B) - 1u);
         w[k] += code << sh;
-        w[k + 1] += code >> (32 - sh);
+        if constexpr (sh + B > 32) w[k + 1] += code >> (32 - sh);
     }
 }
 
-// Quantize coordinates C0 + E, C0 + E + 1 (two at a time: one paired FMA gives
-// both bucket values g = y a + g_off, one more both f = y a + g_off + 1.5 * 2^23,
-// rounded exactly as two scalar FMAs would be).
-// The value compared with the bucket's threshold is g = y ag + goff: the bucket
-// value itself (ag = a, goff = g_off; thresholds in bucket units), or the unit
-// coordinate u (ag = 1 / |y|, goff = 0; thresholds in u units, the
-// block-rotation path), one paired FMA either way.
+// Table entry of bucket j: boundary tau (u units, +inf if none) with its low 4
+// bits replaced by the base code
+__device__ __forceinline__ uint32_t table_entry(float tau, int base)
+{
+    return (__float_as_uint(tau) & ~15u) | static_cast<uint32_t>(base);
+}
+
+// Quantize coordinates C0 + E, C0 + E + 1 (two at a time: one paired multiply
+// gives both unit values u = y / |y|, one paired FMA both f = y a + g_off +
+// 1.5 * 2^23, rounded exactly as two scalar operations would be).
 template <int B, int C0, int E, bool kClamp>
-__device__ __forceinline__ void quantize_chunk(const uint32_t (&v)[32], float2 ag2, float2 goff2, float2 a2,
-                                               float2 offm2, uint32_t tab, uint32_t bias, uint32_t *w)
+__device__ __forceinline__ void quantize_chunk(const uint32_t (&v)[32], float2 ug2, float2 a2, float2 offm2,
+                                               uint32_t tab, uint32_t bias, uint32_t *w)
 {
     if constexpr (E < 32) {
         const float2 y = make_float2(__uint_as_float(v[E]), __uint_as_float(v[E + 1]));
-        const float2 g = __ffma2_rn(y, ag2, goff2);
+        const float2 u = __fmul2_rn(y, ug2);
         const float2 f = __ffma2_rn(y, a2, offm2);
-        place_code<B, (C0 + E) * B, kClamp>(g.x, f.x, tab, bias, w);
-        place_code<B, (C0 + E + 1) * B, kClamp>(g.y, f.y, tab, bias, w);
-        quantize_chunk<B, C0, E + 2, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w);
+        place_code<B, (C0 + E) * B, kClamp>(u.x, f.x, tab, bias, w);
+        place_code<B, (C0 + E + 1) * B, kClamp>(u.y, f.y, tab, bias, w);
+        quantize_chunk<B, C0, E + 2, kClamp>(v, ug2, a2, offm2, tab, bias, w);
     }
 }
 
@@ -179,14 +192,14 @@ __device__ __forceinline__ void h4(const uint32_t (&z)[4][8], int e, float2 (&y)
 // codes of 8 coordinates held in v[24 .. 31] at positions 8 pc .. 8 pc + 7 of a
 // 32-coordinate run (quantize_chunk on the top quarter of v, offset back by 24)
 template <int B, bool kClamp>
-__device__ __forceinline__ void quantize_piece(int pc, const uint32_t (&v)[32], float2 ag2, float2 goff2, float2 a2,
-                                               float2 offm2, uint32_t tab, uint32_t bias, uint32_t *w)
+__device__ __forceinline__ void quantize_piece(int pc, const uint32_t (&v)[32], float2 ug2, float2 a2, float2 offm2,
+                                               uint32_t tab, uint32_t bias, uint32_t *w)
 {
     switch (pc) {
-    case 0: quantize_chunk<B, -24, 24, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w); break;
-    case 1: quantize_chunk<B, -16, 24, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w); break;
-    case 2: quantize_chunk<B, -8, 24, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w); break;
-    default: quantize_chunk<B, 0, 24, kClamp>(v, ag2, goff2, a2, offm2, tab, bias, w); break;
+    case 0: quantize_chunk<B, -24, 24, kClamp>(v, ug2, a2, offm2, tab, bias, w); break;
+    case 1: quantize_chunk<B, -16, 24, kClamp>(v, ug2, a2, offm2, tab, bias, w); break;
+    case 2: quantize_chunk<B, -8, 24, kClamp>(v, ug2, a2, offm2, tab, bias, w); break;
+    default: quantize_chunk<B, 0, 24, kClamp>(v, ug2, a2, offm2, tab, bias, w); break;
     }
 }
 
@@ -266,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
     uint8_t *base = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
     uint8_t *sA = base;                                      // kStages x 32 KB
     uint8_t *sB = sA + kSt * kABytes;                        // NH x 32 KB
-    float2 *sTab = reinterpret_cast<float2 *>(sB + kBRegion);     // kMaxBuckets entries
+    uint32_t *sTab = reinterpret_cast<uint32_t *>(sB + kBRegion);     // kMaxBuckets entries (table_entry)
     Smem &S = *reinterpret_cast<Smem *>(sTab + kMaxBuckets);
 
     const int warp = threadIdx.x >> 5;
@@ -301,7 +314,12 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             float v = 0.0f;
             if ((n >> 2) == (k >> 2)) {
                 Quat qL, qRc;
-                block_quats(p.quats, 32 * l + 4 * j + (n >> 2), qL, qRc);
+                const int m = 32 * l + 4 * j + (n >> 2);
+                if (AXR_IN(p.sp_quats, p.quats + 8 * m, 32)) {
+                    block_quats(p.quats, m, qL, qRc);
+                } else {
+                    unit_quats(qL, qRc);
+                }
                 const int c = k & 3;
                 const Quat y = block_rotate(qL, qRc, {c == 0 ? 1.0f : 0.0f, c == 1 ? 1.0f : 0.0f,
                                                       c == 2 ? 1.0f : 0.0f, c == 3 ? 1.0f : 0.0f});
@@ -329,7 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int k = 8 * c + 2 * e2 + h;
-                const bool neg = ((__popc(n & k) & 1) != 0) != (p.signs[kD * l + k] < 0);
+                const int8_t *sg = p.signs + kD * l + k;
+                const bool neg = ((__popc(n & k) & 1) != 0) != (AXR_IN(p.sp_signs, sg, 1) && *sg < 0);
                 const uint16_t one = kBF16 ? (neg ? 0xBF80 : 0x3F80) : (neg ? 0xBC00 : 0x3C00);
                 pair |= static_cast<uint32_t>(one) << (16 * h);
             }
@@ -340,8 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         *dst = make_uint4(w[0], w[1], w[2], w[3]);
     }
     for (int j = threadIdx.x; j < kMaxBuckets; j += kThreads)
-        sTab[j] = make_float2(j < p.nt ? p.tau[j] : __int_as_float(0x7f800000),
-                              __int_as_float(j < p.nt ? p.base[j] : 0));
+        sTab[j] = table_entry(j < p.nt ? p.tau[j] : __int_as_float(0x7f800000), p.base[j]);
     fence_proxy_async_smem();
     if (warp == 0) {
         tmem_alloc(smem_u32(&S.tmem_base), kTmemCols);
@@ -447,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         float *ss4 = &S.ss[0][0][0];                 // [quarter][key]
         constexpr uint32_t kCentral = (1u << (B - 1)) - 1u;
         const uint32_t tab_u32 = smem_u32(sTab);
-        const uint32_t tab_bias = tab_u32 - kMagicBits * 8u;     // wraps mod 2^32 by design
+        const uint32_t tab_bias = tab_u32 - kMagicBits * 4u;     // wraps mod 2^32 by design
         int it = 0;
         for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
             const uint32_t aph = it & 1;
@@ -485,12 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const bool clamp = !(ss >= 1e-36f);
             const float a = (finite && ss > 0.0f) ? p.g_scale / sqrtf(ss) : 0.0f;
             const float2 a2 = make_float2(a, a);
-            const float2 goff2 = make_float2(p.g_off, p.g_off);
             const float2 offm2 = make_float2(p.g_off + kMagic, p.g_off + kMagic);
-            // the compared value: the bucket value, or u itself for the block rotation
             const float ug = (finite && ss > 0.0f) ? 1.0f / sqrtf(ss) : 0.0f;
-            const float2 ag2 = kBlock ? make_float2(ug, ug) : a2;
-            const float2 gofs2 = kBlock ? make_float2(0.0f, 0.0f) : goff2;
+            const float2 ug2 = make_float2(ug, ug);
             uint32_t w[4][NWQ + 1];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
@@ -520,8 +535,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                 if (finite) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        if (!clamp) quantize_piece<B, false>(pc, v[q], ag2, gofs2, a2, offm2, tab_u32, tab_bias, w[q]);
-                        else quantize_piece<B, true>(pc, v[q], ag2, gofs2, a2, offm2, tab_u32, tab_bias, w[q]);
+                        if (!clamp) quantize_piece<B, false>(pc, v[q], ug2, a2, offm2, tab_u32, tab_bias, w[q]);
+                        else quantize_piece<B, true>(pc, v[q], ug2, a2, offm2, tab_u32, tab_bias, w[q]);
                     }
                 }
             }
@@ -539,8 +554,11 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const int64_t row = static_cast<int64_t>(t) * kTileRows + key;
             if (row < p.n) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) store_words<NWQ>(p.idx + row * P + (4 * q + cq) * NWQ * 4, w[q]);
-                if (cq == 0) __stcs(p.norms + row, norm);
+                for (int q = 0; q < 4; ++q) {
+                    uint8_t *dst = p.idx + row * P + (4 * q + cq) * NWQ * 4;
+                    if (AXR_IN(p.sp_idx, dst, NWQ * 4)) store_words<NWQ>(dst, w[q]);
+                }
+                if (cq == 0 && AXR_IN(p.sp_norms, p.norms + row, 4)) __stcs(p.norms + row, norm);
             }
         }
       } else {
@@ -554,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
         const int key = quad * 32 + lane;            // key within the tile
         constexpr uint32_t kCentral = (1u << (B - 1)) - 1u;
         const uint32_t tab_u32 = smem_u32(sTab);
-        const uint32_t tab_bias = tab_u32 - kMagicBits * 8u;     // wraps mod 2^32 by design
+        const uint32_t tab_bias = tab_u32 - kMagicBits * 4u;     // wraps mod 2^32 by design
         int it = 0;
         const int acc = grp;
         for (int t = blockIdx.x + grp * gridDim.x; t < p.ntiles; t += 2 * gridDim.x, ++it) {
@@ -630,19 +648,16 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
             const bool clamp = !(ss >= 1e-36f);
             const float a = (finite && ss > 0.0f) ? p.g_scale / sqrtf(ss) : 0.0f;
             const float2 a2 = make_float2(a, a);
-            const float2 goff2 = make_float2(p.g_off, p.g_off);
             const float2 offm2 = make_float2(p.g_off + kMagic, p.g_off + kMagic);
-            // the compared value: the bucket value, or u itself for the block rotation
             const float ug = (finite && ss > 0.0f) ? 1.0f / sqrtf(ss) : 0.0f;
-            const float2 ag2 = kBlock ? make_float2(ug, ug) : a2;
-            const float2 gofs2 = kBlock ? make_float2(0.0f, 0.0f) : goff2;
+            const float2 ug2 = make_float2(ug, ug);
             if constexpr (NH == 1) {
                 const uint32_t(&va)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&vh[0]);
                 const uint32_t(&vb)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&vh[32]);
-                if (finite && !clamp) quantize_chunk<B, 0, 0, false>(va, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                else if (finite) quantize_chunk<B, 0, 0, true>(va, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                if (finite && !clamp) quantize_chunk<B, 32, 0, false>(vb, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                else if (finite) quantize_chunk<B, 32, 0, true>(vb, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
+                if (finite && !clamp) quantize_chunk<B, 0, 0, false>(va, ug2, a2, offm2, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 0, 0, true>(va, ug2, a2, offm2, tab_u32, tab_bias, w);
+                if (finite && !clamp) quantize_chunk<B, 32, 0, false>(vb, ug2, a2, offm2, tab_u32, tab_bias, w);
+                else if (finite) quantize_chunk<B, 32, 0, true>(vb, ug2, a2, offm2, tab_u32, tab_bias, w);
             } else {
 #pragma unroll
                 for (int c = 0; c < kHalfCols / 32; ++c) {
@@ -662,19 +677,19 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                     }
                     if (c == 0) {
                         if (finite && !clamp) {
-                            quantize_chunk<B, 0, 0, false>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                            quantize_chunk<B, 0, 0, false>(v1, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w1);
+                            quantize_chunk<B, 0, 0, false>(v, ug2, a2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 0, 0, false>(v1, ug2, a2, offm2, tab_u32, tab_bias, w1);
                         } else if (finite) {
-                            quantize_chunk<B, 0, 0, true>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                            quantize_chunk<B, 0, 0, true>(v1, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w1);
+                            quantize_chunk<B, 0, 0, true>(v, ug2, a2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 0, 0, true>(v1, ug2, a2, offm2, tab_u32, tab_bias, w1);
                         }
                     } else {
                         if (finite && !clamp) {
-                            quantize_chunk<B, 32, 0, false>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                            quantize_chunk<B, 32, 0, false>(v1, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w1);
+                            quantize_chunk<B, 32, 0, false>(v, ug2, a2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 32, 0, false>(v1, ug2, a2, offm2, tab_u32, tab_bias, w1);
                         } else if (finite) {
-                            quantize_chunk<B, 32, 0, true>(v, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w);
-                            quantize_chunk<B, 32, 0, true>(v1, ag2, gofs2, a2, offm2, tab_u32, tab_bias, w1);
+                            quantize_chunk<B, 32, 0, true>(v, ug2, a2, offm2, tab_u32, tab_bias, w);
+                            quantize_chunk<B, 32, 0, true>(v1, ug2, a2, offm2, tab_u32, tab_bias, w1);
                         }
                     }
                 }
@@ -701,9 +716,11 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_keys_tc_kernel(const __g
                 // this warp's 64 coordinates of each 128: runs of NWH words at
                 // coordinates 64 half and (d = 256) 128 + 64 half
                 uint8_t *dst = p.idx + row * P + half * (NWH * 4);
-                store_run<NWH>(dst, w);
-                if constexpr (NH == 2) store_run<NWH>(dst + 2 * NWH * 4, w1);
-                if (half == 0) __stcs(p.norms + row, norm);
+                if (AXR_IN(p.sp_idx, dst, NWH * 4)) store_run<NWH>(dst, w);
+                if constexpr (NH == 2) {
+                    if (AXR_IN(p.sp_idx, dst + 2 * NWH * 4, NWH * 4)) store_run<NWH>(dst + 2 * NWH * 4, w1);
+                }
+                if (half == 0 && AXR_IN(p.sp_norms, p.norms + row, 4)) __stcs(p.norms + row, norm);
             }
         }
       }
@@ -725,8 +742,8 @@ cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_
     constexpr int D = kD * NH;
     auto kernel = quantize_keys_tc_kernel<B, kBF16, NH, kBlock>;
     constexpr size_t kBReg = kBlock ? block_parts<kBF16>() * NH * 8 * kBlkBytes : NH * kBBytes;
-    const size_t smem = 1024 + stages<NH>() * kABytes + kBReg + kMaxBuckets * sizeof(float2) + sizeof(Smem);
-    static_assert(1024 + stages<NH>() * kABytes + kBReg + kMaxBuckets * sizeof(float2) + sizeof(Smem) <= 232448,
+    const size_t smem = 1024 + stages<NH>() * kABytes + kBReg + kMaxBuckets * sizeof(uint32_t) + sizeof(Smem);
+    static_assert(1024 + stages<NH>() * kABytes + kBReg + kMaxBuckets * sizeof(uint32_t) + sizeof(Smem) <= 232448,
                   "shared memory per block");
     static std::atomic<unsigned long long> smem_allowed{0};     // one bit per device
     if (cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(kernel), smem, smem_allowed);
@@ -756,13 +773,17 @@ cudaError_t launch_tc(const QuantizeArgs &a, const BucketTable &tab, cudaStream_
     p.inv_sqrt_d = kBlock ? 1.0f : 1.0f / sqrtf(static_cast<float>(D));
     p.quats = a.quats;
     p.nt = tab.nt;
-    // thresholds in bucket units, or (block rotation, which compares u itself) the
-    // codebook boundary each bucket holds, in u units
+    // the codebook boundary each bucket holds, in u units (the kernel compares u itself)
     for (int j = 0; j < kMaxBuckets; ++j) {
         const bool has = j < tab.nt && tab.tau[j] < INFINITY;
-        p.tau[j] = kBlock ? (has ? a.cb.boundaries[tab.base[j]] : INFINITY) : tab.tau[j];
+        p.tau[j] = has ? a.cb.boundaries[tab.base[j]] : INFINITY;
         p.base[j] = tab.base[j];
     }
+    AXR_DEBUG_ONLY(const int64_t rows = a.out_rows ? a.out_rows : a.n;
+                   p.sp_idx = dbg::span(a.idx, static_cast<uint64_t>(rows) * (D * B / 8));
+                   p.sp_norms = dbg::span(a.norms, static_cast<uint64_t>(rows) * sizeof(float));
+                   p.sp_signs = dbg::span(a.signs, a.signs ? D : 0);
+                   p.sp_quats = dbg::span(a.quats, a.quats ? (D / 4) * 8 * sizeof(float) : 0);)
     const int grid = p.ntiles < device_sm_count() ? p.ntiles : device_sm_count();
     kernel<<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError();

@@ -27,6 +27,13 @@ __device__ __forceinline__ void block_quats(const float *quats, int m, Quat &qL,
     qRc = {r.x, -r.y, -r.z, -r.w};
 }
 
+// qL = conj(qR) = 1: what a debug build substitutes for a block it may not read
+__device__ __forceinline__ void unit_quats(Quat &qL, Quat &qRc)
+{
+    qL = {1.0f, 0.0f, 0.0f, 0.0f};
+    qRc = {1.0f, 0.0f, 0.0f, 0.0f};
+}
+
 __device__ __forceinline__ Quat block_rotate(const Quat &qL, const Quat &qRc, const Quat &v)
 {
     return qmul(qmul(qL, v), qRc);

@@ -42,6 +42,7 @@ struct SParams {
     const float *quats;        // block rotation of the queries instead of H diag(signs), or null
     float *scores;
     float cent[kMaxLevels];
+    AXR_DEBUG_ONLY(dbg::Span sp_q, sp_idx, sp_norms, sp_signs, sp_quats, sp_scores;)
 };
 
 __device__ __forceinline__ float load_q(const void *q, int dtype, int64_t i)
@@ -136,8 +137,14 @@ __global__ void __launch_bounds__(kThreads) scores_kernel(SParams p)
         float *sq = s_q[g];
         if (g < p.group) {
             const int64_t qrow = static_cast<int64_t>(h) * p.group + g;
-            for (int j = lane; j < D; j += 32)
-                sq[j] = (p.quats || p.signs[j] >= 0 ? 1.0f : -1.0f) * load_q(p.q, p.qdtype, qrow * D + j);
+            const int qb = dtype_bytes(p.qdtype);
+            for (int j = lane; j < D; j += 32) {
+                const int64_t qi = qrow * D + j;
+                const bool flip = !p.quats && AXR_IN(p.sp_signs, p.signs + j, 1) && p.signs[j] < 0;
+                const float qv =
+                    AXR_IN(p.sp_q, static_cast<const char *>(p.q) + qi * qb, qb) ? load_q(p.q, p.qdtype, qi) : 0.0f;
+                sq[j] = flip ? -qv : qv;
+            }
         } else {
             for (int j = lane; j < D; j += 32) sq[j] = 0.0f;
         }
@@ -147,7 +154,11 @@ __global__ void __launch_bounds__(kThreads) scores_kernel(SParams p)
             const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
             for (int m = lane; m < D / 4; m += 32) {
                 Quat qL, qRc;
-                block_quats(p.quats, m, qL, qRc);
+                if (AXR_IN(p.sp_quats, p.quats + 8 * m, 32)) {
+                    block_quats(p.quats, m, qL, qRc);
+                } else {
+                    unit_quats(qL, qRc);
+                }
                 const Quat y = block_rotate(qL, qRc, {sq[4 * m], sq[4 * m + 1], sq[4 * m + 2], sq[4 * m + 3]});
                 sq[4 * m] = y.w * inv_sqrt_d;
                 sq[4 * m + 1] = y.x * inv_sqrt_d;
@@ -189,7 +200,8 @@ __global__ void __launch_bounds__(kThreads) scores_kernel(SParams p)
         const int r = r0 + slot;
         const bool valid = r < tile1;
         uint32_t w[NW];
-        load_bytes<WB>(idx_h + static_cast<int64_t>(r) * P + part * WB, valid, w);
+        const uint8_t *src = idx_h + static_cast<int64_t>(r) * P + part * WB;
+        load_bytes<WB>(src, valid && AXR_IN(p.sp_idx, src, WB), w);
         float acc[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) acc[g] = 0.0f;
@@ -204,11 +216,12 @@ __global__ void __launch_bounds__(kThreads) scores_kernel(SParams p)
 #pragma unroll
             for (int g = 0; g < G; ++g) acc[g] += __shfl_xor_sync(kFull, acc[g], m);
         if (valid) {
-            const float nk = __ldg(norms_h + r);
+            const float nk = AXR_IN(p.sp_norms, norms_h + r, 4) ? __ldg(norms_h + r) : 0.0f;
 #pragma unroll
-            for (int g = 0; g < G; ++g)
-                if (g % LR == part && g < p.group)
-                    __stcs(p.scores + (static_cast<int64_t>(h) * p.group + g) * n + r, nk * acc[g]);
+            for (int g = 0; g < G; ++g) {
+                float *dst = p.scores + (static_cast<int64_t>(h) * p.group + g) * n + r;
+                if (g % LR == part && g < p.group && AXR_IN(p.sp_scores, dst, 4)) __stcs(dst, nk * acc[g]);
+            }
         }
     }
 }
@@ -228,6 +241,14 @@ cudaError_t launch_dbg(const ScoresArgs &a, cudaStream_t stream)
     p.quats = a.quats;
     p.scores = a.scores;
     for (int i = 0; i < kMaxLevels; ++i) p.cent[i] = a.cb.centroids[i];
+    AXR_DEBUG_ONLY(const uint64_t rows_q = static_cast<uint64_t>(a.heads) * a.group;
+                   const uint64_t rows_k = static_cast<uint64_t>(a.heads) * a.head_stride;
+                   p.sp_q = dbg::span(a.q, rows_q * D * dtype_bytes(a.qdtype));
+                   p.sp_idx = dbg::span(a.idx, rows_k * (D * B / 8));
+                   p.sp_norms = dbg::span(a.norms, rows_k * sizeof(float));
+                   p.sp_signs = dbg::span(a.signs, a.signs ? D : 0);
+                   p.sp_quats = dbg::span(a.quats, a.quats ? (D / 4) * 8 * sizeof(float) : 0);
+                   p.sp_scores = dbg::span(a.scores, rows_q * a.n * sizeof(float));)
     const dim3 grid(static_cast<unsigned>((a.n + kTile - 1) / kTile), static_cast<unsigned>(a.heads));
     scores_kernel<D, B, G><<<grid, kThreads, 0, stream>>>(p);
     return cudaGetLastError();

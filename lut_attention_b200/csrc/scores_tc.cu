@@ -5,6 +5,10 @@
 // rotated by the Walsh-Hadamard transform or, for keys written with it, by the
 // IsoQuant block rotation.  128-wide heads have their own kernel
 // (scores_tc128.cu); the digits and lookup tables are shared (lut_read.cuh).
+// A decode step (one new key per KV head, axr_append_scores) runs in the same
+// launch: the stream that meets a head's last tile quantizes the new key itself
+// (append_key), stores its codes and norm in the cache and scores it with the
+// rest of the tile.
 //
 // The lookups become fixed-point digits that feed an exact int32 tcgen05.mma
 // kind::i8 contraction over a tile of 128 keys and the G queries of a KV head
@@ -112,9 +116,19 @@ struct TcParams {
     float inv_sc;              // 1 / (128 * S_c)
     int8_t hi[kMaxLevels];     // centroid digits
     int8_t lo[kMaxLevels];
+    // decode step: the key of KV head h in k_new (heads x d, kdtype) is quantized
+    // into row append_pos of that head (the last key scored)
+    int append_pos;            // -1: no key to append
+    int kdtype;
+    const void *k_new;
+    uint8_t *idx_out;
+    float *norms_out;
+    float bnd[kMaxLevels - 1];
+    AXR_DEBUG_ONLY(dbg::Span sp_q, sp_signs, sp_quats, sp_scores, sp_k_new, sp_idx_out, sp_norms_out;)
 };
 
 constexpr int kMaxStreams = 3;
+constexpr int kMaxD = 4 * kD;
 struct Smem {
     uint64_t full[kStagesMax], empty[kStagesMax];
     // per stream and buffer: A written (workers); products done (one commit: A
@@ -125,6 +139,12 @@ struct Smem {
     uint32_t tmem_base;
     float inv[kMaxStreams][kInvSlots][8];   // per stream, head slot and query: 1 / (128 * S_q * S_c)
     float qmax[kMaxStreams][4][8];           // per stream, warp and query: max |q''|
+    // decode step, per stream: the appended key after the in-warp transform
+    // stages, its per-warp sums of squares, and its packed row (+1 spare word)
+    float ky[kMaxStreams][kMaxD];
+    float ksum[kMaxStreams][4];
+    float knorm[kMaxStreams];
+    uint32_t arow[kMaxStreams][kMaxD * kMaxBits / 32 + 1];
 };
 constexpr int kSmemBook = 10240;
 static_assert(sizeof(Smem) <= kSmemBook, "bookkeeping area too small");
@@ -154,12 +174,14 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
 #pragma unroll
     for (int sl = 0; sl < NH; ++sl) {
         const int j = tid + kD * sl;
-        const float sg = (p.quats || p.signs[j] >= 0) ? 1.0f : -1.0f;
+        const float sg = (p.quats || !AXR_IN(p.sp_signs, p.signs + j, 1) || p.signs[j] >= 0) ? 1.0f : -1.0f;
+        [[maybe_unused]] const int qb = dtype_bytes(p.qdtype);
 #pragma unroll
-        for (int qi = 0; qi < NQ; ++qi)
-            q[qi][j] = (qi < p.group)
-                           ? sg * lut::load_q(p.q, p.qdtype, (static_cast<int64_t>(h) * p.group + qi) * D + j)
-                           : 0.0f;
+        for (int qi = 0; qi < NQ; ++qi) {
+            const int64_t at = (static_cast<int64_t>(h) * p.group + qi) * D + j;
+            q[qi][j] = (qi < p.group && AXR_IN(p.sp_q, static_cast<const char *>(p.q) + at * qb, qb))
+                           ? sg * lut::load_q(p.q, p.qdtype, at) : 0.0f;
+        }
     }
     if (!stream_sync(S, g, phase)) return false;
     float qq[NQ][NH];
@@ -171,7 +193,11 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
         for (int sl = 0; sl < NH; ++sl) {
             const int j = tid + kD * sl;
             Quat qL, qRc;
-            block_quats(p.quats, j >> 2, qL, qRc);
+            if (AXR_IN(p.sp_quats, p.quats + 8 * (j >> 2), 32)) {
+                block_quats(p.quats, j >> 2, qL, qRc);
+            } else {
+                unit_quats(qL, qRc);
+            }
             const int b0 = j & ~3;
 #pragma unroll
             for (int qi = 0; qi < NQ; ++qi) {
@@ -224,6 +250,88 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
     }
     fence_proxy_async_smem();
     return stream_sync(S, g, phase);
+}
+
+// Decode step: quantize the appended key of KV head h exactly as the write path
+// defines it (sign flip, Walsh-Hadamard, norm, nearest centroid, packing) with
+// the stream's 128 threads; thread j holds coordinates j + 128 l of the NH
+// slices l.  The transform's strides 128 and 256 run inside the thread, strides
+// 1-16 as shuffles, strides 32 and 64 as one 4-point transform across the
+// stream's warps through shared memory.  Stores the codes and the norm in the
+// cache and leaves the packed row in S.arow[g] and the norm in S.knorm[g].
+template <int B, int NH>
+__device__ bool append_key(const TcParams &p, Smem &S, int g, int h, int &phase)
+{
+    constexpr int D = kD * NH;
+    constexpr int PT = D * B / 8;             // bytes of the whole packed row
+    constexpr int L = 1 << B;
+    static_assert(D <= kMaxD && PT / 4 < kGroupThreads, "append scratch");
+    const int tid = threadIdx.x & (kGroupThreads - 1);
+    const int lane = tid & 31, wq = tid >> 5;
+    [[maybe_unused]] const int kb = dtype_bytes(p.kdtype);
+    float x[NH];
+    float ss = 0.0f;
+#pragma unroll
+    for (int sl = 0; sl < NH; ++sl) {
+        const int j = tid + kD * sl;
+        const int64_t at = static_cast<int64_t>(h) * D + j;
+        const bool flip = AXR_IN(p.sp_signs, p.signs + j, 1) && p.signs[j] < 0;
+        const float kv = AXR_IN(p.sp_k_new, static_cast<const char *>(p.k_new) + at * kb, kb)
+                             ? lut::load_q(p.k_new, p.kdtype, at) : 0.0f;
+        x[sl] = flip ? -kv : kv;
+        ss = fmaf(x[sl], x[sl], ss);
+    }
+#pragma unroll
+    for (int st = 1; st < NH; st <<= 1)
+#pragma unroll
+        for (int sl = 0; sl < NH; ++sl)
+            if (!(sl & st)) {
+                const float a = x[sl], c = x[sl + st];
+                x[sl] = a + c;
+                x[sl + st] = a - c;
+            }
+#pragma unroll
+    for (int st = 1; st < 32; st <<= 1)
+#pragma unroll
+        for (int sl = 0; sl < NH; ++sl) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[sl], st);
+            x[sl] = (lane & st) ? o - x[sl] : x[sl] + o;
+        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) S.ksum[g][wq] = ss;
+    float *y = S.ky[g];
+#pragma unroll
+    for (int sl = 0; sl < NH; ++sl) y[kD * sl + tid] = x[sl];
+    if (tid <= PT / 4) S.arow[g][tid] = 0u;
+    if (!stream_sync(S, g, phase)) return false;
+    const float nk = sqrtf((S.ksum[g][0] + S.ksum[g][1]) + (S.ksum[g][2] + S.ksum[g][3]));
+    // u = y / (sqrt(d) ||k||); idx = number of boundaries below u (a zero key has
+    // u = 0 and takes the central index)
+    const float den = sqrtf(static_cast<float>(D)) * nk;
+#pragma unroll
+    for (int sl = 0; sl < NH; ++sl) {
+        // coordinate (wq, lane) of slice sl = sum over warps v of (-1)^popcount(wq & v) y(v, lane)
+        const float *ys = y + kD * sl;
+        const float v0 = ys[lane], v1 = ys[lane + 32], v2 = ys[lane + 64], v3 = ys[lane + 96];
+        const float a = (wq & 1) ? v0 - v1 : v0 + v1;
+        const float c = (wq & 1) ? v2 - v3 : v2 + v3;
+        const float yv = (wq & 2) ? a - c : a + c;
+        const float u = (nk > 0.0f) ? yv / den : 0.0f;
+        uint32_t code = 0;
+#pragma unroll
+        for (int i = 0; i < L - 1; ++i) code += (u > p.bnd[i]) ? 1u : 0u;
+        const int bit = (kD * sl + tid) * B;
+        atomicOr(&S.arow[g][bit >> 5], code << (bit & 31));
+        if ((bit & 31) + B > 32) atomicOr(&S.arow[g][(bit >> 5) + 1], code >> (32 - (bit & 31)));
+    }
+    if (tid == 0) S.knorm[g] = nk;
+    if (!stream_sync(S, g, phase)) return false;
+    const int64_t row = static_cast<int64_t>(h) * p.head_stride + p.append_pos;
+    uint32_t *dst = reinterpret_cast<uint32_t *>(p.idx_out + row * PT) + tid;
+    if (tid < PT / 4 && AXR_IN(p.sp_idx_out, dst, 4)) *dst = S.arow[g][tid];
+    if (tid == 0 && AXR_IN(p.sp_norms_out, p.norms_out + row, 4)) p.norms_out[row] = nk;
+    return true;
 }
 
 // byte offset of 16-byte chunk c of tile row r in a stage, with the swizzle
@@ -299,7 +407,7 @@ struct Worker {
                 const float hi = __int2float_rn(x[0] * 128 + x[1]);
                 const float lo = __int2float_rn(x[2] * 128 + x[3]);
                 if (qi < p.group) {
-                    __stcs(dst, nk * inv[qi] * fmaf(lo, 1.0f / 16384.0f, hi));
+                    if (AXR_IN(p.sp_scores, dst, 4)) __stcs(dst, nk * inv[qi] * fmaf(lo, 1.0f / 16384.0f, hi));
                     dst += p.n;
                 }
             }
@@ -335,6 +443,17 @@ struct Worker {
 
         for (int tile = t0 + g; tile < t1; tile += C::S, ++k) {
             float nk = 0.0f;
+            // decode step: this head's last tile holds the appended key.  It is
+            // quantized before the tile's stages are read (fewer registers live);
+            // the stages may hold its row as it was before this launch or as
+            // stored here, and the thread of that key takes the row and norm
+            // from shared memory instead either way
+            const bool appending = p.append_pos >= 0 && ti == (p.append_pos >> 7);
+            if (appending && !append_key<B, NH>(p, S, g, h, sync_phase)) {
+                if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                ok = false;
+                break;
+            }
 #pragma unroll 1
             for (int sl = 0; sl < NH; ++sl) {
                 const int m = k * NH + sl;      // this stream's subtile count
@@ -400,6 +519,11 @@ struct Worker {
                             break;
                         }
                     }
+                }
+                if (appending && r == (p.append_pos & (kTileRows - 1))) {
+#pragma unroll
+                    for (int v = 0; v < NW; ++v) w[v] = S.arow[g][sl * NW + v];
+                    if (sl == 0) nk = S.knorm[g];
                 }
 
                 // lookup l fills A columns l (4-byte entries) or 2l, 2l+1 (8-byte entries)
@@ -673,10 +797,26 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     p.group = a.group;
     p.tiles_per_head = static_cast<int>((a.n + kTileRows - 1) / kTileRows);
     p.total_tiles = p.tiles_per_head * a.heads;
+    p.append_pos = a.k_new ? static_cast<int>(a.append_pos) : -1;
+    p.kdtype = a.kdtype;
+    p.k_new = a.k_new;
+    p.idx_out = a.idx_out;
+    p.norms_out = a.norms_out;
+    for (int i = 0; i < kMaxLevels - 1; ++i) p.bnd[i] = a.cb.boundaries[i];
     const int sms = device_sm_count();
     const int grid = p.total_tiles < sms ? p.total_tiles : sms;
     p.tiles_per_cta = (p.total_tiles + grid - 1) / grid;
     lut::centroid_digits(a.cb, p.hi, p.lo, &p.inv_sc);
+    AXR_DEBUG_ONLY(constexpr int D = kD * NH;
+                   const uint64_t rows_q = static_cast<uint64_t>(a.heads) * a.group;
+                   const uint64_t rows_k = static_cast<uint64_t>(a.heads) * a.head_stride;
+                   p.sp_q = dbg::span(a.q, rows_q * D * dtype_bytes(a.qdtype));
+                   p.sp_signs = dbg::span(a.signs, a.signs ? D : 0);
+                   p.sp_quats = dbg::span(a.quats, a.quats ? (D / 4) * 8 * sizeof(float) : 0);
+                   p.sp_scores = dbg::span(a.scores, rows_q * a.n * sizeof(float));
+                   p.sp_k_new = dbg::span(a.k_new, a.k_new ? static_cast<uint64_t>(a.heads) * D * dtype_bytes(a.kdtype) : 0);
+                   p.sp_idx_out = dbg::span(a.idx_out, a.idx_out ? rows_k * PT : 0);
+                   p.sp_norms_out = dbg::span(a.norms_out, a.norms_out ? rows_k * sizeof(float) : 0);)
     const int used = (p.total_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
     kernel<<<used, Cfg<NQ, NH>::kThreads, smem, stream>>>(p);
     return cudaGetLastError();
@@ -704,9 +844,8 @@ cudaError_t launch_h(const ScoresArgs &a, cudaStream_t stream)
 bool scores_tc_supported(const ScoresArgs &a)
 {
     if (a.d == kD) return scores_tc128_supported(a);
-    // d = 256 and 512 run as 2 and 4 slices of 128 coordinates; the fused decode
-    // step (one appended key quantized in the kernel) exists for d = 128 only
-    const bool width = (a.d == 2 * kD || a.d == 4 * kD) && a.k_new == nullptr;
+    // d = 256 and 512 run as 2 and 4 slices of 128 coordinates
+    const bool width = a.d == 2 * kD || a.d == 4 * kD;
     return width && a.b >= 1 && a.b <= 4 && a.group <= 8 && a.n > 0 &&
            static_cast<int64_t>(a.heads) * a.head_stride < (static_cast<int64_t>(1) << 31) - kTileRows &&
            encode_tiled() != nullptr;

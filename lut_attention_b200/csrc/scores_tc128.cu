@@ -74,6 +74,7 @@ struct Params {
     uint8_t *idx_out;
     float *norms_out;
     float bnd[kMaxLevels - 1];
+    AXR_DEBUG_ONLY(dbg::Span sp_q, sp_signs, sp_quats, sp_scores, sp_k_new, sp_idx_out, sp_norms_out;)
 };
 
 // stages planned below the 64 KB-aligned table: at most 62 KB, which the window
@@ -178,17 +179,24 @@ __device__ bool build_b(const Params &p, Book &S, int g, uint8_t *b, int h, floa
 {
     const int tid = threadIdx.x & (kStreamThreads - 1);
     const int lane = tid & 31, wq = tid >> 5;
-    const float sg = (p.quats || p.signs[tid] >= 0) ? 1.0f : -1.0f;
+    const float sg = (p.quats || !AXR_IN(p.sp_signs, p.signs + tid, 1) || p.signs[tid] >= 0) ? 1.0f : -1.0f;
+    [[maybe_unused]] const int qb = dtype_bytes(p.qdtype);
     float qq[NQ];
 #pragma unroll
-    for (int qi = 0; qi < NQ; ++qi)
-        qq[qi] = (qi < p.group) ? sg * lut::load_q(p.q, p.qdtype, (static_cast<int64_t>(h) * p.group + qi) * kD + tid)
-                                : 0.0f;
+    for (int qi = 0; qi < NQ; ++qi) {
+        const int64_t at = (static_cast<int64_t>(h) * p.group + qi) * kD + tid;
+        qq[qi] = (qi < p.group && AXR_IN(p.sp_q, static_cast<const char *>(p.q) + at * qb, qb))
+                     ? sg * lut::load_q(p.q, p.qdtype, at) : 0.0f;
+    }
     if (p.quats) {
         // q'' = T q / sqrt(d): the IsoQuant block rotation times the temperature;
         // the 4 coordinates of a block sit in 4 consecutive lanes
         Quat qL, qRc;
-        block_quats(p.quats, tid >> 2, qL, qRc);
+        if (AXR_IN(p.sp_quats, p.quats + 8 * (tid >> 2), 32)) {
+            block_quats(p.quats, tid >> 2, qL, qRc);
+        } else {
+            unit_quats(qL, qRc);
+        }
         const int b0 = lane & ~3;
 #pragma unroll
         for (int qi = 0; qi < NQ; ++qi) {
@@ -251,8 +259,12 @@ __device__ bool append_key(const Params &p, Book &S, int g, int h, float *y, flo
     constexpr int P = kD * B / 8;
     constexpr int L = 1 << B;
     const int tid = threadIdx.x & (kStreamThreads - 1);
-    const float x = (p.signs[tid] < 0 ? -1.0f : 1.0f) *
-                    lut::load_q(p.k_new, p.kdtype, static_cast<int64_t>(h) * kD + tid);
+    [[maybe_unused]] const int kb = dtype_bytes(p.kdtype);
+    const int64_t at = static_cast<int64_t>(h) * kD + tid;
+    const bool flip = AXR_IN(p.sp_signs, p.signs + tid, 1) && p.signs[tid] < 0;
+    const float kv =
+        AXR_IN(p.sp_k_new, static_cast<const char *>(p.k_new) + at * kb, kb) ? lut::load_q(p.k_new, p.kdtype, at) : 0.0f;
+    const float x = flip ? -kv : kv;
     y[tid] = x;
     float ss = x * x;
 #pragma unroll
@@ -281,8 +293,9 @@ __device__ bool append_key(const Params &p, Book &S, int g, int h, float *y, flo
     if ((bit & 31) + B > 32) atomicOr(&S.arow[g][(bit >> 5) + 1], code >> (32 - (bit & 31)));
     if (!stream_sync(S, g, phase)) return false;
     const int64_t row = static_cast<int64_t>(h) * p.head_stride + p.append_pos;
-    if (tid < P / 4) reinterpret_cast<uint32_t *>(p.idx_out + row * P)[tid] = S.arow[g][tid];
-    if (tid == 0) p.norms_out[row] = nk;
+    uint32_t *dst = reinterpret_cast<uint32_t *>(p.idx_out + row * P) + tid;
+    if (tid < P / 4 && AXR_IN(p.sp_idx_out, dst, 4)) *dst = S.arow[g][tid];
+    if (tid == 0 && AXR_IN(p.sp_norms_out, p.norms_out + row, 4)) p.norms_out[row] = nk;
     *norm = nk;
     return true;
 }
@@ -350,7 +363,7 @@ struct Worker {
 #pragma unroll
             for (int qi = 0; qi < NQ; ++qi) {
                 if (qi < p.group) {
-                    __stcs(dst, nk * inv[qi] * lut::join_sums(acc + 4 * qi));
+                    if (AXR_IN(p.sp_scores, dst, 4)) __stcs(dst, nk * inv[qi] * lut::join_sums(acc + 4 * qi));
                     dst += p.n;
                 }
             }
@@ -655,6 +668,15 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     p.norms_out = a.norms_out;
     for (int i = 0; i < kMaxLevels - 1; ++i) p.bnd[i] = a.cb.boundaries[i];
     lut::centroid_digits(a.cb, p.hi, p.lo, &p.inv_sc);
+    AXR_DEBUG_ONLY(const uint64_t rows_q = static_cast<uint64_t>(a.heads) * a.group;
+                   const uint64_t rows_k = static_cast<uint64_t>(a.heads) * a.head_stride;
+                   p.sp_q = dbg::span(a.q, rows_q * kD * dtype_bytes(a.qdtype));
+                   p.sp_signs = dbg::span(a.signs, a.signs ? kD : 0);
+                   p.sp_quats = dbg::span(a.quats, a.quats ? (kD / 4) * 8 * sizeof(float) : 0);
+                   p.sp_scores = dbg::span(a.scores, rows_q * a.n * sizeof(float));
+                   p.sp_k_new = dbg::span(a.k_new, a.k_new ? static_cast<uint64_t>(a.heads) * kD * dtype_bytes(a.kdtype) : 0);
+                   p.sp_idx_out = dbg::span(a.idx_out, a.idx_out ? rows_k * P : 0);
+                   p.sp_norms_out = dbg::span(a.norms_out, a.norms_out ? rows_k * sizeof(float) : 0);)
     const int sms = device_sm_count();
     const int grid = p.total_tiles < sms ? p.total_tiles : sms;
     p.tiles_per_cta = (p.total_tiles + grid - 1) / grid;

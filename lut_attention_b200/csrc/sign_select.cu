@@ -58,6 +58,7 @@ struct SelParams {
     float bnd[kMaxLevels];    // decision boundaries (L - 1 used)
     float tau[kMaxBuckets];
     int base[kMaxBuckets];
+    AXR_DEBUG_ONLY(dbg::Span sp_K, sp_q, sp_cand, sp_errors;)
 };
 
 __device__ __forceinline__ float load_query(const void *q, int dtype, int64_t i)
@@ -132,9 +133,12 @@ __global__ void __launch_bounds__(kThreads) sign_errors_kernel(const __grid_cons
 
     float2 sg[EH];
 #pragma unroll
-    for (int i = 0; i < EH; ++i)
-        sg[i] = make_float2(dc[element_of<E, TPR>(t, i)] < 0 ? -1.0f : 1.0f,
-                            dc[element_of<E, TPR>(t, i + EH)] < 0 ? -1.0f : 1.0f);
+    for (int i = 0; i < EH; ++i) {
+        const int8_t *c0 = dc + element_of<E, TPR>(t, i), *c1 = dc + element_of<E, TPR>(t, i + EH);
+        sg[i] = make_float2(AXR_IN(p.sp_cand, c0, 1) && *c0 < 0 ? -1.0f : 1.0f,
+                            AXR_IN(p.sp_cand, c1, 1) && *c1 < 0 ? -1.0f : 1.0f);
+    }
+    const int qb = dtype_bytes(p.qdtype);
 
     const float sqrt_d = sqrtf(static_cast<float>(D));
     const uint32_t last = static_cast<uint32_t>(p.nt - 1);
@@ -144,8 +148,12 @@ __global__ void __launch_bounds__(kThreads) sign_errors_kernel(const __grid_cons
     for (int s = 0; s < p.samples; ++s) {
         __syncthreads();                  // the previous sample's reads of the queries are done
         const int64_t q0 = (static_cast<int64_t>(s) * p.heads + h) * G * D;
-        for (int i = threadIdx.x; i < G * D; i += kThreads)
-            s_q[i] = (dc[i % D] < 0) ? -load_query(p.q, p.qdtype, q0 + i) : load_query(p.q, p.qdtype, q0 + i);
+        for (int i = threadIdx.x; i < G * D; i += kThreads) {
+            const bool flip = AXR_IN(p.sp_cand, dc + i % D, 1) && dc[i % D] < 0;
+            const float qv = AXR_IN(p.sp_q, static_cast<const char *>(p.q) + (q0 + i) * qb, qb)
+                                 ? load_query(p.q, p.qdtype, q0 + i) : 0.0f;
+            s_q[i] = flip ? -qv : qv;
+        }
         __syncthreads();
         // Walsh-Hadamard butterflies (Sylvester order) over each of the G rows;
         // the 1/sqrt(D) of q' is folded into the key's factor below
@@ -174,8 +182,9 @@ __global__ void __launch_bounds__(kThreads) sign_errors_kernel(const __grid_cons
             float v[E];
 #pragma unroll
             for (int k = 0; k < NCH; ++k) {
-                if (valid) {
-                    Load8<T, false>::run(Ks, row * D + 8 * t + 8 * TPR * k, v + 8 * k);
+                const int64_t at = row * D + 8 * t + 8 * TPR * k;
+                if (valid && AXR_IN(p.sp_K, static_cast<const T *>(Ks) + at, 8 * sizeof(T))) {
+                    Load8<T, false>::run(Ks, at, v + 8 * k);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) v[8 * k + e] = 0.0f;
@@ -265,13 +274,16 @@ __global__ void __launch_bounds__(kThreads) sign_errors_kernel(const __grid_cons
         double tot = 0.0;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) tot += s_red[w];
-        p.errors[static_cast<int64_t>(c) * p.heads + h] = static_cast<float>(tot * p.inv_count);
+        float *dst = p.errors + static_cast<int64_t>(c) * p.heads + h;
+        if (AXR_IN(p.sp_errors, dst, 4)) *dst = static_cast<float>(tot * p.inv_count);
     }
 }
 
 // best = argmin over c of max over h of errors[c][h], the lowest c among equal
 // values; -1 if no candidate compares (every error NaN).
-__global__ void __launch_bounds__(kThreads) select_best_kernel(const float *errors, int C, int heads, int *best)
+__global__ void __launch_bounds__(kThreads)
+    select_best_kernel(const float *errors, int C, int heads, int *best AXR_DEBUG_ONLY(, dbg::Span sp_errors,
+                                                                                        dbg::Span sp_best))
 {
     __shared__ float s_v[kThreads];
     __shared__ int s_i[kThreads];
@@ -280,7 +292,8 @@ __global__ void __launch_bounds__(kThreads) select_best_kernel(const float *erro
     for (int c = threadIdx.x; c < C; c += kThreads) {   // increasing c: strict < keeps the lowest
         float worst = -INFINITY;
         for (int h = 0; h < heads; ++h) {
-            const float e = errors[static_cast<int64_t>(c) * heads + h];
+            const float *src = errors + static_cast<int64_t>(c) * heads + h;
+            const float e = AXR_IN(sp_errors, src, 4) ? *src : NAN;
             if (e > worst || e != e) worst = e;             // a NaN head makes the candidate's worst NaN
         }
         if (worst < bv || (worst == bv && bi == INT_MAX)) {
@@ -302,7 +315,7 @@ __global__ void __launch_bounds__(kThreads) select_best_kernel(const float *erro
         }
         __syncthreads();
     }
-    if (threadIdx.x == 0) *best = (s_i[0] == INT_MAX) ? -1 : s_i[0];
+    if (threadIdx.x == 0 && AXR_IN(sp_best, best, 4)) *best = (s_i[0] == INT_MAX) ? -1 : s_i[0];
 }
 
 template <int D, int B, typename T>
@@ -331,6 +344,11 @@ cudaError_t launch_typed(const SignSelectArgs &a, const BucketTable &tab, cudaSt
     constexpr int E = D >= 32 ? 32 : D;
     constexpr int TPR = D / E;
     const size_t smem = static_cast<size_t>(a.group) * (D + TPR * (E / 2 + 2) * 2) * sizeof(float);
+    AXR_DEBUG_ONLY(const uint64_t rows = static_cast<uint64_t>(a.samples) * a.heads;
+                   p.sp_K = dbg::span(a.K, rows * a.n * D * sizeof(T));
+                   p.sp_q = dbg::span(a.q, rows * a.group * D * dtype_bytes(a.qdtype));
+                   p.sp_cand = dbg::span(a.candidates, static_cast<uint64_t>(a.candidates_count) * D);
+                   p.sp_errors = dbg::span(a.errors, static_cast<uint64_t>(a.candidates_count) * a.heads * 4);)
     sign_errors_kernel<D, B, T><<<a.candidates_count * a.heads, kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
@@ -373,7 +391,10 @@ cudaError_t launch_sign_select(const SignSelectArgs &a, cudaStream_t stream)
     default: e = launch_d<512>(a, tab, stream); break;
     }
     if (e != cudaSuccess || !a.best) return e;
-    select_best_kernel<<<1, kThreads, 0, stream>>>(a.errors, a.candidates_count, a.heads, a.best);
+    select_best_kernel<<<1, kThreads, 0, stream>>>(
+        a.errors, a.candidates_count, a.heads,
+        a.best AXR_DEBUG_ONLY(, dbg::span(a.errors, static_cast<uint64_t>(a.candidates_count) * a.heads * 4),
+                              dbg::span(a.best, 4)));
     return cudaGetLastError();
 }
 

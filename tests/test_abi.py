@@ -175,3 +175,26 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         axr.axr_scores(torch.zeros(1, 128), torch.zeros(1, 4, 64, dtype=torch.uint8),
                        torch.zeros(1, 4), 1, 4, s)
+
+
+def test_debug_library_exports_every_declared_symbol_and_says_so(axr_lib):
+    """libaxr_debug.so (-DAXR_DEBUG) has the same boundary; axr_debug_build tells
+    the two apart and the span slack exists only in the debug build."""
+    from lut_attention_b200 import build
+
+    if not os.path.exists(build.DEBUG_LIB_PATH):
+        build.build(debug=True)
+    dbg = ctypes.CDLL(build.DEBUG_LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+    dbg.axr_debug_build.restype = ctypes.c_int
+    dbg.axr_debug_set_span_slack.restype = ctypes.c_int
+    dbg.axr_debug_set_span_slack.argtypes = [ctypes.c_int64]
+    assert dbg.axr_debug_build() == 1
+    assert dbg.axr_debug_set_span_slack(-1) == axr.AXR_EINVAL
+    assert dbg.axr_debug_set_span_slack(4) == axr.AXR_OK
+    assert dbg.axr_debug_set_span_slack(0) == axr.AXR_OK
+    assert axr_lib.axr_debug_build() == int(axr.DEBUG)
+    if not axr.DEBUG:
+        assert axr_lib.axr_debug_set_span_slack(0) == axr.AXR_EUNSUPPORTED
+        assert b"debug build" in axr_lib.axr_last_error()

@@ -39,6 +39,8 @@ def _cache(heads, capacity, pos, d, b, dtype, seed):
 @pytest.mark.parametrize("d,b,group,dtype", [
     (128, 4, 4, "bf16"), (128, 3, 1, "f16"), (128, 2, 8, "bf16"), (128, 4, 2, "f32"),
     (64, 3, 4, "bf16"), (256, 2, 2, "f16"), (512, 2, 8, "f16"), (8, 1, 3, "f32"),
+    (256, 4, 4, "bf16"), (256, 3, 8, "f32"), (256, 1, 1, "f16"), (512, 4, 4, "bf16"), (512, 3, 2, "f16"),
+    (512, 1, 5, "f32"),
 ])
 def test_append_then_scores(d, b, group, dtype):
     heads, capacity, pos = 3, 704, 517          # 704 * P bytes: every head 16-byte aligned
@@ -62,12 +64,13 @@ def test_append_then_scores(d, b, group, dtype):
     assert check_scores(q, idx[:, :pos + 1].contiguous(), norms[:, :pos + 1].contiguous(), out, group, b, s) <= 1e-4
 
 
+@pytest.mark.parametrize("d", [128, 256, 512])
 @pytest.mark.parametrize("pos,capacity", [(0, 1), (0, 300), (299, 300), (128, 129), (255, 1000)])
-def test_append_edges_of_the_cache(pos, capacity):
+def test_append_edges_of_the_cache(d, pos, capacity):
     """Empty cache (pos 0), the last slot, and positions on tile edges."""
-    d, b, group, heads = 128, 4, 4, 2
-    keys, s, idx, norms = _cache(heads, capacity, pos, d, b, "bf16", seed=pos + capacity)
-    wl = workloads.GQA_DECODE_128K.with_(batch=1, kv_heads=heads, group=group, T=pos + 1)
+    b, group, heads = 4, 4, 2
+    keys, s, idx, norms = _cache(heads, capacity, pos, d, b, "bf16", seed=pos + capacity + d)
+    wl = workloads.GQA_DECODE_128K.with_(d=d, batch=1, kv_heads=heads, group=group, T=pos + 1)
     q = workloads.make_queries(wl, DEV)
     out = axr.axr_append_scores(keys[:, pos].contiguous(), q, idx, norms, pos, group, b, s)
     assert axr.axr_device_status() == 0
@@ -94,3 +97,28 @@ def test_decode_loop_builds_the_cache_key_by_key():
                          norms[:, :steps].reshape(-1), b, s)
     assert rep.ok(), rep
     assert torch.all(idx[:, steps:] == 0xA5)
+
+
+@pytest.mark.parametrize("d,launches", [(128, 1), (256, 1), (512, 1), (64, 2)])
+def test_decode_step_launch_count(d, launches):
+    """At d = 128, 256 and 512 the decode step is one launch of the tensor-core
+    read kernel, which quantizes the new keys itself; below 128 it is the write
+    kernel followed by the read kernel."""
+    from torch.profiler import ProfilerActivity, profile
+
+    b, group, heads, pos, capacity = 4, 4, 2, 200, 256
+    keys, s, idx, norms = _cache(heads, capacity, pos, d, b, "bf16", seed=d)
+    q = workloads.make_queries(workloads.GQA_DECODE_128K.with_(d=d, batch=1, kv_heads=heads, group=group), DEV)
+    k_new = keys[:, pos].contiguous()
+    axr.axr_append_scores(k_new, q, idx, norms, pos, group, b, s)
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        axr.axr_append_scores(k_new, q, idx, norms, pos, group, b, s)
+        torch.cuda.synchronize()
+    kernels = [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+    if not kernels:
+        pytest.skip("the profiler recorded no kernels on this machine")
+    ours = [k for k in kernels if "axr" in k]
+    assert len(ours) == launches, ours
+    if launches == 1:
+        assert "scores_tc" in ours[0], ours

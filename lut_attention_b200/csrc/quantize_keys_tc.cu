@@ -107,15 +107,16 @@ struct Smem {
 // Insert the code of one coordinate (unit value u) into the packed words at bit
 // offset O.  Its bucket is round(g) for g = u g_scale + g_off, read from the
 // bits of f = g + 1.5 * 2^23 (entry address bits(f) * 4 + bias, or the clamped
-// bucket).  An entry is the codebook boundary the bucket holds (u units, +inf
-// if none) with its low 4 mantissa bits replaced by the bucket's base code (the
-// number of boundaries below the bucket).  Compared with u as a float it is the
-// boundary moved by at most 15 ulp (at most 2.3e-7 for d >= 128, inside the
-// 1e-6 boundary window); +inf with a base is a NaN and compares false.  The
-// code is the low bits of entry + (u > entry).  At b = 1, 2, 4 the codes of a
-// 32-bit word arrive in coordinate order and each enters at the top of the word
-// with one funnel shift, moving the earlier ones down; at b = 3 they are
-// masked and added at their offsets.
+// bucket).  An entry is the codebook boundary the bucket holds (u units; 2 if
+// none, which no |u| <= 1 exceeds) with its low 4 mantissa bits replaced by the
+// bucket's base code (the number of boundaries below the bucket).  Read as a
+// float it is the boundary moved by at most 15 ulp (at most 2.3e-7 for
+// d >= 128, inside the 1e-6 boundary window).  u > entry is the sign bit of
+// entry - u (exact in sign, and +0 when the two are equal), so the code is the
+// low bits of entry + that bit.  At b = 1, 2, 4 the codes of a 32-bit word
+// arrive in coordinate order and each enters at the top of the word with one
+// funnel shift, moving the earlier ones down; at b = 3 they are masked and
+// added at their offsets.
 template <int B, int O, bool kClamp>
 __device__ __forceinline__ void place_code(float u, float f, uint32_t tab, uint32_t bias, uint32_t *w)
 {
@@ -128,7 +129,7 @@ __device__ __forceinline__ void place_code(float u, float f, uint32_t tab, uint3
     }
     uint32_t e;
     asm("ld.shared.b32 %0, [%1];" : "=r"(e) : "r"(addr));
-    if (u > __uint_as_float(e)) ++e;
+    e += __float_as_uint(__fsub_rn(__uint_as_float(e), u)) >> 31;
     constexpr int k = O >> 5, sh = O & 31;
     if constexpr (32 % B == 0) {
         w[k] = __funnelshift_r(w[k], e, B);
@@ -139,11 +140,12 @@ __device__ __forceinline__ void place_code(float u, float f, uint32_t tab, uint3
     }
 }
 
-// Table entry of bucket j: boundary tau (u units, +inf if none) with its low 4
-// bits replaced by the base code
+// Table entry of bucket j: boundary tau (u units; 2 for none, tau = +inf) with
+// its low 4 bits replaced by the base code
 __device__ __forceinline__ uint32_t table_entry(float tau, int base)
 {
-    return (__float_as_uint(tau) & ~15u) | static_cast<uint32_t>(base);
+    const float t = tau < 2.0f ? tau : 2.0f;
+    return (__float_as_uint(t) & ~15u) | static_cast<uint32_t>(base);
 }
 
 // Quantize coordinates C0 + E, C0 + E + 1 (two at a time: one paired multiply

@@ -80,7 +80,8 @@ template <int NQ, int NH>
 struct Cfg {
     static_assert(NH == 2 || NH == 4, "128-wide heads run in scores_tc128.cu");
     static constexpr int N = 4 * NQ;                  // B rows = D columns
-    static constexpr int S = (NH == 2) ? ((NQ <= 4) ? 3 : 2) : ((NQ <= 4) ? 2 : 1);   // tile streams
+    // tile streams: 3 wherever tensor memory and the B buffers allow it
+    static constexpr int S = (NH == 2) ? ((NQ <= 4) ? 3 : 2) : ((NQ <= 4) ? 3 : 1);
     static constexpr int kBBufs = 1;                  // B buffers per stream
     static constexpr int kWorkerWarps = 4 * S;
     static constexpr int kWarpTma = kWorkerWarps;
@@ -89,8 +90,12 @@ struct Cfg {
     static constexpr int kDOff = S * 2 * kACols;      // A buffers first, then D buffers
     static constexpr int kSliceB = N * kK;            // B bytes of one subtile's K block
     static constexpr int kBBytes = kSliceB * NH;      // one B buffer
-    static constexpr int kStages = kStagesMax;
+    // stages in flight: 12, or 9 at d = 512 with three streams, whose B buffers
+    // (3 x 16 KB) take the shared memory of three stages
+    static constexpr int kStages = (NH == 4 && NQ <= 4) ? 9 : kStagesMax;
+    static constexpr int kBRegion = S * kBBufs * kBBytes;   // the streams' B buffers
     static_assert(kStages % S == 0, "streams must own whole stages");
+    static_assert(kStages > kLowStages, "stages below and after the table");
     static_assert(kDOff + S * 2 * N <= kTmemCols, "tensor memory budget");
     static_assert(kSliceB <= kBBytesMax, "B buffer");
     static_assert(kBBytes >= NQ * kD * NH * 4, "a wide head's B buffer holds its rotation scratch");
@@ -347,10 +352,10 @@ __device__ __forceinline__ int chunk_offset(int r, int c)
 // Dynamic shared memory: the table on a 64 KB boundary of the shared window
 // (so one PRMT forms a full address).  The request covers the table's
 // alignment gap (at most 64 KB, which holds stages 0-5 when it is large
-// enough), the table, and after it kRestBytes: stages 6-11, B and the
-// bookkeeping.
-constexpr int kBRegion = 32768;       // two B buffers per stream, for every stream
-constexpr int kRestBytes = (kStagesMax - kLowStages) * kStageBytes + kBRegion + kSmemBook;
+// enough), the table, and after it kRestBytes: stages 6-11 (6-8 with nine
+// stages), the B buffers and the bookkeeping.
+constexpr int kBRegionMax = 32768;    // B buffers with 12 stages
+constexpr int kRestBytes = (kStagesMax - kLowStages) * kStageBytes + kBRegionMax + kSmemBook;
 static_assert(kLowStages * kStageBytes == (kStagesMax - kLowStages) * kStageBytes, "either half of the stages");
 constexpr size_t kSmemRequest = 1024 + 65536 + kLutBytes + kRestBytes;
 static_assert(kSmemRequest <= 232448, "shared memory per block");
@@ -365,17 +370,21 @@ struct StageMap {
         return s < kLowStages ? lo + s * kStageBytes : hi + (s - kLowStages) * kStageBytes;
     }
 };
+// the stages after the table, the B buffers and the bookkeeping fit in kRestBytes
 template <int NQ, int NH>
 constexpr bool b_fits()
 {
-    return Cfg<NQ, NH>::S * Cfg<NQ, NH>::kBBufs * Cfg<NQ, NH>::kBBytes <= kBRegion;
+    using C = Cfg<NQ, NH>;
+    return (C::kStages - kLowStages) * kStageBytes + C::kBRegion + kSmemBook <= kRestBytes && C::kBRegion % 1024 == 0;
 }
 static_assert(b_fits<4, 2>() && b_fits<8, 2>() && b_fits<4, 4>() && b_fits<8, 4>(),
               "B buffers of every stream fit");
 
 // Worker threads of tile stream g (local tiles k = 0, 1, ... are the CTA's
 // tiles t0 + g + S*k): one thread per key of a tile.
-template <int B, int NQ, int NH>
+// kAppend: the instantiation that serves the decode step (axr_append_scores);
+// plain scoring runs the one without the append code
+template <int B, int NQ, int NH, bool kAppend>
 struct Worker {
     using LK = Lookup<B>;
     using C = Cfg<NQ, NH>;
@@ -448,7 +457,7 @@ struct Worker {
             // the stages may hold its row as it was before this launch or as
             // stored here, and the thread of that key takes the row and norm
             // from shared memory instead either way
-            const bool appending = p.append_pos >= 0 && ti == (p.append_pos >> 7);
+            const bool appending = kAppend && p.append_pos >= 0 && ti == (p.append_pos >> 7);
             if (appending && !append_key<B, NH>(p, S, g, h, sync_phase)) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
                 ok = false;
@@ -580,7 +589,7 @@ struct Worker {
     }
 };
 
-template <int B, int NQ, int NH>
+template <int B, int NQ, int NH, bool kAppend>
 __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(const __grid_constant__ TcParams p)
 {
     using LK = Lookup<B>;
@@ -601,14 +610,14 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
     const uint32_t st_lo = low ? base1k : hi_pos;
     const uint32_t st_hi = low ? hi_pos : hi_pos + kLowStages * kStageBytes;
     const uint32_t b_pos = st_hi + (C::kStages - kLowStages) * kStageBytes;
-    if (b_pos + kBRegion + kSmemBook > raw + static_cast<uint32_t>(kSmemRequest)) {
+    if (b_pos + C::kBRegion + kSmemBook > raw + static_cast<uint32_t>(kSmemRequest)) {
         if (threadIdx.x == 0) atomicOr(&g_status, kErrLayout);
         return;
     }
     uint8_t *sLut = smem_raw + (lut_pos - raw);
     const StageMap<C::kStages> sm{smem_raw + (st_lo - raw), smem_raw + (st_hi - raw)};
     uint8_t *sB = smem_raw + (b_pos - raw);                          // S streams x 2 B buffers
-    Smem &S = *reinterpret_cast<Smem *>(sB + kBRegion);
+    Smem &S = *reinterpret_cast<Smem *>(sB + C::kBRegion);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -735,7 +744,7 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
         }
     } else {
         // ----------------------------------------------------------- workers
-        Worker<B, NQ, NH>::run(p, S, warp / 4, sm, sB, lut_pos, tmem, t0, t1);
+        Worker<B, NQ, NH, kAppend>::run(p, S, warp / 4, sm, sB, lut_pos, tmem, t0, t1);
     }
 
     tc_fence_before_sync();
@@ -753,10 +762,11 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
 {
     constexpr int P = kD * B / 8;             // one slice of a row: the TMA box width
     constexpr int PT = P * NH;                // the whole packed row
-    auto kernel = scores_tc_kernel<B, NQ, NH>;
+    const bool append = a.k_new != nullptr;
+    auto kernel = append ? scores_tc_kernel<B, NQ, NH, true> : scores_tc_kernel<B, NQ, NH, false>;
     const size_t smem = kSmemRequest;
-    static std::atomic<unsigned long long> smem_allowed{0};     // one bit per device
-    if (cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(kernel), smem, smem_allowed);
+    static std::atomic<unsigned long long> smem_allowed[2] = {0, 0};     // one bit per device
+    if (cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(kernel), smem, smem_allowed[append]);
         e != cudaSuccess)
         return e;
     EncodeTiledFn enc = encode_tiled();

@@ -312,8 +312,10 @@ __device__ __forceinline__ int chunk_offset(int r, int c)
 }
 
 // Worker threads of tile stream g (local tiles k = 0, 1, ... are the CTA's
-// tiles t0 + g + 4k): one thread per key of a tile.
-template <int B, int NQ>
+// tiles t0 + g + S k): one thread per key of a tile.  kAppend: the
+// instantiation that serves the decode step (axr_append_scores); plain scoring
+// runs the one without the append code.
+template <int B, int NQ, bool kAppend>
 struct Worker {
     using LK = lut::Lookup<B>;
     using C = Cfg<NQ>;
@@ -443,7 +445,7 @@ struct Worker {
             }
             // decode step: this head's last tile holds the appended key, whose row
             // the stage has only as it was before this launch
-            if (p.append_pos >= 0 && ti == (p.append_pos >> 7)) {
+            if (kAppend && p.append_pos >= 0 && ti == (p.append_pos >> 7)) {
                 float nka;
                 if (!append_key<B>(p, S, g, h, S.y[g], &nka, sync_phase)) {
                     if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
@@ -488,7 +490,7 @@ struct Worker {
     }
 };
 
-template <int B, int NQ>
+template <int B, int NQ, bool kAppend>
 __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc128_kernel(const __grid_constant__ Params p)
 {
     using C = Cfg<NQ>;
@@ -550,7 +552,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc128_kernel(cons
 
     if (threadIdx.x < C::kWorkerThreads) {
         const int g = threadIdx.x / kStreamThreads;
-        Worker<B, NQ>::run(p, S, g, stage, sB, lut_pos, tmem, t0, t1);
+        Worker<B, NQ, kAppend>::run(p, S, g, stage, sB, lut_pos, tmem, t0, t1);
     } else if (warp == C::kWarpTma) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
@@ -617,10 +619,11 @@ template <int B, int NQ>
 cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
 {
     constexpr int P = kD * B / 8;
-    auto kernel = scores_tc128_kernel<B, NQ>;
+    const bool append = a.k_new != nullptr;
+    auto kernel = append ? scores_tc128_kernel<B, NQ, true> : scores_tc128_kernel<B, NQ, false>;
     constexpr size_t smem = smem_request<B, NQ>();
-    static std::atomic<unsigned long long> smem_allowed{0};     // one bit per device
-    if (cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(kernel), smem, smem_allowed);
+    static std::atomic<unsigned long long> smem_allowed[2] = {0, 0};     // one bit per device
+    if (cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(kernel), smem, smem_allowed[append]);
         e != cudaSuccess)
         return e;
     EncodeTiledFn enc = encode_tiled();

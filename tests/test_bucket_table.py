@@ -97,19 +97,19 @@ def test_table_lookup_counts_boundaries(tables, d, b):
 @pytest.mark.parametrize("b", [1, 2, 3, 4])
 def test_packed_table_entries_count_boundaries(tables, d, b):
     """The tensor-core write kernel keeps one 32-bit word per bucket: the
-    boundary the bucket holds in u units (+inf if none) with its low 4 mantissa
+    boundary the bucket holds in u units (2 if none) with its low 4 mantissa
     bits replaced by the base code.  It compares u with that word read as a
-    float (the boundary moved by at most 15 ulp; +inf with a base is a NaN and
-    compares false) and takes the low b bits of word + (u > word).  Emulated in
-    fp32 here, that is #{i : u > t_i} for every unit coordinate u outside 1e-6
-    of a boundary."""
+    float (the boundary moved by at most 15 ulp) through the sign bit of
+    word - u, and takes the low b bits of word + that bit.  Emulated in fp32
+    here, that is #{i : u > t_i} for every unit coordinate u outside 1e-6 of a
+    boundary."""
     t = tables[(d, b)]
     _, bnd = axr.axr_make_codebook(d, b)
     nt = t["nt"]
-    tau_u = np.array([bnd[t["base"][j]] if np.isfinite(t["tau"][j]) else np.inf for j in range(nt)], np.float32)
+    tau_u = np.array([bnd[t["base"][j]] if np.isfinite(t["tau"][j]) else 2.0 for j in range(nt)], np.float32)
     words = (tau_u.view(np.uint32) & np.uint32(0xFFFFFFF0)) | t["base"][:nt].astype(np.uint32)
     # every moved boundary stays within 2.3e-7 of the true one
-    fin = np.isfinite(tau_u)
+    fin = tau_u < 2.0
     moved = words[fin].view(np.float32).astype(np.float64) - tau_u[fin].astype(np.float64)
     assert np.all(np.abs(moved) <= 2.3e-7)
     rng = np.random.default_rng(d * 10 + b + 7)
@@ -121,9 +121,10 @@ def test_packed_table_entries_count_boundaries(tables, d, b):
     j = f.view(np.uint32).astype(np.int64) - 0x4B400000
     assert j.min() >= 0 and j.max() < nt
     w = words[j]
-    with np.errstate(invalid="ignore"):
-        above = u > w.view(np.float32)
-    code = (w + above.astype(np.uint32)) & np.uint32((1 << b) - 1)
+    diff = w.view(np.float32) - u                       # fp32, exact in sign
+    above = diff.view(np.uint32) >> np.uint32(31)
+    assert np.array_equal(above == 1, u > w.view(np.float32))
+    code = (w + above) & np.uint32((1 << b) - 1)
     true = (u.astype(np.float64)[:, None] > bnd.astype(np.float64)[None, :]).sum(axis=1)
     near = np.min(np.abs(u.astype(np.float64)[:, None] - bnd.astype(np.float64)[None, :]), axis=1) < 1e-6
     assert np.all(code[~near] == true[~near])

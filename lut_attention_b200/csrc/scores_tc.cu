@@ -148,7 +148,6 @@ struct Smem {
     // stages, its per-warp sums of squares, and its packed row (+1 spare word)
     float ky[kMaxStreams][kMaxD];
     float ksum[kMaxStreams][4];
-    float knorm[kMaxStreams];
     uint32_t arow[kMaxStreams][kMaxD * kMaxBits / 32 + 1];
 };
 constexpr int kSmemBook = 10240;
@@ -263,7 +262,7 @@ __device__ bool build_b(const TcParams &p, Smem &S, int g, uint8_t *b, float *in
 // slices l.  The transform's strides 128 and 256 run inside the thread, strides
 // 1-16 as shuffles, strides 32 and 64 as one 4-point transform across the
 // stream's warps through shared memory.  Stores the codes and the norm in the
-// cache and leaves the packed row in S.arow[g] and the norm in S.knorm[g].
+// cache.
 template <int B, int NH>
 __device__ bool append_key(const TcParams &p, Smem &S, int g, int h, int &phase)
 {
@@ -330,7 +329,6 @@ __device__ bool append_key(const TcParams &p, Smem &S, int g, int h, int &phase)
         atomicOr(&S.arow[g][bit >> 5], code << (bit & 31));
         if ((bit & 31) + B > 32) atomicOr(&S.arow[g][(bit >> 5) + 1], code >> (32 - (bit & 31)));
     }
-    if (tid == 0) S.knorm[g] = nk;
     if (!stream_sync(S, g, phase)) return false;
     const int64_t row = static_cast<int64_t>(h) * p.head_stride + p.append_pos;
     uint32_t *dst = reinterpret_cast<uint32_t *>(p.idx_out + row * PT) + tid;
@@ -450,19 +448,32 @@ struct Worker {
         int inv_hc = -1;                    // head number whose query scales `inv` holds
         float inv[NQ];
 
+        if constexpr (kAppend) {
+            // decode step: before any tile, quantize the appended key of every head
+            // whose last tile (the one holding append_pos) this stream scores, and
+            // store it in the cache; then one barrier, so that every thread's
+            // stores are visible to the key's owner in the loop below
+            if (p.append_pos >= 0) {
+                const int at = p.append_pos >> 7;
+                for (int hh = (t0 + g) / p.tiles_per_head; ok && hh * p.tiles_per_head + at < t1; ++hh) {
+                    const int tile = hh * p.tiles_per_head + at;
+                    if (tile < t0 + g || (tile - t0 - g) % C::S != 0) continue;
+                    ok = append_key<B, NH>(p, S, g, hh, sync_phase);
+                }
+                ok = ok && stream_sync(S, g, sync_phase);
+                if (!ok) {
+                    if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                    t1 = t0;                   // no tiles
+                }
+            }
+        }
+
         for (int tile = t0 + g; tile < t1; tile += C::S, ++k) {
             float nk = 0.0f;
-            // decode step: this head's last tile holds the appended key.  It is
-            // quantized before the tile's stages are read (fewer registers live);
-            // the stages may hold its row as it was before this launch or as
-            // stored here, and the thread of that key takes the row and norm
-            // from shared memory instead either way
-            const bool appending = kAppend && p.append_pos >= 0 && ti == (p.append_pos >> 7);
-            if (appending && !append_key<B, NH>(p, S, g, h, sync_phase)) {
-                if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
-                ok = false;
-                break;
-            }
+            // decode step: the appended key's row and norm, which the stages may hold
+            // as they were before this launch, come from the cache for its thread
+            const bool mine = kAppend && p.append_pos >= 0 && ti == (p.append_pos >> 7) &&
+                              r == (p.append_pos & (kTileRows - 1));
 #pragma unroll 1
             for (int sl = 0; sl < NH; ++sl) {
                 const int m = k * NH + sl;      // this stream's subtile count
@@ -529,10 +540,12 @@ struct Worker {
                         }
                     }
                 }
-                if (appending && r == (p.append_pos & (kTileRows - 1))) {
+                if (mine) {
+                    const int64_t row = static_cast<int64_t>(h) * p.head_stride + p.append_pos;
+                    const uint32_t *src = reinterpret_cast<const uint32_t *>(p.idx_out + row * (P * NH)) + sl * NW;
 #pragma unroll
-                    for (int v = 0; v < NW; ++v) w[v] = S.arow[g][sl * NW + v];
-                    if (sl == 0) nk = S.knorm[g];
+                    for (int v = 0; v < NW; ++v) w[v] = AXR_IN(p.sp_idx_out, src + v, 4) ? __ldcg(src + v) : 0u;
+                    if (sl == 0) nk = AXR_IN(p.sp_norms_out, p.norms_out + row, 4) ? __ldcg(p.norms_out + row) : 0.0f;
                 }
 
                 // lookup l fills A columns l (4-byte entries) or 2l, 2l+1 (8-byte entries)

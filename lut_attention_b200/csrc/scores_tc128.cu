@@ -135,7 +135,8 @@ struct Book {
     uint64_t drain[kMaxStreams];
     uint32_t tmem_base;
     float inv[kMaxStreams][4][8];      // per stream, head number mod 4 and query: 1 / (128 S_q S_c)
-    float qmax[kMaxStreams][4][8];     // per stream, warp and query: max |q''| (append: sums of squares)
+    float qmax[kMaxStreams][4][8];     // per stream, warp and query: max |q''|
+    float ksum[kMaxStreams][4];        // per stream and warp: sum of squares of an appended key
     uint32_t arow[kMaxStreams][17];    // per stream: packed row of an appended key
     float y[kMaxStreams][kD];          // per stream: rotation scratch of an appended key
 };
@@ -269,7 +270,7 @@ __device__ bool append_key(const Params &p, Book &S, int g, int h, float *y, flo
     float ss = x * x;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if ((tid & 31) == 0) S.qmax[g][tid >> 5][0] = ss;
+    if ((tid & 31) == 0) S.ksum[g][tid >> 5] = ss;
     if (tid <= P / 4) S.arow[g][tid] = 0u;
     if (!stream_sync(S, g, phase)) return false;
     for (int hh = 1; hh < kD; hh <<= 1) {
@@ -281,7 +282,7 @@ __device__ bool append_key(const Params &p, Book &S, int g, int h, float *y, flo
         }
         if (!stream_sync(S, g, phase)) return false;
     }
-    const float nk = sqrtf((S.qmax[g][0][0] + S.qmax[g][1][0]) + (S.qmax[g][2][0] + S.qmax[g][3][0]));
+    const float nk = sqrtf((S.ksum[g][0] + S.ksum[g][1]) + (S.ksum[g][2] + S.ksum[g][3]));
     // u = y / (sqrt(d) ||k||); idx = number of boundaries below u (a zero key has
     // u = 0 and takes the central index)
     const float u = (nk > 0.0f) ? y[tid] / (sqrtf(static_cast<float>(kD)) * nk) : 0.0f;

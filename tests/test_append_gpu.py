@@ -122,3 +122,18 @@ def test_decode_step_launch_count(d, launches):
     assert len(ours) == launches, ours
     if launches == 1:
         assert "scores_tc" in ours[0], ours
+
+
+@pytest.mark.parametrize("d", [128, 256, 512])
+def test_append_on_many_single_tile_heads(d):
+    """Short caches (every head one tile): a stream rotates a head's queries and
+    quantizes its new key in the same tile, for hundreds of heads in one launch.
+    The key's sums of squares must not share scratch with the queries' maxima."""
+    b, group, heads, pos, capacity = 4, 4, 300, 50, 64
+    keys, s, idx, norms = _cache(heads, capacity, pos, d, b, "bf16", seed=d + 5)
+    wl = workloads.GQA_DECODE_128K.with_(d=d, batch=1, kv_heads=heads, group=group, T=pos + 1, seed=d + 6)
+    q = workloads.make_queries(wl, DEV)
+    out = axr.axr_append_scores(keys[:, pos].contiguous(), q, idx, norms, pos, group, b, s)
+    assert axr.axr_device_status() == 0
+    assert check_quantize(keys[:, pos], idx[:, pos], norms[:, pos], b, s).ok(flip_fraction=None)
+    assert check_scores(q, idx[:, :pos + 1].contiguous(), norms[:, :pos + 1].contiguous(), out, group, b, s) <= 1e-4

@@ -109,10 +109,13 @@ def job_scores_per_s(wl: workloads.Workload, world: int, ms_per_step: float) -> 
 def kernel_file(kind: str, wl: workloads.Workload) -> str:
     """Source file of the kernel the library runs for this workload (api.cu takes the
     tensor-core kernels at d = 128, 256 and 512, for the write path with bf16/f16 keys;
-    the read path at d = 128 has a kernel of its own)."""
+    the read path at d = 128 has a kernel of its own; AXR_READ_KERNEL=cuda_core sends
+    every read to the CUDA-core kernel)."""
     tc_width = wl.d in (128, 256, 512)
     if kind == "quantize_keys":
         return "quantize_keys_tc.cu" if tc_width and wl.dtype in ("bf16", "f16") else "quantize_keys.cu"
+    if os.environ.get("AXR_READ_KERNEL") == "cuda_core":
+        return "scores.cu"
     if wl.d == 128:
         return "scores_tc128.cu"
     return "scores_tc.cu" if tc_width else "scores.cu"
@@ -577,6 +580,7 @@ def config_dict(wl, world):
         "d": wl.d, "b": wl.b, "context": wl.T, "key_dtype": wl.dtype,
         "global_batch": wl.batch * world, "parallelism": f"shard{world}" if world > 1 else "single",
         "l2": "inputs larger than L2 (126 MB); read kernel scores the cache written one step earlier",
+        "read_kernel": "cuda_core" if os.environ.get("AXR_READ_KERNEL") == "cuda_core" else "auto",
     }
 
 
@@ -588,6 +592,9 @@ def main():
     ap.add_argument("--impl", choices=["axr", "reference"], default="axr")
     ap.add_argument("--workload", default="gqa_decode_128k", choices=sorted(workloads.BY_NAME))
     ap.add_argument("--b", type=int, default=None, help="bits per coordinate (default: the workload's)")
+    ap.add_argument("--read-kernel", choices=["auto", "cuda_core"], default="auto",
+                    help="cuda_core: run every read on the CUDA-core kernel (sets AXR_READ_KERNEL before the "
+                         "library loads), to compare it with the tensor-core read on the same workload")
     ap.add_argument("--tokens", type=int, default=None,
                     help="keys per KV head instead of the workload's context: a reduced case for profiler "
                          "captures (its line is not the workload's figure and carries no profiled traffic)")
@@ -601,6 +608,8 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
+    if args.read_kernel == "cuda_core":
+        os.environ["AXR_READ_KERNEL"] = "cuda_core"
     world, rank, local = dist_env()
     base = workloads.BY_NAME[args.workload]
     if args.b is not None:

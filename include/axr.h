@@ -27,6 +27,10 @@
  *     same one (AXELRAM abstract: the transform's sign pattern, chosen once).
  *   - Supported shapes: d a power of two in [8, 512]; b in {1, 2, 3, 4};
  *     group in [1, 8].
+ *   - The read calls run the tensor-core kernels at d = 128, 256 and 512 and the
+ *     CUDA-core kernel otherwise.  AXR_READ_KERNEL=cuda_core in the environment
+ *     (read once per process) routes every read to the CUDA-core kernel, to
+ *     compare the two; the results agree within the score tolerance.
  *
  * Packed index layout (one row per key, P = d*b/8 bytes, rows back to back):
  *   bit i of idx_j is bit (j*b + i) of the row's bit stream, and byte k of the

@@ -33,6 +33,9 @@
 // A tcgen05.mma issue blocks while the tensor pipe works, and a tile's 8
 // products take longer than its decode, so every stream has its own issuer:
 // together they keep the pipe fed while each waits for its own workers.
+#include <cstdlib>
+#include <cstring>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -864,8 +867,21 @@ cudaError_t launch_h(const ScoresArgs &a, cudaStream_t stream)
 
 }  // namespace
 
+// AXR_READ_KERNEL=cuda_core in the environment routes every read to the
+// CUDA-core kernel (scores.cu), to compare the two on the same calls; read once
+// per process.
+static bool read_forced_to_cuda_cores()
+{
+    static const bool forced = [] {
+        const char *v = std::getenv("AXR_READ_KERNEL");
+        return v != nullptr && std::strcmp(v, "cuda_core") == 0;
+    }();
+    return forced;
+}
+
 bool scores_tc_supported(const ScoresArgs &a)
 {
+    if (read_forced_to_cuda_cores()) return false;
     if (a.d == kD) return scores_tc128_supported(a);
     // d = 256 and 512 run as 2 and 4 slices of 128 coordinates
     const bool width = a.d == 2 * kD || a.d == 4 * kD;

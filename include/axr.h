@@ -135,8 +135,9 @@ int axr_scores(const void *q, int qdtype, const uint8_t *idx, const float *norms
  * capacity  keys each head's cache holds, >= 1; 0 <= pos < capacity (else AXR_EINVAL).
  * scores  device float[(heads*group) * (pos+1)] output; row h*group+g holds the
  *         pos+1 scores of that query head (row stride pos+1).
- * The two parts are enqueued on `stream` in order; the call is asynchronous like
- * the others.
+ * At d = 128, 256 and 512 both parts run in one kernel launch (the tensor-core
+ * read quantizes the new keys itself); at smaller d they are two launches,
+ * enqueued on `stream` in order.  The call is asynchronous like the others.
  */
 int axr_append_scores(const void *k_new, int kdtype, const void *q, int qdtype, uint8_t *idx,
                       float *norms, int64_t capacity, int64_t pos, int heads, int group, int d, int b,

@@ -78,6 +78,32 @@ inline void centroid_digits(const Codebook &cb, int8_t hi[kMaxLevels], int8_t lo
     }
 }
 
+// Contiguous tile ranges for the persistent CTAs of a read kernel (host): CTA c
+// scores tiles [starts[c], starts[c + 1]).  A CTA whose range crosses into a new
+// KV head rebuilds its query digits there, which the split charges as
+// change_cost tiles: the cost of the tiles before t is
+//     t + change_cost * floor(t / tiles_per_head),
+// and each CTA gets an equal share of the total cost, so CTAs with a head change
+// get fewer tiles and all end together.
+constexpr int kMaxCtas = 160;
+inline void balanced_ranges(int total_tiles, int tiles_per_head, int ctas, int change_cost, int *starts)
+{
+    const int64_t tph = tiles_per_head, cc = change_cost;
+    const int64_t total = total_tiles + cc * (total_tiles / tiles_per_head - 1);
+    starts[0] = 0;
+    for (int c = 1; c < ctas; ++c) {
+        const int64_t target = total * c / ctas;
+        // first t whose cost reaches target: inside head h (cost h (tph + cc) + r)
+        // at t = h tph + r, or at the next head's first tile if target falls
+        // into the jump at the boundary
+        const int64_t h = target / (tph + cc);
+        const int64_t r = target - h * (tph + cc);
+        const int64_t t = r < tph ? h * tph + r : (h + 1) * tph;
+        starts[c] = static_cast<int>(t < total_tiles ? t : total_tiles);
+    }
+    starts[ctas] = total_tiles;
+}
+
 __device__ __forceinline__ float load_q(const void *q, int dtype, int64_t i)
 {
     switch (dtype) {

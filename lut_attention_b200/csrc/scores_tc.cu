@@ -14,7 +14,8 @@
 // kind::i8 contraction over a tile of 128 keys and the G queries of a KV head
 // (lut_read.cuh states the digits and their error bound).
 //
-// One CTA per SM, persistent over a contiguous range of 128-key tiles, which it
+// One CTA per SM, persistent over a contiguous range of 128-key tiles (split so
+// that each CTA's tiles plus its KV-head changes cost the same), which it
 // deals round-robin to S tile streams (S = 3 for up to 4 queries per KV head,
 // else 2).  Per stream:
 //   4 worker warps : one thread per key (= tensor-memory lane).  For tile k:
@@ -120,7 +121,7 @@ struct TcParams {
     int group;
     int tiles_per_head;
     int total_tiles;
-    int tiles_per_cta;
+    int tile_start[lut::kMaxCtas + 1];   // CTA c scores tiles [tile_start[c], tile_start[c + 1])
     float inv_sc;              // 1 / (128 * S_c)
     int8_t hi[kMaxLevels];     // centroid digits
     int8_t lo[kMaxLevels];
@@ -637,8 +638,8 @@ __global__ void __launch_bounds__(Cfg<NQ, NH>::kThreads, 1) scores_tc_kernel(con
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * p.tiles_per_cta;
-    const int t1 = min(p.total_tiles, t0 + p.tiles_per_cta);
+    const int t0 = p.tile_start[blockIdx.x];
+    const int t1 = p.tile_start[blockIdx.x + 1];
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -829,9 +830,11 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
     p.idx_out = a.idx_out;
     p.norms_out = a.norms_out;
     for (int i = 0; i < kMaxLevels - 1; ++i) p.bnd[i] = a.cb.boundaries[i];
-    const int sms = device_sm_count();
+    const int sms = device_sm_count() < lut::kMaxCtas ? device_sm_count() : lut::kMaxCtas;
     const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-    p.tiles_per_cta = (p.total_tiles + grid - 1) / grid;
+    // a head change (the query rotation over d coordinates) costs a stream a few
+    // microseconds: about 12 tiles of 128 coordinates
+    lut::balanced_ranges(p.total_tiles, p.tiles_per_head, grid, 12 / NH, p.tile_start);
     lut::centroid_digits(a.cb, p.hi, p.lo, &p.inv_sc);
     AXR_DEBUG_ONLY(constexpr int D = kD * NH;
                    const uint64_t rows_q = static_cast<uint64_t>(a.heads) * a.group;
@@ -843,8 +846,7 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
                    p.sp_k_new = dbg::span(a.k_new, a.k_new ? static_cast<uint64_t>(a.heads) * D * dtype_bytes(a.kdtype) : 0);
                    p.sp_idx_out = dbg::span(a.idx_out, a.idx_out ? rows_k * PT : 0);
                    p.sp_norms_out = dbg::span(a.norms_out, a.norms_out ? rows_k * sizeof(float) : 0);)
-    const int used = (p.total_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
-    kernel<<<used, Cfg<NQ, NH>::kThreads, smem, stream>>>(p);
+    kernel<<<grid, Cfg<NQ, NH>::kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -4,8 +4,9 @@
 //
 // The lookups feed an exact int32 contraction over a tile of 128 keys and the G
 // query heads of a KV head (fixed-point digits, lut_read.cuh):
-//   * one CTA per SM, persistent over a contiguous range of 128-key tiles, dealt
-//     round-robin to S tile streams (S = 3 for up to 4 queries per KV head, 2
+//   * one CTA per SM, persistent over a contiguous range of 128-key tiles (split
+//     so that each CTA's tiles plus its KV-head changes cost the same,
+//     lut::balanced_ranges), dealt round-robin to S tile streams (S = 3 for up to 4 queries per KV head, 2
 //     for up to 8), each of 4 worker warps (one thread per key = tensor-memory
 //     lane) and one MMA warp;
 //   * one TMA warp streams every tile's packed rows and key norms into a ring of
@@ -62,7 +63,7 @@ struct Params {
     int group;
     int tiles_per_head;
     int total_tiles;
-    int tiles_per_cta;
+    int tile_start[lut::kMaxCtas + 1];   // CTA c scores tiles [tile_start[c], tile_start[c + 1])
     float inv_sc;              // 1 / (128 * S_c)
     int8_t hi[kMaxLevels];     // centroid digits
     int8_t lo[kMaxLevels];
@@ -519,8 +520,8 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc128_kernel(cons
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * p.tiles_per_cta;
-    const int t1 = min(p.total_tiles, t0 + p.tiles_per_cta);
+    const int t0 = p.tile_start[blockIdx.x];
+    const int t1 = p.tile_start[blockIdx.x + 1];
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < St::kCount; ++s) {
@@ -681,11 +682,11 @@ cudaError_t launch_bn(const ScoresArgs &a, cudaStream_t stream)
                    p.sp_k_new = dbg::span(a.k_new, a.k_new ? static_cast<uint64_t>(a.heads) * kD * dtype_bytes(a.kdtype) : 0);
                    p.sp_idx_out = dbg::span(a.idx_out, a.idx_out ? rows_k * P : 0);
                    p.sp_norms_out = dbg::span(a.norms_out, a.norms_out ? rows_k * sizeof(float) : 0);)
-    const int sms = device_sm_count();
+    const int sms = device_sm_count() < lut::kMaxCtas ? device_sm_count() : lut::kMaxCtas;
     const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-    p.tiles_per_cta = (p.total_tiles + grid - 1) / grid;
-    const int used = (p.total_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
-    kernel<<<used, Cfg<NQ>::kThreads, smem, stream>>>(p);
+    // a head change costs a stream about 4 us, some 12 tiles of a CTA's time
+    lut::balanced_ranges(p.total_tiles, p.tiles_per_head, grid, 12, p.tile_start);
+    kernel<<<grid, Cfg<NQ>::kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -164,18 +164,23 @@ __device__ __forceinline__ float join_sums(const uint32_t *x)
 }
 
 // Table entry of one field value: C hi digits then C lo digits, replicated for
-// the 32 lanes (entry (field, lane) at field * 256 + lane * EB), written as
-// 32-bit words.
+// the 32 lanes (entry (field, lane) at field * 256 + lane * EB).  One thread
+// per (row, table) forms the entry once and writes its 32 copies as 16-byte
+// chunks (4 or 2 copies each), starting at a chunk that rotates with the row so
+// that the threads of a warp spread their stores over all banks.
 template <int B>
 __device__ void build_lut(const int8_t *hi, const int8_t *lo, uint8_t *lut, int tid, int nthreads)
 {
     using LK = Lookup<B>;
     constexpr uint32_t mask = (1u << B) - 1u;
     constexpr int kTables = LK::kByteTables ? 2 : 1;
-    for (int e = tid; e < LK::kRows * 32 * kTables; e += nthreads) {
-        const int row = e / (32 * kTables), ln = e % 32, tab = (e / 32) % kTables;
+    constexpr int kChunks = 32 * LK::EB / 16;       // 16-byte chunks of one row of one table
+    static_assert(LK::EB == 4 || LK::EB == 8, "entries of one or two words");
+    static_assert(kTables * 32 * LK::EB <= 256, "a row holds every table's 32 entries");
+    for (int e = tid; e < LK::kRows * kTables; e += nthreads) {
+        const int row = e / kTables, tab = e % kTables;
         const int field = LK::kByteTables ? ((tab == 0) ? (row & (LK::NF - 1)) : (row >> 2)) : row;
-        uint32_t words[LK::EB / 4] = {};
+        uint32_t words[2] = {0u, 0u};
 #pragma unroll
         for (int i = 0; i < LK::C; ++i) {
             const int code = (field >> (B * i)) & mask;
@@ -183,9 +188,14 @@ __device__ void build_lut(const int8_t *hi, const int8_t *lo, uint8_t *lut, int 
             words[bh / 4] |= static_cast<uint32_t>(static_cast<uint8_t>(hi[code])) << (8 * (bh % 4));
             words[bl / 4] |= static_cast<uint32_t>(static_cast<uint8_t>(lo[code])) << (8 * (bl % 4));
         }
-        uint32_t *dst = reinterpret_cast<uint32_t *>(lut + row * 256 + tab * 128 + ln * LK::EB);
+        const uint4 v = (LK::EB == 4) ? make_uint4(words[0], words[0], words[0], words[0])
+                                      : make_uint4(words[0], words[1], words[0], words[1]);
+        uint8_t *dst = lut + row * 256 + tab * 128;
 #pragma unroll
-        for (int i = 0; i < LK::EB / 4; ++i) dst[i] = words[i];
+        for (int c = 0; c < kChunks; ++c) {
+            const int j = (c + e) & (kChunks - 1);
+            *reinterpret_cast<uint4 *>(dst + 16 * j) = v;
+        }
     }
 }
 

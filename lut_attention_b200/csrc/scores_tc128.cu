@@ -168,28 +168,36 @@ __device__ __forceinline__ bool stream_sync(Book &S, int g, int &phase)
     return __all_sync(0xffffffffu, ok) != 0;
 }
 
-// Rotate the G queries of KV head h and write their digits into the stream's
-// B buffer b (thread j of the stream owns coordinate j of every query), and
-// each query's score scale 1 / (128 S_q S_c) into inv[] (every thread writes
-// the same values, so each reads back its own).  The Walsh-Hadamard transform
-// runs its strides 1-16 with shuffles and its strides 32 and 64 as one 4-point
-// transform across the stream's warps, through the B buffer (free: its last
-// products are done; every read of it precedes the barrier before the digits
-// are written).
-template <int B, int NQ>
-__device__ bool build_b(const Params &p, Book &S, int g, uint8_t *b, int h, float *inv, int &phase)
+// This thread's coordinate (its index in the stream) of the G queries of KV
+// head h, times the sign pattern D unless the keys were written with the block
+// rotation; 0 for the padding queries past the group.
+template <int NQ>
+__device__ __forceinline__ void load_queries(const Params &p, int h, float (&qq)[NQ])
 {
     const int tid = threadIdx.x & (kStreamThreads - 1);
-    const int lane = tid & 31, wq = tid >> 5;
     const float sg = (p.quats || !AXR_IN(p.sp_signs, p.signs + tid, 1) || p.signs[tid] >= 0) ? 1.0f : -1.0f;
     [[maybe_unused]] const int qb = dtype_bytes(p.qdtype);
-    float qq[NQ];
 #pragma unroll
     for (int qi = 0; qi < NQ; ++qi) {
         const int64_t at = (static_cast<int64_t>(h) * p.group + qi) * kD + tid;
         qq[qi] = (qi < p.group && AXR_IN(p.sp_q, static_cast<const char *>(p.q) + at * qb, qb))
                      ? sg * lut::load_q(p.q, p.qdtype, at) : 0.0f;
     }
+}
+
+// Rotate the G queries qq (as load_queries gives them) and write their digits
+// into the stream's B buffer b (thread j of the stream owns coordinate j of
+// every query), and each query's score scale 1 / (128 S_q S_c) into inv[]
+// (every thread writes the same values, so each reads back its own).  The
+// Walsh-Hadamard transform runs its strides 1-16 with shuffles and its strides
+// 32 and 64 as one 4-point transform across the stream's warps, through the B
+// buffer (free: its last products are done; every read of it precedes the
+// barrier before the digits are written).
+template <int B, int NQ>
+__device__ bool build_b(const Params &p, Book &S, int g, uint8_t *b, float (&qq)[NQ], float *inv, int &phase)
+{
+    const int tid = threadIdx.x & (kStreamThreads - 1);
+    const int lane = tid & 31, wq = tid >> 5;
     if (p.quats) {
         // q'' = T q / sqrt(d): the IsoQuant block rotation times the temperature;
         // the 4 coordinates of a block sit in 4 consecutive lanes
@@ -374,6 +382,11 @@ struct Worker {
         }
     }
 
+    // On entering a KV head (the first one too) the stream writes the head's
+    // query digits before it waits for the tile's stage.  The first head's
+    // queries were loaded before the CTA's set-up (so that their latency
+    // overlaps it) and wait in the B buffer, this thread's coordinate of query i
+    // at float i * 128 + (thread in stream).
     static __device__ void run(const Params &p, Book &S, int g, const StageMap<B> &stage, uint8_t *sB,
                                uint32_t lut_base, uint32_t tmem, int t0, int t1)
     {
@@ -397,6 +410,28 @@ struct Worker {
         uint32_t sph = 0;
         int k = 0;
         for (; tile < t1; tile += C::S, ++k) {
+            const int ab = k & 1;
+            if (h != prev_h) {
+                // one B buffer: the products of tile k - 1 (the last to read it) must be done
+                if (k >= 1 && !mbar_wait_warp(smem_u32(&S.mma_done[g][ab ^ 1]), ((k - 1) >> 1) & 1)) {
+                    if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
+                    return;
+                }
+                tc_fence_after_sync();
+                prev_h = h;
+                ++hc;
+                float qq[NQ];
+                if (k == 0) {
+#pragma unroll
+                    for (int qi = 0; qi < NQ; ++qi) qq[qi] = reinterpret_cast<const float *>(b)[qi * kD + r];
+                } else {
+                    load_queries<NQ>(p, h, qq);
+                }
+                if (!build_b<B, NQ>(p, S, g, b, qq, S.inv[g][hc & 3], sync_phase)) {
+                    if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
+                    return;
+                }
+            }
             if (!mbar_wait_warp(smem_u32(&S.full[s]), sph)) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutLoad);
                 return;
@@ -424,27 +459,12 @@ struct Worker {
             }
             // the products of tile k - 2 are done: its A buffer is free, and its D
             // buffer holds its sums
-            const int ab = k & 1;
             if (!mbar_wait_warp(smem_u32(&S.mma_done[g][ab]), ((k >> 1) & 1) ^ 1)) {
                 if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
                 return;
             }
             tc_fence_after_sync();
             if (k >= 2) emit(p, S, g, tl + C::kDOff + (2 * g + ab) * C::N, h2, ti2, r, nk2, hc2, inv_hc, inv);
-            if (h != prev_h) {
-                // one B buffer: the products of tile k - 1 (the last to read it) must be done
-                if (k >= 1 && !mbar_wait_warp(smem_u32(&S.mma_done[g][ab ^ 1]), ((k - 1) >> 1) & 1)) {
-                    if (lane == 0) atomicOr(&g_status, kErrTimeoutMma);
-                    return;
-                }
-                tc_fence_after_sync();
-                prev_h = h;
-                ++hc;
-                if (!build_b<B, NQ>(p, S, g, b, h, S.inv[g][hc & 3], sync_phase)) {
-                    if (lane == 0) atomicOr(&g_status, kErrTimeoutDrain);
-                    return;
-                }
-            }
             // decode step: this head's last tile holds the appended key, whose row
             // the stage has only as it was before this launch
             if (kAppend && p.append_pos >= 0 && ti == (p.append_pos >> 7)) {
@@ -522,6 +542,12 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc128_kernel(cons
     const int lane = threadIdx.x & 31;
     const int t0 = p.tile_start[blockIdx.x];
     const int t1 = p.tile_start[blockIdx.x + 1];
+    // the worker threads' coordinates of their first KV head's queries, loaded
+    // now and left in their stream's B buffer after the set-up
+    float q0[NQ];
+    const int first_tile = t0 + static_cast<int>(threadIdx.x / kStreamThreads);
+    const bool has_first = threadIdx.x < C::kWorkerThreads && first_tile < t1;
+    if (has_first) load_queries<NQ>(p, first_tile / p.tiles_per_head, q0);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < St::kCount; ++s) {
@@ -543,6 +569,11 @@ __global__ void __launch_bounds__(Cfg<NQ>::kThreads, 1) scores_tc128_kernel(cons
         prefetch_tensormap(&p.nmap);
     }
     lut::build_lut<B>(p.hi, p.lo, sLut, threadIdx.x, C::kThreads);
+    if (has_first) {
+        float *x = reinterpret_cast<float *>(sB + (threadIdx.x / kStreamThreads) * C::kBBytes);
+#pragma unroll
+        for (int qi = 0; qi < NQ; ++qi) x[qi * kD + (threadIdx.x & (kStreamThreads - 1))] = q0[qi];
+    }
     if (warp == 0) {
         tmem_alloc(smem_u32(&S.tmem_base), kTmemCols);
         tmem_relinquish();

@@ -167,9 +167,10 @@ __device__ __forceinline__ float join_sums(const uint32_t *x)
 // the 32 lanes (entry (field, lane) at field * 256 + lane * EB).  One thread
 // per (row, table) forms the entry once and writes its 32 copies as 16-byte
 // chunks (4 or 2 copies each), starting at a chunk that rotates with the row so
-// that the threads of a warp spread their stores over all banks.
+// that the threads of a warp spread their stores over all banks.  Also built as
+// host code, so that a CPU test can check the table against its definition.
 template <int B>
-__device__ void build_lut(const int8_t *hi, const int8_t *lo, uint8_t *lut, int tid, int nthreads)
+__host__ __device__ void build_lut(const int8_t *hi, const int8_t *lo, uint8_t *lut, int tid, int nthreads)
 {
     using LK = Lookup<B>;
     constexpr uint32_t mask = (1u << B) - 1u;
